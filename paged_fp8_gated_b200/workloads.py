@@ -1,0 +1,177 @@
+"""Seeded synthetic inputs for one attention step (decode or verify block).
+
+This module only draws random inputs with the shapes, value distributions and
+paging structure of the loads on the task page "Gated attention decode
+(muse_attention_decode)" (sections "Shapes" and the load table).  It holds
+none of the attention arithmetic: the pre-existing cache contents are shaped
+with torch's own normalisation and float8 cast, which are distribution
+recipes, not steps of the method.  Both the CUDA path and the oracle consume
+what it returns.
+
+Layouts (all torch CPU tensors):
+  qkv        bf16  [T, 2304]  q 16x64 | k 2x64 | v 2x64 | gate 16x64, T = B*L
+  positions  int64 [T]        seq_lens[b] + j for token t = b*L + j
+  seq_lens   int32 [B]        tokens cached before this step
+  page_table int32 [B, max_pages]
+  cache_loc  int64 [T]        cache row (page*page_size + slot) of token t
+  k_cache    uint8 [num_pages, page_size, 2, 64]   E4M3 codes
+  v_cache    uint8 [num_pages, page_size, 2, 64]
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+HQ, HKV, D = 16, 2, 64
+QKV_COLS = HQ * D + 2 * HKV * D + HQ * D  # 2304
+GATE_OFF = HQ * D + 2 * HKV * D           # 1280
+ROW_BYTES = HKV * D                       # 128
+
+
+@dataclass
+class Spec:
+    """One synthetic step.  ``seq_lens`` may be a list, or None with ``ctx``
+    (all requests at ``ctx``) or ``ctx_range`` (uniform integers, inclusive)."""
+    name: str
+    B: int
+    L: int = 1
+    ctx: int | None = None
+    ctx_range: tuple[int, int] | None = None
+    seq_lens: list[int] | None = None
+    window: int = 0            # > 0: sliding window; 0: full attention
+    use_rope: bool = False
+    page_size: int = 1
+    permute: bool = True       # shuffle page ids over the pool
+    kv_scale: float = 1.0
+    gate_std: float = 1.0
+    seed: int = 0
+    spare_pages: int = 0       # unused pages in the pool
+    extra: dict = field(default_factory=dict)
+
+
+def _unit_rms(x: torch.Tensor) -> torch.Tensor:
+    return x * torch.rsqrt(x.pow(2).mean(-1, keepdim=True) + 1e-6)
+
+
+def _to_e4m3_codes(x: torch.Tensor) -> torch.Tensor:
+    return x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def resolve_seq_lens(spec: Spec, gen: torch.Generator) -> np.ndarray:
+    if spec.seq_lens is not None:
+        s = np.asarray(spec.seq_lens, dtype=np.int64)
+    elif spec.ctx_range is not None:
+        lo, hi = spec.ctx_range
+        s = torch.randint(lo, hi + 1, (spec.B,), generator=gen).numpy().astype(np.int64)
+    else:
+        s = np.full(spec.B, int(spec.ctx), dtype=np.int64)
+    assert s.shape == (spec.B,) and (s >= 0).all()
+    return s
+
+
+def make_inputs(spec: Spec) -> dict:
+    """Draw one step's inputs.  Deterministic in ``spec`` (including its seed)."""
+    gen = torch.Generator().manual_seed(int(spec.seed))
+    B, L, ps = spec.B, spec.L, spec.page_size
+    T = B * L
+    seq = resolve_seq_lens(spec, gen)
+    total = seq + L                                   # keys per request after the append
+    pages_per_req = (total + ps - 1) // ps
+    n_pages = int(pages_per_req.sum()) + int(spec.spare_pages)
+    max_pages = int(pages_per_req.max())
+    max_pages = (max_pages + 3) // 4 * 4              # 16-byte row pitch for the page table
+
+    if spec.permute:
+        pool = torch.randperm(n_pages, generator=gen).numpy().astype(np.int64)
+    else:
+        pool = np.arange(n_pages, dtype=np.int64)
+    page_table = np.zeros((B, max_pages), dtype=np.int32)
+    off = 0
+    for b in range(B):
+        n = int(pages_per_req[b])
+        page_table[b, :n] = pool[off:off + n]
+        off += n
+
+    positions = (seq[:, None] + np.arange(L)[None, :]).reshape(-1).astype(np.int64)
+    b_of_t = np.repeat(np.arange(B), L)
+    cache_loc = (page_table[b_of_t, positions // ps].astype(np.int64) * ps + positions % ps)
+
+    qkv = torch.randn(T, QKV_COLS, generator=gen)
+    if spec.gate_std != 1.0:
+        qkv[:, GATE_OFF:] *= spec.gate_std
+    qkv = qkv.to(torch.bfloat16)
+
+    # Pre-existing cache: K = E4M3(unit-RMS N(0,1) / scale), V = E4M3(N(0,1) / scale),
+    # drawn for every slot of the pool (including the rows this step overwrites).
+    rows = n_pages * ps
+    k_cache = torch.empty(rows, HKV, D, dtype=torch.uint8)
+    v_cache = torch.empty(rows, HKV, D, dtype=torch.uint8)
+    chunk = 1 << 20
+    inv = 1.0 / float(spec.kv_scale)
+    for r0 in range(0, rows, chunk):
+        r1 = min(rows, r0 + chunk)
+        kx = _unit_rms(torch.randn(r1 - r0, HKV, D, generator=gen))
+        vx = torch.randn(r1 - r0, HKV, D, generator=gen)
+        k_cache[r0:r1] = _to_e4m3_codes(kx * inv)
+        v_cache[r0:r1] = _to_e4m3_codes(vx * inv)
+
+    return dict(
+        name=spec.name,
+        B=B, L=L, page_size=ps, window=int(spec.window), use_rope=bool(spec.use_rope),
+        k_scale=float(spec.kv_scale), v_scale=float(spec.kv_scale),
+        qkv=qkv,
+        positions=torch.from_numpy(positions),
+        seq_lens=torch.from_numpy(seq.astype(np.int32)),
+        page_table=torch.from_numpy(page_table),
+        cache_loc=torch.from_numpy(cache_loc),
+        k_cache=k_cache.view(n_pages, ps, HKV, D),
+        v_cache=v_cache.view(n_pages, ps, HKV, D),
+    )
+
+
+def keys_attended(inp: dict) -> int:
+    """Distinct cache rows the step reads: sum over requests of the union of
+    its tokens' key ranges (full: p_last + 1; sliding: at most W + L - 1)."""
+    pos = inp["positions"].numpy().reshape(inp["B"], inp["L"])
+    last = pos[:, -1]
+    first = pos[:, 0]
+    W = inp["window"]
+    lo = np.maximum(0, first - W + 1) if W > 0 else np.zeros_like(first)
+    return int((last - lo + 1).sum())
+
+
+# ----------------------------------------------------------------------------
+# The page's loads (section "Shapes" and the load table), at the sizes used here
+# ----------------------------------------------------------------------------
+
+def named(name: str, seed: int = 0) -> Spec:
+    """The standard synthetic steps.  Seed 0 for all, mixed with a per-step offset."""
+    specs = {
+        # one request, 4096 cached keys + 1 new, full attention, identity pages
+        "pr1": Spec("pr1", B=1, L=1, ctx=4096, permute=False, seed=seed),
+        # one request at 80,000 cached keys, sliding (window 2048, RoPE) or full
+        "decode1_sliding": Spec("decode1_sliding", B=1, L=1, ctx=80000, window=2048,
+                                use_rope=True, seed=seed + 11),
+        "decode1_full": Spec("decode1_full", B=1, L=1, ctx=80000, seed=seed + 12),
+        # 32 requests, contexts uniform in [40000, 80000], permuted page-1 table
+        "decode32_full": Spec("decode32_full", B=32, L=1, ctx_range=(40000, 80000),
+                              seed=seed + 2),
+        "decode32_sliding": Spec("decode32_sliding", B=32, L=1, ctx_range=(40000, 80000),
+                                 window=2048, use_rope=True, seed=seed + 21),
+        # 16 requests, 8-token causal verify blocks at 80,000 cached keys
+        "verify16_sliding": Spec("verify16_sliding", B=16, L=8, ctx=80000, window=2048,
+                                 use_rope=True, seed=seed + 31),
+        "verify16_full": Spec("verify16_full", B=16, L=8, ctx=80000, seed=seed + 32),
+        # 64-token pages with shuffled ids, cache scale 1/64, gate N(0, 4)
+        "paged_full": Spec("paged_full", B=4, L=8, ctx=65536, page_size=64, kv_scale=1 / 64,
+                           gate_std=2.0, seed=seed + 41),
+        "paged_sliding": Spec("paged_sliding", B=4, L=8, ctx=65536, page_size=64, window=2048,
+                              use_rope=True, kv_scale=1 / 64, gate_std=2.0, seed=seed + 42),
+    }
+    return specs[name]
+
+
+NAMED = ["pr1", "decode1_sliding", "decode1_full", "decode32_full", "decode32_sliding",
+         "verify16_sliding", "verify16_full", "paged_full", "paged_sliding"]
