@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Benchmark of one attention step of paged FP8 gated attention decode.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path (prep -> split-KV decode -> combine
+with the gated output norm) over one seeded synthetic batch, replayed as a
+CUDA graph with a cold L2 before every step.  Default workload: 32 requests,
+contexts uniform in [40000, 80000], full attention, page size 1 with a
+permuted page table (KV cache about 491 MB, larger than L2).
+
+Prints one JSON line (rank 0).  `value` is the whole-job KV-cache bandwidth
+(GB/s) and `ms_per_step` the step time; `roofline` reports the decode kernel's
+algorithmic bytes over its own CUDA-event time against the measured HBM copy
+bandwidth; `cpu_baseline` times the CPU oracle (rank 0, N=1 only).
+
+With N > 1 (torchrun) every rank runs an independent replica of the step on
+its own GPU: the op has no cross-GPU exchange ("replicas only"), so scaling
+is weak and the job value is the sum of the ranks' KV bytes over the slowest
+rank's time.
+
+--impl reference times the CPU oracle itself as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "µs/step and KV-cache GB/s (% of HBM roofline), decode-32 full-attn ctx 80K"
+BYTES_PER_KEY = 256          # K and V rows: 2 KV heads x 64 E4M3 codes each
+PT_BYTES_PER_KEY = {1: 4, 64: 4 / 64}   # page-table bytes read per key
+FALLBACK_HBM_GBS = 6650.0
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one decode-kernel launch on the
+# default workload, from the ncu capture summarised in profiles/, keyed by the
+# hash of the kernel sources it was taken on (null once the sources change).
+TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "paged_fp8_gated_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_cpu_rate(inp: dict, max_key_heads: float = 40e6) -> dict:
+    """Time the CPU oracle on a bounded prefix of the step's requests (all heads
+    and tokens of each); returns KV-cache GB/s over that sample."""
+    import numpy as np
+    import torch
+    from oracle import oracle as O
+    from paged_fp8_gated_b200 import workloads as W
+
+    B, L = inp["B"], inp["L"]
+    pos = inp["positions"].numpy().reshape(B, L)
+    W_ = inp["window"]
+    keys = []
+    for b in range(B):
+        lo = max(0, int(pos[b, 0]) - W_ + 1) if W_ > 0 else 0
+        keys.append(int(pos[b, -1]) - lo + 1)
+    nb, kh = 0, 0.0
+    while nb < B and (nb == 0 or kh + keys[nb] * 16 * L <= max_key_heads):
+        kh += keys[nb] * 16 * L
+        nb += 1
+    T = nb * L
+    qkv = inp["qkv"][:T].view(torch.int16).numpy().astype(np.uint16)
+    threads = os.cpu_count() or 1
+    t = time.perf_counter()
+    O.attn_decode(qkv, inp["positions"][:T], inp["page_table"][:nb], inp["cache_loc"][:T],
+                  inp["k_cache"].reshape(-1, 128), inp["v_cache"].reshape(-1, 128),
+                  inp["k_scale"], inp["v_scale"], inp["page_size"], inp["window"],
+                  inp["use_rope"], nthreads=threads)
+    dt = time.perf_counter() - t
+    kv = sum(keys[:nb]) * BYTES_PER_KEY
+    return {"value": kv / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "seconds": dt,
+            "sample": f"requests 0..{nb - 1} of {B} ({sum(keys[:nb])} keys, all 16 heads x {L} "
+                      f"tokens), FP64 C oracle incl. its cache copy"}
+
+
+def run_reference(args, rank: int, world: int):
+    """Reference arm: the CPU oracle on this machine's host cores."""
+    if rank != 0:
+        return
+    from paged_fp8_gated_b200 import workloads as W
+    inp = W.make_inputs(W.named(args.workload))
+    budget = 150.0 / max(1, args.steps + args.warmup)   # seconds of CPU work per step
+    # size the per-step sample from one probe run
+    probe = oracle_cpu_rate(inp, max_key_heads=2e6)
+    rate_kh = 2e6 / max(probe["seconds"], 1e-3)
+    max_kh = max(2e6, min(40e6, rate_kh * budget))
+    vals, secs = [], []
+    for i in range(args.warmup + args.steps):
+        r = oracle_cpu_rate(inp, max_key_heads=max_kh)
+        if i >= args.warmup:
+            vals.append(r["value"])
+            secs.append(r["seconds"])
+    v = statistics.median(vals)
+    kv_bytes = W.keys_attended(inp) * BYTES_PER_KEY
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(kv_bytes / (v * 1e9) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B": inp["B"], "L": inp["L"],
+                   "page_size": inp["page_size"], "window": inp["window"],
+                   "note": "ms_per_step extrapolated from the sample's GB/s to the whole step"},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": r["cores"],
+                         "kind": "oracle", "sample": r["sample"]},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode32_full")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from paged_fp8_gated_b200 import binding
+    from paged_fp8_gated_b200 import workloads as W
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    spec = W.named(args.workload, seed=1000 * rank)
+    inp = W.make_inputs(spec)
+    B, L, ps = inp["B"], inp["L"], inp["page_size"]
+    T = B * L
+    keys = W.keys_attended(inp)
+    kv_bytes = keys * BYTES_PER_KEY
+    alg_bytes = keys * (BYTES_PER_KEY + PT_BYTES_PER_KEY[ps])   # decode kernel, per launch
+
+    d = {k: inp[k].to(dev) for k in ("qkv", "positions", "seq_lens", "page_table", "cache_loc",
+                                       "k_cache", "v_cache")}
+    k_scale = torch.tensor([inp["k_scale"]], dtype=torch.float32, device=dev)
+    v_scale = torch.tensor([inp["v_scale"]], dtype=torch.float32, device=dev)
+    out = torch.empty(B, L, 1024, dtype=torch.bfloat16, device=dev)
+    ws = binding.alloc_workspace(B, L, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # 256 MiB > 126 MB L2
+    flush_sink = torch.empty((), dtype=torch.int64, device=dev)
+
+    def step(events=None):
+        binding.attn_decode(d["qkv"], d["positions"], d["seq_lens"], d["page_table"],
+                            d["cache_loc"], d["k_cache"], d["v_cache"], k_scale, v_scale, ps,
+                            inp["window"], inp["use_rope"], L=L, out=out, workspace=ws,
+                            events=events)
+
+    def cold_l2():
+        flush.fill_(1)                                     # write > L2 ...
+        torch.sum(flush.view(torch.int64), dim=0, out=flush_sink)  # ... then read it back clean
+
+    # capture one step as a CUDA graph (the way a serving loop replays it)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        step()
+    side.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        step()
+    torch.cuda.synchronize(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---- device-timed steps: graph replay, cold L2 before each ----
+    for _ in range(args.warmup):
+        cold_l2()
+        graph.replay()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    wall0 = time.perf_counter()
+    for s_ev, e_ev in evs:
+        cold_l2()
+        s_ev.record()
+        graph.replay()
+        e_ev.record()
+    torch.cuda.synchronize(dev)
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    barrier()
+    step_ms = [s.elapsed_time(e) for s, e in evs]
+    mean_ms = max_over_ranks(statistics.mean(step_ms))
+    median_ms = max_over_ranks(statistics.median(step_ms))
+
+    # ---- per-kernel device times (profiling entry point, kernels serialised) ----
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for _ in range(3):
+        cold_l2()
+        step(events=kev[0])
+    torch.cuda.synchronize(dev)
+    for ev in kev:
+        cold_l2()
+        step(events=ev)
+    torch.cuda.synchronize(dev)
+    prep_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in kev)
+    dec_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in kev))
+    comb_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in kev)
+
+    # ---- end to end through the public API from pinned host buffers ----
+    host = {k: inp[k].pin_memory() for k in ("qkv", "positions", "seq_lens", "page_table",
+                                              "cache_loc")}
+    out_host = torch.empty(B, L, 1024, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k, t in host.items():
+            d[k].copy_(t, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        cold_l2()
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for s_ev, e_ev in eev:
+        cold_l2()
+        s_ev.record()
+        e2e_step()
+        e_ev.record()
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(statistics.mean(s.elapsed_time(e) for s, e in eev))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_cpu_rate(inp)
+        cpu.pop("seconds", None)
+        cpu["value"] = round(cpu["value"], 4)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = measured_peaks()
+    achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
+    traffic = TRAFFIC.get((args.workload, kernel_source_hash()))
+    line = {
+        "metric": METRIC,
+        "value": round(world * kv_bytes / (mean_ms * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(mean_ms, 5),
+        "us_per_step": round(mean_ms * 1e3, 2),
+        "us_per_step_median": round(median_ms * 1e3, 2),
+        "hbm_frac_step": round(kv_bytes / (mean_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3 cache, f16 MMA / f32 accumulate, bf16 out",
+        "data": "synthetic",
+        "config": {
+            "workload": args.workload, "B": B, "L": L, "page_size": ps,
+            "window": inp["window"], "use_rope": inp["use_rope"],
+            "keys_attended": keys, "kv_bytes_per_step": kv_bytes,
+            "parallelism": f"replicas x{world}",
+            "l2": "256 MiB write+read before every timed step; KV (per step) also exceeds L2",
+            "timing": "CUDA-graph replay of the 3-kernel step, per-step CUDA events",
+        },
+        "roofline": {
+            "kernel": "decode_kernel", "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": int(alg_bytes),
+            "kernel_us": round(dec_ms * 1e3, 2),
+            "prep_us": round(prep_ms * 1e3, 2), "combine_us": round(comb_ms * 1e3, 2),
+        },
+        "e2e": {"value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "us_per_step": round(e2e_ms * 1e3, 2),
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+        "wall_s_timed_region": round(wall, 4),
+        "cpu_baseline": cpu,
+        "kernel_sources": kernel_source_hash(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

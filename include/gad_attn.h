@@ -1,0 +1,143 @@
+/*
+ * gad_attn.h - C ABI of the paged FP8 gated attention decode library
+ * (libgad_attn.so, hand-written CUDA for sm_100a).
+ *
+ * One call runs one decode step (q_len 1) or one causal verify block
+ * (q_len <= 8) of gated grouped-query attention over a paged FP8 E4M3 KV
+ * cache, as defined on the task page "Gated attention decode
+ * (muse_attention_decode)", section "What to compute":
+ *
+ *   q, k, v, gate = split(qkv[t])
+ *   q = rmsnorm(q) * 5.473 ; k = rmsnorm(k)           per 64-wide head
+ *   q, k = rope(q, p), rope(k, p)                      when use_rope != 0
+ *   cache[cache_loc[t]] = fp8(k), fp8(v)               E4M3, scaled
+ *   a = softmax(q . K^T / 8) . V                       keys up to p (window or all)
+ *   out = rmsnorm(a) * sigmoid(gate)                   bf16
+ *
+ * Model shape (section "Shapes"): 16 query heads, 2 KV heads, head dim 64;
+ * query head h reads KV head h / 8.  Readings of points the page leaves open:
+ * rmsnorm eps 1e-6 with unit weights; RoPE is the NeoX half-split rotation of
+ * dims (i, i+32) by p * 10000^(-2i/64); a sliding window W attends keys i with
+ * p - W < i <= p; stored code = E4M3(x / scale) with round-to-nearest-even and
+ * saturation to +-448, dequantised value = code * scale.
+ *
+ * All pointers are DEVICE pointers unless stated.  All buffers belong to the
+ * caller; the library keeps no state between calls except per-device launch
+ * settings.  Calls are asynchronous on `stream`, never synchronise the host,
+ * never read device values on the host and never allocate, so they can be
+ * captured in a CUDA graph.
+ */
+#ifndef GAD_ATTN_H
+#define GAD_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Fixed model shape. */
+#define GAD_HQ 16          /* query heads per GPU            */
+#define GAD_HKV 2          /* key/value heads per GPU        */
+#define GAD_HEAD_DIM 64
+#define GAD_QKV_COLS 2304  /* q 16x64 | k 2x64 | v 2x64 | gate 16x64 */
+#define GAD_OUT_COLS 1024  /* 16 heads x 64                  */
+#define GAD_ROW_BYTES 128  /* one cache row: 2 KV heads x 64 E4M3 codes */
+#define GAD_MAX_L 8        /* longest verify block           */
+#define GAD_MAX_B 4096     /* most requests in one call      */
+
+/* Return codes (0 = success). */
+typedef enum {
+    GAD_OK = 0,
+    GAD_ERR_NULL = -1,        /* a required pointer is NULL                     */
+    GAD_ERR_SHAPE = -2,       /* B, L, max_pages or num_rows out of range       */
+    GAD_ERR_ALIGN = -3,       /* a pointer is not aligned as documented         */
+    GAD_ERR_UNSUPPORTED = -4, /* page_size not 1 or 64, or window < 0           */
+    GAD_ERR_WORKSPACE = -5,   /* workspace NULL or smaller than required        */
+    GAD_ERR_CUDA = -6,        /* a CUDA call or kernel launch failed            */
+    GAD_ERR_DEVICE = -7       /* current device is not compute capability 10.x  */
+} gad_status;
+
+/*
+ * Bytes of device workspace that gad_attn_decode needs for B requests of L
+ * tokens on the CURRENT device (it depends on the device's SM count).
+ * Returns 0 and sets gad_last_error() when B or L is out of range or no CUDA
+ * device is present.  Host-only; launches nothing.
+ */
+size_t gad_attn_workspace_bytes(int B, int L);
+
+/*
+ * One step.  T = B * L tokens; token t = b * L + j is token j of request b.
+ *
+ *   qkv         bf16 [T, 2304], row-major, 16-byte aligned.  Columns:
+ *               q heads [0,1024), k heads [1024,1152), v heads [1152,1280),
+ *               gate [1280,2304); each head 64 contiguous values.
+ *   positions   int64 [T]: position p of each token.  Token t attends the
+ *               cache keys i with lo <= i <= p, lo = 0 (window == 0) or
+ *               max(0, p - window + 1).  Contract: p = seq_lens[b] + j.
+ *   seq_lens    int32 [B]: keys cached before this step (the serving stack's
+ *               lengths).  Accepted for interface compatibility; the ranges
+ *               come from `positions`.  May be NULL.
+ *   page_table  int32 [B, max_pages], row-major: cache row of key i of request
+ *               b is page_table[b][i / page_size] * page_size + i % page_size.
+ *   cache_loc   int64 [T]: the cache row receiving token t's k and v.
+ *               Contract: cache_loc[t] is the row of key positions[t], and no
+ *               request reads a row that another token of this step writes
+ *               (except its own block's new keys).
+ *   k_cache,    uint8 [num_rows, 2, 64] E4M3 codes, 16-byte aligned, with
+ *   v_cache     num_rows = num_pages * page_size.  Rows cache_loc[t] are
+ *               overwritten; no other byte is written.
+ *   k_scale,    float32 [1] each (device): the caches' dequantisation scales.
+ *   v_scale
+ *   page_size   1 or 64.
+ *   window      > 0: sliding window of that many keys; 0: full attention.
+ *   use_rope    nonzero: rotate q and k by their position.
+ *   out         bf16 [T, 1024], row-major, 16-byte aligned.
+ *   workspace   device scratch of at least gad_attn_workspace_bytes(B, L)
+ *               bytes, 256-byte aligned, owned by the caller; its contents on
+ *               entry do not matter.  Calls that overlap on the GPU must use
+ *               different workspaces.
+ *   stream      a cudaStream_t (NULL = legacy default stream).
+ *
+ * Errors: argument checks run on the host before any launch; on failure the
+ * call launches nothing and returns a negative gad_status.  Device VALUES
+ * (positions, page_table, cache_loc) are not checked against the contract:
+ * keys whose page index falls outside the page-table row, and rows outside
+ * [0, num_rows), are read as zeros and never written, so a contract
+ * violation gives wrong numbers but no out-of-bounds access.
+ */
+int gad_attn_decode(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                    const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,
+                    uint8_t* v_cache, const float* k_scale, const float* v_scale, int B, int L,
+                    int max_pages, int64_t num_rows, int page_size, int window, int use_rope,
+                    void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Profiling variant of gad_attn_decode: same arguments and semantics, plus
+ * `events`, an array of four cudaEvent_t created by the caller.  It records
+ * events[0] before the prep kernel, events[1] between prep and decode,
+ * events[2] between decode and combine and events[3] after combine, all on
+ * `stream`, so cudaEventElapsedTime gives each kernel's device time.  Because
+ * an event sits between the kernels, they run strictly one after another
+ * (no programmatic dependent launch overlap); use gad_attn_decode in
+ * production.  Returns GAD_ERR_NULL if events or any of its entries is NULL.
+ */
+int gad_attn_decode_timed(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                          const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,
+                          uint8_t* v_cache, const float* k_scale, const float* v_scale, int B,
+                          int L, int max_pages, int64_t num_rows, int page_size, int window,
+                          int use_rope, void* out, void* workspace, size_t workspace_bytes,
+                          void* stream, void* const* events);
+
+/* Message for the last nonzero status returned on this host thread. */
+const char* gad_last_error(void);
+
+/* Static name of a gad_status value. */
+const char* gad_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GAD_ATTN_H */

@@ -1,0 +1,167 @@
+"""Python binding of libgad_attn.so (argument marshalling only).
+
+Every step of the computation runs in the library's CUDA kernels; this module
+only checks torch tensors' dtypes and layouts, allocates the output and the
+workspace with torch when the caller does not pass them, and forwards raw
+device pointers and the current CUDA stream to the C ABI (include/gad_attn.h).
+
+Importing it fails loudly when the library has not been built: there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgad_attn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is not built; run `python -m paged_fp8_gated_b200.build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp = ctypes.c_void_p
+_lib.gad_attn_workspace_bytes.restype = ctypes.c_size_t
+_lib.gad_attn_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
+_lib.gad_attn_decode.restype = ctypes.c_int
+_lib.gad_attn_decode.argtypes = [
+    _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,            # qkv .. v_scale
+    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,  # B, L, max_pages, num_rows
+    ctypes.c_int, ctypes.c_int, ctypes.c_int,               # page_size, window, use_rope
+    _vp, _vp, ctypes.c_size_t, _vp]                         # out, workspace, bytes, stream
+_lib.gad_attn_decode_timed.restype = ctypes.c_int
+_lib.gad_attn_decode_timed.argtypes = list(_lib.gad_attn_decode.argtypes) + [_vp]
+_lib.gad_last_error.restype = ctypes.c_char_p
+_lib.gad_last_error.argtypes = []
+_lib.gad_status_string.restype = ctypes.c_char_p
+_lib.gad_status_string.argtypes = [ctypes.c_int]
+
+HQ, HKV, D = 16, 2, 64
+QKV_COLS, OUT_COLS, ROW_BYTES = 2304, 1024, 128
+
+EXPORTED = ("gad_attn_decode", "gad_attn_decode_timed", "gad_attn_workspace_bytes",
+            "gad_last_error", "gad_status_string")
+
+
+class GadError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib.gad_last_error().decode(errors="replace")
+        name = _lib.gad_status_string(status).decode()
+        super().__init__(f"{where}: {name} ({status}): {msg}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def workspace_bytes(B: int, L: int) -> int:
+    n = _lib.gad_attn_workspace_bytes(int(B), int(L))
+    if n == 0:
+        raise GadError(-2, "gad_attn_workspace_bytes")
+    return int(n)
+
+
+def alloc_workspace(B: int, L: int, device=None) -> torch.Tensor:
+    """Caller-owned scratch for gad_attn_decode (256-byte aligned by torch's allocator)."""
+    return torch.empty(workspace_bytes(B, L), dtype=torch.uint8, device=device or "cuda")
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+def attn_decode(qkv: torch.Tensor, positions: torch.Tensor, seq_lens: torch.Tensor | None,
+                page_table: torch.Tensor, cache_loc: torch.Tensor, k_cache: torch.Tensor,
+                v_cache: torch.Tensor, k_scale: torch.Tensor, v_scale: torch.Tensor,
+                page_size: int, window: int, use_rope: bool, L: int = 1,
+                out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                stream: torch.cuda.Stream | None = None,
+                events: list | None = None) -> torch.Tensor:
+    """One decode step (L = 1) or verify block (L <= 8); returns out bf16 [B, L, 1024].
+
+    Shapes: qkv bf16 [B*L, 2304]; positions, cache_loc int64 [B*L]; seq_lens int32 [B]
+    (optional); page_table int32 [B, max_pages]; k_cache / v_cache uint8
+    [num_pages, page_size, 2, 64] (mutated in the rows cache_loc); k_scale / v_scale
+    float32 [1] on the device.  With ``events`` (four torch.cuda.Event with timing),
+    the profiling entry point records them around the three kernels.
+    """
+    _need(qkv, "qkv", torch.bfloat16, 2)
+    _need(positions, "positions", torch.int64, 1)
+    _need(page_table, "page_table", torch.int32, 2)
+    _need(cache_loc, "cache_loc", torch.int64, 1)
+    _need(k_cache, "k_cache", torch.uint8)
+    _need(v_cache, "v_cache", torch.uint8)
+    _need(k_scale, "k_scale", torch.float32)
+    _need(v_scale, "v_scale", torch.float32)
+    if seq_lens is not None:
+        _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, max_pages = page_table.shape
+    T = qkv.shape[0]
+    if qkv.shape[1] != QKV_COLS or T != B * L:
+        raise ValueError(f"qkv must be [B*L={B * L}, {QKV_COLS}], got {tuple(qkv.shape)}")
+    if positions.numel() != T or cache_loc.numel() != T:
+        raise ValueError("positions and cache_loc need one entry per token")
+    if k_cache.shape != v_cache.shape or k_cache.numel() % ROW_BYTES:
+        raise ValueError("k_cache and v_cache must have the same shape, 128 bytes per row")
+    num_rows = k_cache.numel() // ROW_BYTES
+    if out is None:
+        out = torch.empty(B, L, OUT_COLS, dtype=torch.bfloat16, device=qkv.device)
+    else:
+        _need(out, "out", torch.bfloat16)
+        if out.numel() != T * OUT_COLS:
+            raise ValueError("out must hold B*L*1024 values")
+    if workspace is None:
+        workspace = alloc_workspace(B, L, qkv.device)
+    else:
+        _need(workspace, "workspace", torch.uint8)
+    s = (stream or torch.cuda.current_stream(qkv.device)).cuda_stream
+    args = (_ptr(qkv), _ptr(positions), _ptr(seq_lens), _ptr(page_table), _ptr(cache_loc),
+            _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), int(B), int(L),
+            int(max_pages), int(num_rows), int(page_size), int(window), int(bool(use_rope)),
+            _ptr(out), _ptr(workspace), int(workspace.numel()), ctypes.c_void_p(s))
+    if events is None:
+        st = _lib.gad_attn_decode(*args)
+    else:
+        if len(events) != 4:
+            raise ValueError("events must hold four torch.cuda.Event")
+        for ev in events:   # materialise the underlying cudaEvent_t
+            if ev.cuda_event == 0:
+                ev.record()
+        arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(ev.cuda_event) for ev in events])
+        st = _lib.gad_attn_decode_timed(*args, arr)
+    if st != 0:
+        raise GadError(st, "gad_attn_decode")
+    return out
+
+
+def raw_call(**kw) -> int:
+    """Call the C entry point with raw values (for boundary tests); returns the status."""
+    args = [kw.get(k) for k in ("qkv", "positions", "seq_lens", "page_table", "cache_loc",
+                                "k_cache", "v_cache", "k_scale", "v_scale")]
+    args = [a if (a is None or isinstance(a, ctypes.c_void_p)) else ctypes.c_void_p(a) for a in args]
+    return _lib.gad_attn_decode(*args, kw.get("B", 1), kw.get("L", 1), kw.get("max_pages", 1),
+                                kw.get("num_rows", 1), kw.get("page_size", 1),
+                                kw.get("window", 0), kw.get("use_rope", 0), kw.get("out"),
+                                kw.get("workspace"), kw.get("workspace_bytes", 0),
+                                kw.get("stream"))
+
+
+def last_error() -> str:
+    return _lib.gad_last_error().decode(errors="replace")

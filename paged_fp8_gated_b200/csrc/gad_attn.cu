@@ -1,0 +1,285 @@
+// gad_attn.cu - C ABI of libgad_attn.so: argument checks, workspace layout and
+// the three launches (prep -> decode -> combine, chained with programmatic
+// dependent launch so each kernel's launch latency hides behind the previous
+// kernel's tail).
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "gad_attn.h"
+#include "gad_kernels.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int status, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return status;
+}
+
+constexpr int kMaxCtasPerSm = 2;
+constexpr int kMaxDevices = 64;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct WsLayout {
+    size_t q_off, po_off, pml_off, meta_off, total;
+    int slots, lt;
+};
+
+WsLayout ws_layout(int B, int L, int sms) {
+    WsLayout w{};
+    w.lt = L == 1 ? 1 : GAD_MAX_L;
+    w.slots = sms * kMaxCtasPerSm + B;
+    const size_t T = static_cast<size_t>(B) * L;
+    size_t off = 0;
+    w.q_off = off;
+    off = align_up(off + T * GAD_HQ * GAD_HEAD_DIM * 2);
+    w.po_off = off;
+    off = align_up(off + static_cast<size_t>(w.slots) * w.lt * GAD_HQ * GAD_HEAD_DIM * 4);
+    w.pml_off = off;
+    off = align_up(off + static_cast<size_t>(w.slots) * w.lt * GAD_HQ * 2 * 4);
+    w.meta_off = off;
+    off = align_up(off + static_cast<size_t>(B + 3) * 4);
+    w.total = off;
+    return w;
+}
+
+int current_device_sms(int* sms, int* major) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    e = cudaDeviceGetAttribute(major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    return GAD_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+cudaLaunchAttribute pdl_attr() {
+    cudaLaunchAttribute a;
+    std::memset(&a, 0, sizeof(a));
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+    return a;
+}
+
+template <int LT, int PS, int KG, int NS, int MINB>
+int launch_decode(const gad::StepParams& prm, int sms, int tiles_upper, cudaStream_t stream,
+                  bool pdl) {
+    using C = gad::DecodeCfg<LT, KG, NS>;
+    auto kern = gad::decode_kernel<LT, PS, KG, NS, MINB>;
+    const size_t smem = C::smem_bytes(prm.B);
+    // Raise the kernel's dynamic shared-memory limit once per device, to the
+    // largest size any B needs, so no attribute call happens during capture.
+    static std::atomic<bool> attr_done[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", dev);
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(C::smem_bytes(GAD_MAX_B)));
+        if (e != cudaSuccess)
+            return fail(GAD_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, gad::DEC_THREADS, smem);
+    if (e != cudaSuccess || occ < 1)
+        return fail(GAD_ERR_CUDA, "decode kernel does not fit on an SM (smem %zu B): %s", smem,
+                    cudaGetErrorString(e));
+    occ = occ > kMaxCtasPerSm ? kMaxCtasPerSm : occ;
+    long long grid = static_cast<long long>(sms) * occ;
+    if (grid > tiles_upper) grid = tiles_upper;
+    if (grid < 1) grid = 1;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(gad::DEC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr = pdl_attr();
+    cfg.attrs = &attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, prm);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    return GAD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gad_last_error(void) { return g_last_error.c_str(); }
+
+const char* gad_status_string(int status) {
+    switch (status) {
+        case GAD_OK: return "GAD_OK";
+        case GAD_ERR_NULL: return "GAD_ERR_NULL";
+        case GAD_ERR_SHAPE: return "GAD_ERR_SHAPE";
+        case GAD_ERR_ALIGN: return "GAD_ERR_ALIGN";
+        case GAD_ERR_UNSUPPORTED: return "GAD_ERR_UNSUPPORTED";
+        case GAD_ERR_WORKSPACE: return "GAD_ERR_WORKSPACE";
+        case GAD_ERR_CUDA: return "GAD_ERR_CUDA";
+        case GAD_ERR_DEVICE: return "GAD_ERR_DEVICE";
+        default: return "unknown gad_status";
+    }
+}
+
+size_t gad_attn_workspace_bytes(int B, int L) {
+    if (B < 1 || B > GAD_MAX_B || L < 1 || L > GAD_MAX_L) {
+        fail(GAD_ERR_SHAPE, "B=%d must be in [1,%d] and L=%d in [1,%d]", B, GAD_MAX_B, L, GAD_MAX_L);
+        return 0;
+    }
+    int sms = 0, major = 0;
+    if (current_device_sms(&sms, &major) != GAD_OK) return 0;
+    return ws_layout(B, L, sms).total;
+}
+
+static int run_step(const void* qkv, const int64_t* positions, const int32_t* page_table,
+                    const int64_t* cache_loc, uint8_t* k_cache, uint8_t* v_cache,
+                    const float* k_scale, const float* v_scale, int B, int L, int max_pages,
+                    int64_t num_rows, int page_size, int window, int use_rope, void* out,
+                    void* workspace, size_t workspace_bytes, void* stream, void* const* events) {
+    if (!qkv || !positions || !page_table || !cache_loc || !k_cache || !v_cache || !k_scale ||
+        !v_scale || !out)
+        return fail(GAD_ERR_NULL, "a required pointer is NULL");
+    if (!workspace) return fail(GAD_ERR_WORKSPACE, "workspace is NULL");
+    if (B < 1 || B > GAD_MAX_B) return fail(GAD_ERR_SHAPE, "B=%d not in [1,%d]", B, GAD_MAX_B);
+    if (L < 1 || L > GAD_MAX_L) return fail(GAD_ERR_SHAPE, "L=%d not in [1,%d]", L, GAD_MAX_L);
+    if (max_pages < 1) return fail(GAD_ERR_SHAPE, "max_pages=%d < 1", max_pages);
+    if (page_size != 1 && page_size != 64)
+        return fail(GAD_ERR_UNSUPPORTED, "page_size=%d (supported: 1, 64)", page_size);
+    if (num_rows < 1 || num_rows % page_size != 0)
+        return fail(GAD_ERR_SHAPE, "num_rows=%lld must be a positive multiple of page_size",
+                    static_cast<long long>(num_rows));
+    if (static_cast<long long>(max_pages) * page_size > INT32_MAX)
+        return fail(GAD_ERR_SHAPE, "max_pages * page_size exceeds 2^31");
+    if (window < 0) return fail(GAD_ERR_UNSUPPORTED, "window=%d < 0", window);
+    if (!aligned(qkv, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+        return fail(GAD_ERR_ALIGN, "qkv, out, k_cache and v_cache must be 16-byte aligned");
+    if (!aligned(positions, 8) || !aligned(cache_loc, 8) || !aligned(page_table, 4) ||
+        !aligned(k_scale, 4) || !aligned(v_scale, 4))
+        return fail(GAD_ERR_ALIGN, "positions/cache_loc need 8-byte, page_table/scales 4-byte alignment");
+    if (!aligned(workspace, kAlign)) return fail(GAD_ERR_ALIGN, "workspace must be 256-byte aligned");
+
+    int sms = 0, major = 0;
+    int st = current_device_sms(&sms, &major);
+    if (st != GAD_OK) return st;
+    if (major != 10) return fail(GAD_ERR_DEVICE, "compute capability %d.x; this build targets sm_100a", major);
+    const WsLayout w = ws_layout(B, L, sms);
+    if (workspace_bytes < w.total)
+        return fail(GAD_ERR_WORKSPACE, "workspace %zu B < required %zu B", workspace_bytes, w.total);
+
+    gad::StepParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.qkv = static_cast<const __nv_bfloat16*>(qkv);
+    prm.positions = positions;
+    prm.page_table = page_table;
+    prm.cache_loc = cache_loc;
+    prm.k_cache = k_cache;
+    prm.v_cache = v_cache;
+    prm.k_scale = k_scale;
+    prm.v_scale = v_scale;
+    prm.out = static_cast<__nv_bfloat16*>(out);
+    prm.B = B;
+    prm.L = L;
+    prm.max_pages = max_pages;
+    prm.window = window;
+    prm.use_rope = use_rope ? 1 : 0;
+    prm.num_rows = num_rows;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    prm.q_ws = reinterpret_cast<__half*>(ws + w.q_off);
+    prm.part_o = reinterpret_cast<float*>(ws + w.po_off);
+    prm.part_ml = reinterpret_cast<float*>(ws + w.pml_off);
+    prm.meta = reinterpret_cast<int*>(ws + w.meta_off);
+    prm.lt = w.lt;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int T = B * L;
+
+    // upper bound of tiles in the step (only caps the grid; the split itself is on device)
+    long long per_req;
+    if (window > 0) per_req = (static_cast<long long>(window) + L - 1 + gad::TILE - 1) / gad::TILE + 1;
+    else per_req = (static_cast<long long>(max_pages) * page_size + gad::TILE - 1) / gad::TILE + 1;
+    long long tiles_upper_ll = per_req * B;
+    const int tiles_upper = tiles_upper_ll > INT32_MAX ? INT32_MAX : static_cast<int>(tiles_upper_ll);
+
+    const bool timed = events != nullptr;
+    cudaError_t e;
+    if (timed) {
+        e = cudaEventRecord(static_cast<cudaEvent_t>(events[0]), s);
+        if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaEventRecord: %s", cudaGetErrorString(e));
+    }
+    gad::prep_kernel<<<T, gad::PREP_THREADS, 0, s>>>(prm);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
+    if (timed) cudaEventRecord(static_cast<cudaEvent_t>(events[1]), s);
+
+    if (L == 1) {
+        st = page_size == 1 ? launch_decode<1, 1, 4, 4, 2>(prm, sms, tiles_upper, s, !timed)
+                            : launch_decode<1, 64, 4, 4, 2>(prm, sms, tiles_upper, s, !timed);
+    } else {
+        st = page_size == 1 ? launch_decode<8, 1, 2, 4, 1>(prm, sms, tiles_upper, s, !timed)
+                            : launch_decode<8, 64, 2, 4, 1>(prm, sms, tiles_upper, s, !timed);
+    }
+    if (st != GAD_OK) return st;
+    if (timed) cudaEventRecord(static_cast<cudaEvent_t>(events[2]), s);
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(T));
+    cfg.blockDim = dim3(gad::COMB_THREADS);
+    cfg.stream = s;
+    cudaLaunchAttribute attr = pdl_attr();
+    cfg.attrs = &attr;
+    cfg.numAttrs = timed ? 0 : 1;
+    e = cudaLaunchKernelEx(&cfg, gad::combine_kernel, prm);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+    if (timed) {
+        e = cudaEventRecord(static_cast<cudaEvent_t>(events[3]), s);
+        if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaEventRecord: %s", cudaGetErrorString(e));
+    }
+    return GAD_OK;
+}
+
+int gad_attn_decode(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                    const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,
+                    uint8_t* v_cache, const float* k_scale, const float* v_scale, int B, int L,
+                    int max_pages, int64_t num_rows, int page_size, int window, int use_rope,
+                    void* out, void* workspace, size_t workspace_bytes, void* stream) {
+    (void)seq_lens;
+    return run_step(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale, B,
+                    L, max_pages, num_rows, page_size, window, use_rope, out, workspace,
+                    workspace_bytes, stream, nullptr);
+}
+
+int gad_attn_decode_timed(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                          const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,
+                          uint8_t* v_cache, const float* k_scale, const float* v_scale, int B,
+                          int L, int max_pages, int64_t num_rows, int page_size, int window,
+                          int use_rope, void* out, void* workspace, size_t workspace_bytes,
+                          void* stream, void* const* events) {
+    (void)seq_lens;
+    if (!events || !events[0] || !events[1] || !events[2] || !events[3])
+        return fail(GAD_ERR_NULL, "events must hold four cudaEvent_t");
+    return run_step(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale, B,
+                    L, max_pages, num_rows, page_size, window, use_rope, out, workspace,
+                    workspace_bytes, stream, events);
+}
+
+}  // extern "C"

@@ -1,0 +1,630 @@
+// gad_kernels.cuh - the three sm_100a kernels of one attention step.
+//
+//   prep_kernel     per token: QK-norm, RoPE, E4M3 quantise-and-scatter of k/v
+//                   into the cache rows cache_loc[t]; normalised q -> workspace.
+//   decode_kernel   persistent split-KV flash decode over the paged FP8 cache:
+//                   cp.async gathers into a swizzled shared-memory ring, tensor-
+//                   core QK^T and PV (m16n8k16 fp16, fp32 accumulate) with the
+//                   query heads of one KV head packed into the MMA's N side,
+//                   online softmax, one (o, max, sum) partial per CTA segment.
+//   combine_kernel  log-sum-exp merge of the partials fused with the gated
+//                   output norm  out = rmsnorm(a) * sigmoid(gate)  -> bf16.
+//
+// Method: task page "Gated attention decode (muse_attention_decode)", section
+// "What to compute"; shapes from its section "Shapes".
+#pragma once
+
+#include <cfloat>
+#include <climits>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "gad_ptx.cuh"
+
+namespace gad {
+
+constexpr int HQ = 16;         // query heads
+constexpr int HKV = 2;         // key/value heads
+constexpr int HD = 64;         // head dim
+constexpr int GRP = HQ / HKV;  // query heads per KV head (8)
+constexpr int QKV_COLS = 2304;
+constexpr int K_OFF = 1024, V_OFF = 1152, G_OFF = 1280;
+constexpr int OUT_COLS = 1024;
+constexpr int ROWB = 128;                   // bytes per cache row: 2 KV heads x 64 codes
+constexpr int TILE = 64;                    // keys per pipeline stage
+constexpr int STAGE_BYTES = 2 * TILE * ROWB;  // K tile then V tile: 16 KB
+constexpr int DEC_THREADS = 256;
+constexpr int PREP_THREADS = (HQ + HKV) * 32;
+constexpr int COMB_THREADS = HQ * 32;
+
+struct StepParams {
+    const __nv_bfloat16* qkv;
+    const int64_t* positions;
+    const int32_t* page_table;
+    const int64_t* cache_loc;
+    uint8_t* k_cache;
+    uint8_t* v_cache;
+    const float* k_scale;
+    const float* v_scale;
+    __nv_bfloat16* out;
+    int B, L, max_pages, window, use_rope;
+    int64_t num_rows;
+    // workspace views
+    __half* q_ws;    // [T][16][64]  normalised (rotated) queries
+    float* part_o;   // [slots][lt][16][64]  un-normalised partial outputs
+    float* part_ml;  // [slots][lt][16][2]   (running max in log2 units, sum)
+    int* meta;       // [0] total tiles, [1] tiles per CTA, [2 .. 2+B] tile prefix
+    int lt;          // token capacity of one partial slot (1 or 8)
+};
+
+// ---------------------------------------------------------------------------
+// Kernel 1: split + QK-norm + RoPE + E4M3 quantise-and-scatter.
+// One block per token; warp w < 16 handles query head w, warps 16 and 17 the
+// two KV heads.  Lane l owns the RoPE pair (l, l + 32).  Done in double so the
+// cache bytes match the double-precision definition exactly: the sum of squares
+// runs in index order with explicit round-to-nearest operations (no fused
+// multiply-add), as does the rotation.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) {
+    pdl_launch_dependents();
+    const int t = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const __nv_bfloat16* row = p.qkv + static_cast<size_t>(t) * QKV_COLS;
+    const bool is_q = warp < HQ;
+    const int g = warp - HQ;
+    const int off = is_q ? warp * HD : K_OFF + g * HD;
+    const double x0 = static_cast<double>(__bfloat162float(row[off + lane]));
+    const double x1 = static_cast<double>(__bfloat162float(row[off + lane + 32]));
+
+    double ss = 0.0;
+    for (int d = 0; d < 32; ++d) {
+        const double v = __shfl_sync(0xffffffffu, x0, d);
+        ss = __dadd_rn(ss, __dmul_rn(v, v));
+    }
+    for (int d = 0; d < 32; ++d) {
+        const double v = __shfl_sync(0xffffffffu, x1, d);
+        ss = __dadd_rn(ss, __dmul_rn(v, v));
+    }
+    const double r = sqrt(__dadd_rn(ss / 64.0, 1e-6));
+    double u0 = x0 / r, u1 = x1 / r;
+    if (is_q) {
+        u0 = __dmul_rn(u0, 5.473);
+        u1 = __dmul_rn(u1, 5.473);
+    }
+    if (p.use_rope) {
+        const double pos = static_cast<double>(p.positions[t]);
+        const double inv_freq = pow(10000.0, -2.0 * lane / 64.0);
+        const double phi = __dmul_rn(pos, inv_freq);
+        const double c = cos(phi), s = sin(phi);
+        const double r0 = __dsub_rn(__dmul_rn(u0, c), __dmul_rn(u1, s));
+        const double r1 = __dadd_rn(__dmul_rn(u1, c), __dmul_rn(u0, s));
+        u0 = r0;
+        u1 = r1;
+    }
+    if (is_q) {
+        __half* q = p.q_ws + (static_cast<size_t>(t) * HQ + warp) * HD;
+        q[lane] = __double2half(u0);
+        q[lane + 32] = __double2half(u1);
+        return;
+    }
+    const int64_t crow = p.cache_loc[t];
+    if (crow < 0 || crow >= p.num_rows) return;
+    const double ks = static_cast<double>(__ldg(p.k_scale));
+    const double vs = static_cast<double>(__ldg(p.v_scale));
+    uint8_t* kd = p.k_cache + crow * ROWB + g * HD;
+    uint8_t* vd = p.v_cache + crow * ROWB + g * HD;
+    kd[lane] = __nv_cvt_float_to_fp8(__double2float_rn(u0 / ks), __NV_SATFINITE, __NV_E4M3);
+    kd[lane + 32] = __nv_cvt_float_to_fp8(__double2float_rn(u1 / ks), __NV_SATFINITE, __NV_E4M3);
+    const double v0 = static_cast<double>(__bfloat162float(row[V_OFF + g * HD + lane]));
+    const double v1 = static_cast<double>(__bfloat162float(row[V_OFF + g * HD + lane + 32]));
+    vd[lane] = __nv_cvt_float_to_fp8(__double2float_rn(v0 / vs), __NV_SATFINITE, __NV_E4M3);
+    vd[lane + 32] = __nv_cvt_float_to_fp8(__double2float_rn(v1 / vs), __NV_SATFINITE, __NV_E4M3);
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 2: split-KV decode.
+//
+// Work split.  Request b attends keys [lo_b, hi_b] (the union of its tokens'
+// ranges).  Its keys fall into 64-key tiles aligned to absolute key index
+// (so a 64-key page is exactly one tile).  All requests' tiles form one list;
+// CTA c takes tiles [c*per, (c+1)*per) of it, crossing request boundaries,
+// and writes one partial per (CTA, request) it touches into slot c + b
+// (unique, since both c and b only grow along the list).
+//
+// Shared-memory tile layout.  A stage holds 64 rows of K then 64 rows of V,
+// 128 bytes per row (both KV heads), 16-byte chunk j of row r stored at chunk
+// j ^ (r & 7) (the 128-byte swizzle).  The MMA's logical key l in a 16-key
+// group lives in row kappa(l) of that group; kappa is chosen so that both the
+// QK^T operand loads (16 bytes per lane) and the PV operand loads (8 bytes per
+// lane) are free of bank conflicts under that swizzle.
+//
+// MMA mapping (m16n8k16, transposed so the 8 query heads of a KV head fill N):
+//   S^T[key][head] = K[key][:] . Q[head][:]        A = K (fp16 from E4M3), B = Q
+//   O^T[dim][head] += V^T[dim][key] . P^T[key][head]  A = V^T, B = P^T
+// Each lane holds 16 contiguous K bytes of a row (dims permuted across k-steps
+// identically for K and Q), and 8 contiguous V dims; P^T's B fragment comes
+// from S^T's accumulator by one movmatrix transpose per 8x8 block.
+//
+// Warps: 8 = 2 KV heads x RG row groups (tokens) x KG key groups.  Each warp
+// runs its own online softmax over its keys; key groups are merged in shared
+// memory at the end of each segment.
+// ---------------------------------------------------------------------------
+template <int LT, int KG, int NS>
+struct DecodeCfg {
+    static constexpr int WARPS = DEC_THREADS / 32;
+    static constexpr int RG = WARPS / (HKV * KG);
+    static constexpr int NT = LT / RG;              // tokens per warp (MMA N tiles)
+    static constexpr int MT = (TILE / 16) / KG;     // 16-key groups per warp per tile
+    static constexpr int IDX_SLOTS = 2 * NS;
+    static constexpr int MERGE_WARPS = (KG - 1) * HKV * RG;
+    static constexpr int MERGE_FLOATS_PER_WARP = NT * 32 * 20;
+    static constexpr size_t KV_BYTES = static_cast<size_t>(NS) * STAGE_BYTES;
+    static constexpr size_t IDX_BYTES = static_cast<size_t>(IDX_SLOTS) * TILE * 4;
+    static constexpr size_t MERGE_BYTES =
+        static_cast<size_t>(MERGE_WARPS) * MERGE_FLOATS_PER_WARP * 4;
+    static size_t smem_bytes(int B) {
+        return KV_BYTES + IDX_BYTES + MERGE_BYTES + static_cast<size_t>(3 * B + 1) * 4;
+    }
+    static_assert(RG >= 1 && RG * HKV * KG == WARPS, "warp split");
+    static_assert(NT * RG == LT && MT * KG == TILE / 16, "tile split");
+};
+
+// Row (within a 16-key group) holding the MMA's logical key l.
+__device__ __forceinline__ int kappa(int l) {
+    const int x = l & 7;
+    const int s = ((((x & 1) << 2) ^ (((x >> 1) & 3) << 1)) | ((x >> 2) & 1));
+    return (l & 8) | s;
+}
+
+template <int LT, int PS, int KG, int NS, int MINB>
+__global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepParams p) {
+    using C = DecodeCfg<LT, KG, NS>;
+    constexpr int NT = C::NT, MT = C::MT, RG = C::RG;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* kv_smem = smem;
+    int* idx_smem = reinterpret_cast<int*>(smem + C::KV_BYTES);
+    float* merge_smem = reinterpret_cast<float*>(smem + C::KV_BYTES + C::IDX_BYTES);
+    int* tpre = reinterpret_cast<int*>(smem + C::KV_BYTES + C::IDX_BYTES + C::MERGE_BYTES);
+    int* rlo = tpre + p.B + 1;
+    int* rhi = rlo + p.B;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int g = warp % HKV;
+    const int rg = (warp / HKV) % RG;
+    const int kg = warp / (HKV * RG);
+    const int B = p.B, L = p.L;
+
+    // ---- request key ranges and the tile list (reads inputs only) ----
+    for (int b = tid; b < B; b += DEC_THREADS) {
+        int lo = INT_MAX, hi = -1;
+        for (int j = 0; j < L; ++j) {
+            const int pos = static_cast<int>(p.positions[static_cast<size_t>(b) * L + j]);
+            const int l = p.window > 0 ? max(0, pos - p.window + 1) : 0;
+            lo = min(lo, l);
+            hi = max(hi, pos);
+        }
+        rlo[b] = lo;
+        rhi[b] = hi;
+        tpre[b + 1] = (hi >= lo && hi >= 0) ? (hi / TILE - lo / TILE + 1) : 0;
+    }
+    if (tid == 0) tpre[0] = 0;
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        for (int base = 1; base <= B; base += 32) {
+            const int i = base + lane;
+            int v = i <= B ? tpre[i] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += n;
+            }
+            if (i <= B) tpre[i] = v + carry;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    __syncthreads();
+    const int total = tpre[B];
+    const int per = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+    const int t0 = static_cast<int>(blockIdx.x) * per;
+    const int t1 = min(t0 + per, total);
+    if (blockIdx.x == 0) {
+        for (int i = tid; i <= B; i += DEC_THREADS) p.meta[2 + i] = tpre[i];
+        if (tid == 0) {
+            p.meta[0] = total;
+            p.meta[1] = per;
+        }
+    }
+    // q and this step's cache rows come from the prep kernel
+    pdl_wait_primary();
+    if (t0 >= t1) return;
+
+    const float C2 = __ldg(p.k_scale) * 0.125f * 1.4426950408889634f;  // raw score -> log2 units
+
+    // ---- tile cursors ----
+    auto find_req = [&](int tau) {
+        int lo = 0, hi = B;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tpre[mid] <= tau) lo = mid;
+            else hi = mid;
+        }
+        return lo;
+    };
+    auto advance = [&](int& tau, int& b) {
+        ++tau;
+        while (b < B - 1 && tau >= tpre[b + 1]) ++b;
+    };
+    auto tile_k0 = [&](int tau, int b) { return (rlo[b] / TILE + (tau - tpre[b])) * TILE; };
+
+    // ---- async loads ----
+    auto issue_idx = [&](int tau, int b) {
+        if (tau >= t1) return;
+        const int k0 = tile_k0(tau, b);
+        int* dst = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TILE;
+        const int32_t* pt = p.page_table + static_cast<size_t>(b) * p.max_pages;
+        if (PS == 1) {
+            if (tid < TILE) {
+                const int k = k0 + tid;
+                if (k >= rlo[b] && k <= rhi[b] && k < p.max_pages) cp_async4(smem_addr(dst + tid), pt + k);
+                else dst[tid] = -1;
+            }
+        } else {
+            if (tid == 0) {
+                const int pg = k0 / PS;
+                if (pg < p.max_pages) cp_async4(smem_addr(dst), pt + pg);
+                else dst[0] = -1;
+            }
+        }
+    };
+    auto issue_kv = [&](int tau, int b) {
+        if (tau >= t1) return;
+        const int k0 = tile_k0(tau, b);
+        const int* ix = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TILE;
+        const uint32_t base = smem_addr(kv_smem + ((tau - t0) % NS) * STAGE_BYTES);
+        const int lo = rlo[b], hi = rhi[b];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int r = (tid >> 3) + 32 * i;  // tile row
+            const int j = tid & 7;              // 16-byte chunk
+            const int k = k0 + r;
+            int64_t crow;
+            if (PS == 1) crow = ix[r];
+            else crow = ix[0] >= 0 ? static_cast<int64_t>(ix[0]) * PS + r : -1;
+            const bool ok = k >= lo && k <= hi && crow >= 0 && crow < p.num_rows;
+            const size_t off = ok ? static_cast<size_t>(crow) * ROWB + j * 16 : 0;
+            const uint32_t d = base + r * ROWB + ((j ^ (r & 7)) << 4);
+            cp_async16(d, p.k_cache + off, ok ? 16 : 0);
+            cp_async16(d + TILE * ROWB, p.v_cache + off, ok ? 16 : 0);
+        }
+    };
+
+    // ---- per-warp state ----
+    float o_acc[NT][4][4];
+    float m_run[NT][2], l_run[NT][2];
+    uint32_t qf[NT][8];
+    int tok_lo[NT], tok_hi[NT];
+    int req_lo_max = 0, req_hi_min = -1;
+
+    const int krow = kappa(gid);             // QK^T: rows krow, krow + 8 of each group
+    const int vrow0 = kappa(2 * tig), vrow1 = kappa(2 * tig + 1);  // PV: + 0 and + 8
+
+    auto begin_request = [&](int b) {
+        req_lo_max = 0;
+        req_hi_min = INT_MAX;
+        for (int j = 0; j < L; ++j) {
+            const int pos = static_cast<int>(p.positions[static_cast<size_t>(b) * L + j]);
+            const int l = p.window > 0 ? max(0, pos - p.window + 1) : 0;
+            req_lo_max = max(req_lo_max, l);
+            req_hi_min = min(req_hi_min, pos);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int j = rg * NT + nt;
+            if (j < L) {
+                const size_t t = static_cast<size_t>(b) * L + j;
+                const int pos = static_cast<int>(p.positions[t]);
+                tok_hi[nt] = pos;
+                tok_lo[nt] = p.window > 0 ? max(0, pos - p.window + 1) : 0;
+                const uint4* q = reinterpret_cast<const uint4*>(
+                    p.q_ws + (t * HQ + g * GRP + gid) * HD + 16 * tig);
+                const uint4 a = q[0], c = q[1];
+                qf[nt][0] = a.x; qf[nt][1] = a.y; qf[nt][2] = a.z; qf[nt][3] = a.w;
+                qf[nt][4] = c.x; qf[nt][5] = c.y; qf[nt][6] = c.z; qf[nt][7] = c.w;
+            } else {
+                tok_lo[nt] = INT_MAX;
+                tok_hi[nt] = -1;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) qf[nt][i] = 0u;
+            }
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                m_run[nt][e] = -INFINITY;
+                l_run[nt][e] = 0.f;
+            }
+#pragma unroll
+            for (int dt = 0; dt < 4; ++dt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) o_acc[nt][dt][c] = 0.f;
+        }
+    };
+
+    auto compute_tile = [&](int slot, int k0) {
+        const uint32_t kbase = smem_addr(kv_smem + slot * STAGE_BYTES);
+        const uint32_t vbase = kbase + TILE * ROWB;
+        const bool need_mask = !(k0 >= req_lo_max && k0 + TILE - 1 <= req_hi_min);
+        float s[MT][NT][4];
+        // S^T = K . Q^T
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+            const int ra = (kg * MT + i) * 16 + krow;
+            const uint32_t chunk = static_cast<uint32_t>(((4 * g + tig) ^ (ra & 7)) << 4);
+            const uint4 ka = lds128(kbase + ra * ROWB + chunk);
+            const uint4 kb = lds128(kbase + (ra + 8) * ROWB + chunk);
+            const uint32_t kaw[4] = {ka.x, ka.y, ka.z, ka.w};
+            const uint32_t kbw[4] = {kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) s[i][nt][c] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                uint32_t a[4];
+                a[0] = e4m3x2_to_f16x2(kaw[ks]);
+                a[1] = e4m3x2_to_f16x2(kbw[ks]);
+                a[2] = e4m3x2_to_f16x2(kaw[ks] >> 16);
+                a[3] = e4m3x2_to_f16x2(kbw[ks] >> 16);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_16816(s[i][nt], a, qf[nt][2 * ks], qf[nt][2 * ks + 1]);
+            }
+        }
+        if (need_mask) {
+#pragma unroll
+            for (int i = 0; i < MT; ++i) {
+                const int key_a = k0 + (kg * MT + i) * 16 + krow;
+                const int key_b = key_a + 8;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (key_a < tok_lo[nt] || key_a > tok_hi[nt]) s[i][nt][0] = s[i][nt][1] = -INFINITY;
+                    if (key_b < tok_lo[nt] || key_b > tok_hi[nt]) s[i][nt][2] = s[i][nt][3] = -INFINITY;
+                }
+            }
+        }
+        // online softmax (per token, per head 2*tig + e)
+        uint32_t pf[MT][NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < MT; ++i) mx = fmaxf(mx, fmaxf(s[i][nt][e], s[i][nt][2 + e]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float m_new = fmaxf(m_run[nt][e], mx);
+                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+                const float alpha = fast_exp2((m_run[nt][e] - m_use) * C2);
+                m_run[nt][e] = m_new;
+                float lsum = l_run[nt][e] * alpha;
+#pragma unroll
+                for (int dt = 0; dt < 4; ++dt) {
+                    o_acc[nt][dt][e] *= alpha;
+                    o_acc[nt][dt][2 + e] *= alpha;
+                }
+                const float mc = m_use * C2;
+#pragma unroll
+                for (int i = 0; i < MT; ++i) {
+                    const float p0 = fast_exp2(fmaf(s[i][nt][e], C2, -mc));
+                    const float p1 = fast_exp2(fmaf(s[i][nt][2 + e], C2, -mc));
+                    s[i][nt][e] = p0;
+                    s[i][nt][2 + e] = p1;
+                    lsum += p0 + p1;
+                }
+                l_run[nt][e] = lsum;
+            }
+#pragma unroll
+            for (int i = 0; i < MT; ++i) {
+                pf[i][nt][0] = movmatrix_t(pack_f16x2(s[i][nt][0], s[i][nt][1]));
+                pf[i][nt][1] = movmatrix_t(pack_f16x2(s[i][nt][2], s[i][nt][3]));
+            }
+        }
+        // O^T += V^T . P^T
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+            const int gb = (kg * MT + i) * 16;
+            const int r0 = gb + vrow0, r1 = gb + vrow1;
+            const int cpos = 4 * g + (gid >> 1);
+            const uint32_t sub = static_cast<uint32_t>((gid & 1) * 8);
+            const uint2 x0 = lds64(vbase + r0 * ROWB + ((cpos ^ (r0 & 7)) << 4) + sub);
+            const uint2 x1 = lds64(vbase + r1 * ROWB + ((cpos ^ (r1 & 7)) << 4) + sub);
+            const uint2 x2 = lds64(vbase + (r0 + 8) * ROWB + ((cpos ^ (r0 & 7)) << 4) + sub);
+            const uint2 x3 = lds64(vbase + (r1 + 8) * ROWB + ((cpos ^ (r1 & 7)) << 4) + sub);
+#pragma unroll
+            for (int dt = 0; dt < 4; ++dt) {
+                const uint32_t w0 = dt < 2 ? x0.x : x0.y, w1 = dt < 2 ? x1.x : x1.y;
+                const uint32_t w2 = dt < 2 ? x2.x : x2.y, w3 = dt < 2 ? x3.x : x3.y;
+                const uint32_t sel = (dt & 1) ? 0x7362u : 0x5140u;
+                const uint32_t p01 = __byte_perm(w0, w1, sel);
+                const uint32_t p23 = __byte_perm(w2, w3, sel);
+                uint32_t a[4];
+                a[0] = e4m3x2_to_f16x2(p01);
+                a[1] = e4m3x2_to_f16x2(p01 >> 16);
+                a[2] = e4m3x2_to_f16x2(p23);
+                a[3] = e4m3x2_to_f16x2(p23 >> 16);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_16816(o_acc[nt][dt], a, pf[i][nt][0], pf[i][nt][1]);
+            }
+        }
+    };
+
+    auto flush = [&](int b) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float l = l_run[nt][e];
+                l += __shfl_xor_sync(0xffffffffu, l, 4);
+                l += __shfl_xor_sync(0xffffffffu, l, 8);
+                l += __shfl_xor_sync(0xffffffffu, l, 16);
+                l_run[nt][e] = l;
+            }
+        if (KG > 1) {
+            if (kg > 0) {
+                float* buf = merge_smem +
+                             static_cast<size_t>(((kg - 1) * HKV * RG + g * RG + rg) * NT) * 640;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    float* d = buf + (nt * 32 + lane) * 20;
+#pragma unroll
+                    for (int dt = 0; dt < 4; ++dt)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) d[dt * 4 + c] = o_acc[nt][dt][c];
+                    d[16] = m_run[nt][0];
+                    d[17] = m_run[nt][1];
+                    d[18] = l_run[nt][0];
+                    d[19] = l_run[nt][1];
+                }
+            }
+            __syncthreads();
+            if (kg == 0) {
+                for (int k = 1; k < KG; ++k) {
+                    const float* buf = merge_smem +
+                                       static_cast<size_t>(((k - 1) * HKV * RG + g * RG + rg) * NT) * 640;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const float* d = buf + (nt * 32 + lane) * 20;
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const float mo = d[16 + e], lo = d[18 + e];
+                            const float M = fmaxf(m_run[nt][e], mo);
+                            if (M == -INFINITY) continue;
+                            const float a = fast_exp2((m_run[nt][e] - M) * C2);
+                            const float ao = fast_exp2((mo - M) * C2);
+                            l_run[nt][e] = a * l_run[nt][e] + ao * lo;
+                            m_run[nt][e] = M;
+#pragma unroll
+                            for (int dt = 0; dt < 4; ++dt) {
+                                o_acc[nt][dt][e] = a * o_acc[nt][dt][e] + ao * d[dt * 4 + e];
+                                o_acc[nt][dt][2 + e] = a * o_acc[nt][dt][2 + e] + ao * d[dt * 4 + 2 + e];
+                            }
+                        }
+                    }
+                }
+            }
+            __syncthreads();
+        }
+        if (kg == 0) {
+            const size_t slot = static_cast<size_t>(blockIdx.x) + b;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int j = rg * NT + nt;
+                if (j >= L) continue;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int h = g * GRP + 2 * tig + e;
+                    const size_t base = (slot * p.lt + j) * HQ + h;
+                    float4* dst = reinterpret_cast<float4*>(p.part_o + base * HD + 8 * gid);
+                    dst[0] = make_float4(o_acc[nt][0][e], o_acc[nt][0][2 + e], o_acc[nt][1][e],
+                                         o_acc[nt][1][2 + e]);
+                    dst[1] = make_float4(o_acc[nt][2][e], o_acc[nt][2][2 + e], o_acc[nt][3][e],
+                                         o_acc[nt][3][2 + e]);
+                    if (gid == 0) {
+                        p.part_ml[base * 2 + 0] = m_run[nt][e] * C2;
+                        p.part_ml[base * 2 + 1] = l_run[nt][e];
+                    }
+                }
+            }
+        }
+    };
+
+    // ---- pipeline ----
+    int xt = t0, xb = find_req(t0);  // idx issue cursor
+    int kt = t0, kb = xb;            // kv issue cursor
+    int ct = t0, cb = xb;            // compute cursor
+    for (int d = 0; d < NS - 1; ++d) {
+        issue_idx(xt, xb);
+        advance(xt, xb);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    for (int d = 0; d < NS - 1; ++d) {
+        issue_kv(kt, kb);
+        advance(kt, kb);
+        issue_idx(xt, xb);
+        advance(xt, xb);
+        cp_async_commit();
+    }
+    int cur_b = -1;
+    for (int i = 0; ct < t1; ++i) {
+        cp_async_wait<NS - 2>();
+        __syncthreads();
+        issue_kv(kt, kb);
+        advance(kt, kb);
+        issue_idx(xt, xb);
+        advance(xt, xb);
+        cp_async_commit();
+        if (cb != cur_b) {
+            if (cur_b >= 0) flush(cur_b);
+            begin_request(cb);
+            cur_b = cb;
+        }
+        compute_tile(i % NS, tile_k0(ct, cb));
+        advance(ct, cb);
+    }
+    flush(cur_b);
+    cp_async_wait<0>();
+    pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 3: merge the partials of each (token, head) and apply the gated
+// output norm.  One block per token, one warp per head, two dims per lane.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams p) {
+    pdl_wait_primary();
+    const int t = blockIdx.x;
+    const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = t / p.L, j = t % p.L;
+    const int tp = p.meta[2 + b];
+    const int n = p.meta[3 + b] - tp;
+    const int per = p.meta[1];
+    const int d0 = 2 * lane;
+    float y0 = NAN, y1 = NAN;
+    if (n > 0 && per > 0) {
+        const int c_lo = tp / per, c_hi = (tp + n - 1) / per;
+        float M = -INFINITY;
+        for (int c = c_lo; c <= c_hi; ++c) {
+            const size_t base = (static_cast<size_t>(c + b) * p.lt + j) * HQ + h;
+            M = fmaxf(M, p.part_ml[base * 2]);
+        }
+        float l = 0.f, o0 = 0.f, o1 = 0.f;
+        for (int c = c_lo; c <= c_hi; ++c) {
+            const size_t base = (static_cast<size_t>(c + b) * p.lt + j) * HQ + h;
+            const float ms = p.part_ml[base * 2], ls = p.part_ml[base * 2 + 1];
+            const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+            const float2 o = *reinterpret_cast<const float2*>(p.part_o + base * HD + d0);
+            l += w * ls;
+            o0 += w * o.x;
+            o1 += w * o.y;
+        }
+        const float vs = __ldg(p.v_scale);
+        const float a0 = o0 / l * vs, a1 = o1 / l * vs;
+        float ss = a0 * a0 + a1 * a1;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float rinv = 1.0f / sqrtf(ss * (1.0f / 64.0f) + 1e-6f);
+        const __nv_bfloat16* gate = p.qkv + static_cast<size_t>(t) * QKV_COLS + G_OFF + h * HD + d0;
+        const float g0 = __bfloat162float(gate[0]), g1 = __bfloat162float(gate[1]);
+        y0 = a0 * rinv / (1.0f + expf(-g0));
+        y1 = a1 * rinv / (1.0f + expf(-g1));
+    }
+    *reinterpret_cast<__nv_bfloat162*>(p.out + static_cast<size_t>(t) * OUT_COLS + h * HD + d0) =
+        __floats2bfloat162_rn(y0, y1);
+}
+
+}  // namespace gad

@@ -1,0 +1,93 @@
+"""The C-ABI library loads, exports every function include/gad_attn.h declares,
+and rejects bad arguments on the host before touching a GPU (no GPU needed:
+every call here fails validation before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gad_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_fp8_gated_b200 import build
+    build.build()
+    from paged_fp8_gated_b200 import binding
+    return binding
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(gad_[A-Za-z0-9_]+)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("gad_attn_decode", "gad_attn_workspace_bytes", "gad_last_error", "gad_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(so, n), n
+    assert set(lib.EXPORTED) <= set(declared_functions())
+
+
+def test_status_strings(lib):
+    so = lib.lib()
+    assert so.gad_status_string(0) == b"GAD_OK"
+    assert so.gad_status_string(-4) == b"GAD_ERR_UNSUPPORTED"
+
+
+FAKE = 0x10000  # never dereferenced: validation fails before any device work
+
+
+def _ok_args(**over):
+    a = dict(qkv=FAKE, positions=FAKE, seq_lens=None, page_table=FAKE, cache_loc=FAKE,
+             k_cache=FAKE, v_cache=FAKE, k_scale=FAKE, v_scale=FAKE, B=2, L=1, max_pages=8,
+             num_rows=64, page_size=1, window=0, use_rope=0, out=FAKE, workspace=FAKE,
+             workspace_bytes=1 << 20, stream=None)
+    a.update(over)
+    return a
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(qkv=None), -1),
+    (dict(out=None), -1),
+    (dict(k_scale=None), -1),
+    (dict(workspace=None), -5),
+    (dict(B=0), -2),
+    (dict(B=5000), -2),
+    (dict(L=0), -2),
+    (dict(L=9), -2),
+    (dict(max_pages=0), -2),
+    (dict(page_size=16), -4),
+    (dict(page_size=64, num_rows=100), -2),
+    (dict(num_rows=0), -2),
+    (dict(window=-1), -4),
+    (dict(qkv=FAKE + 8), -3),
+    (dict(k_cache=FAKE + 4), -3),
+    (dict(positions=FAKE + 4), -3),
+    (dict(workspace=FAKE + 16), -3),
+])
+def test_argument_checks_fail_before_launch(lib, over, status):
+    assert lib.raw_call(**_ok_args(**over)) == status
+    assert lib.last_error()
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 2304, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        lib.attn_decode(x, torch.zeros(1, dtype=torch.int64), None,
+                        torch.zeros(1, 4, dtype=torch.int32), torch.zeros(1, dtype=torch.int64),
+                        torch.zeros(4, 1, 2, 64, dtype=torch.uint8),
+                        torch.zeros(4, 1, 2, 64, dtype=torch.uint8), torch.ones(1), torch.ones(1),
+                        1, 0, False)

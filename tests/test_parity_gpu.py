@@ -1,0 +1,154 @@
+"""Parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Cache bytes written by the step: bit-exact everywhere (the whole cache is
+compared, so rows the step must not touch are checked too).  Output: max
+|gpu - oracle| <= 2e-2 + 2e-2 |oracle| element-wise, on every output for the
+small cases and on sampled (token, head) outputs at the full workload sizes.
+"""
+import numpy as np
+import pytest
+import torch
+
+from paged_fp8_gated_b200 import workloads as W
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+S = W.Spec
+
+SMALL = [
+    # the page's gating shapes (section "Shapes"), shrunk only where noted
+    S("b1_ctx10_sliding", B=1, ctx=10, window=2048, use_rope=True, page_size=64, seed=101),
+    S("b3_ctx2047_sliding", B=3, ctx=2047, window=2048, use_rope=True, page_size=64, seed=102),
+    S("b5_ctx5000_sliding_v8_p1", B=5, L=8, ctx=5000, window=2048, use_rope=True, seed=103),
+    S("b4_ctx3000_full", B=4, ctx=3000, page_size=64, seed=104),
+    S("b8_ctx8192_full_mixed", B=8, ctx_range=(1, 8192), page_size=64, seed=105),
+    S("b3_ctx4000_sliding_v8_p1_s64", B=3, L=8, ctx=4000, window=2048, use_rope=True,
+      kv_scale=1 / 64, seed=106),
+    S("b2_ctx9000_full_s64", B=2, ctx=9000, page_size=64, kv_scale=1 / 64, seed=107),
+    S("b4_ctx6000_sliding_v8_p64", B=4, L=8, ctx=6000, window=2048, use_rope=True,
+      page_size=64, seed=108),
+    # edge cases
+    S("ctx0_and_1", B=3, seq_lens=[0, 1, 2], seed=110),
+    S("ctx0_verify", B=2, L=8, seq_lens=[0, 3], seed=111),
+    S("window1", B=2, seq_lens=[0, 500], window=1, use_rope=True, seed=112),
+    S("window_gt_ctx", B=2, L=8, seq_lens=[30, 700], window=5000, use_rope=True, seed=113),
+    S("ragged_pages", B=4, seq_lens=[63, 64, 65, 127], page_size=64, seed=114),
+    S("ragged_pages_v8", B=4, L=8, seq_lens=[56, 57, 63, 120], page_size=64, seed=115),
+    S("L3_block", B=3, L=3, seq_lens=[100, 1000, 64], seed=116),
+    S("many_requests", B=40, ctx_range=(0, 3000), seed=117),
+    S("many_requests_v8_sliding", B=40, L=8, ctx_range=(0, 5000), window=256, use_rope=True,
+      seed=118),
+    S("gate_std2_s64", B=2, L=8, ctx=1500, page_size=64, kv_scale=1 / 64, gate_std=2.0, seed=119),
+    S("spare_pages", B=2, seq_lens=[333, 777], page_size=64, spare_pages=5, seed=120),
+]
+
+
+def _check(inp, want=None, label=""):
+    gpu_out, gpu_k, gpu_v = H.run_gpu(inp)
+    ref = H.run_oracle(inp, want=want)
+    assert np.array_equal(gpu_k, ref.k_cache), f"{label}: k cache bytes differ"
+    assert np.array_equal(gpu_v, ref.v_cache), f"{label}: v cache bytes differ"
+    st = H.compare(gpu_out, ref, want)
+    assert st["ok"], f"{label}: {st}"
+    return st
+
+
+@pytest.mark.parametrize("spec", SMALL, ids=lambda s: s.name)
+def test_small_full_compare(spec, cuda_dev):
+    _check(W.make_inputs(spec), label=spec.name)
+
+
+def test_verify_full_ctx100k(cuda_dev):
+    # "batch 2, ctx 100000, heads tp8, layer full, q_len 8, page 1"
+    _check(W.make_inputs(S("b2_ctx100k_full_v8", B=2, L=8, ctx=100000, seed=121)))
+
+
+def test_long_ctx_1m_sampled(cuda_dev):
+    # "batch 1, ctx 1048576, heads tp8, layer full, q_len 8": sampled heads
+    inp = W.make_inputs(S("b1_ctx1m_full_v8", B=1, L=8, ctx=1048576, page_size=64, seed=122))
+    _check(inp, want=H.sample_want(8, 6, seed=1))
+
+
+FULL = ["pr1", "decode1_sliding", "decode1_full", "decode32_full", "decode32_sliding",
+        "verify16_sliding", "verify16_full", "paged_full", "paged_sliding"]
+SAMPLED = {"decode32_full": 24, "verify16_full": 24, "paged_full": 32}
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", FULL)
+def test_named_workloads(name, cuda_dev):
+    inp = W.make_inputs(W.named(name))
+    T = inp["B"] * inp["L"]
+    want = H.sample_want(T, SAMPLED[name], seed=3) if name in SAMPLED else None
+    _check(inp, want=want, label=name)
+
+
+def test_page_size_1_and_64_agree_bitwise(cuda_dev):
+    inp64 = W.make_inputs(S("p64", B=3, L=8, seq_lens=[70, 5, 700], page_size=64, seed=130))
+    pt64 = inp64["page_table"].numpy()
+    kc64 = inp64["k_cache"].reshape(-1, 128).numpy()
+    vc64 = inp64["v_cache"].reshape(-1, 128).numpy()
+    pos = inp64["positions"].numpy()
+    B, L = 3, 8
+    total = pos.reshape(B, L)[:, -1] + 1
+    perm = np.random.default_rng(5).permutation(int(total.sum()))
+    maxp = int((total.max() + 3) // 4 * 4)
+    pt1 = np.zeros((B, maxp), np.int32)
+    kc1 = np.zeros((perm.size, 128), np.uint8)
+    vc1 = np.zeros_like(kc1)
+    off = 0
+    for b in range(B):
+        for i in range(int(total[b])):
+            src = pt64[b, i // 64] * 64 + i % 64
+            pt1[b, i] = perm[off + i]
+            kc1[perm[off + i]] = kc64[src]
+            vc1[perm[off + i]] = vc64[src]
+        off += int(total[b])
+    inp1 = dict(inp64)
+    inp1.update(page_size=1, page_table=torch.from_numpy(pt1),
+                cache_loc=torch.from_numpy(pt1[np.repeat(np.arange(B), L), pos].astype(np.int64)),
+                k_cache=torch.from_numpy(kc1).view(-1, 1, 2, 64),
+                v_cache=torch.from_numpy(vc1).view(-1, 1, 2, 64))
+    o64, _, _ = H.run_gpu(inp64)
+    o1, _, _ = H.run_gpu(inp1)
+    assert np.array_equal(o64, o1)
+
+
+def test_repeatable_and_workspace_reuse(cuda_dev):
+    from paged_fp8_gated_b200 import binding
+    inp = W.make_inputs(S("rep", B=6, L=8, ctx_range=(100, 4000), seed=131))
+    ws = binding.alloc_workspace(6, 8)
+    ws.fill_(0xAB)                         # contents on entry must not matter
+    a = H.run_gpu(inp, workspace=ws)
+    b = H.run_gpu(inp, workspace=ws)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_graph_capture_replay_matches_eager(cuda_dev):
+    from paged_fp8_gated_b200 import binding
+    inp = W.make_inputs(S("graph", B=4, ctx_range=(500, 9000), seed=132))
+    d = H.to_device(inp)
+    k0, v0 = d["k_cache"].clone(), d["v_cache"].clone()
+    ws = binding.alloc_workspace(4, 1)
+    out = torch.empty(4, 1, 1024, dtype=torch.bfloat16, device="cuda")
+    args = (d["qkv"], d["positions"], d["seq_lens"], d["page_table"], d["cache_loc"],
+            d["k_cache"], d["v_cache"], d["k_scale_t"], d["v_scale_t"], 1, 0, False)
+    binding.attn_decode(*args, L=1, out=out, workspace=ws)
+    eager = out.clone()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        binding.attn_decode(*args, L=1, out=out, workspace=ws)  # warm up on the side stream
+        s.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            binding.attn_decode(*args, L=1, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    out.zero_()
+    d["k_cache"].copy_(k0)
+    d["v_cache"].copy_(v0)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager)
