@@ -46,6 +46,7 @@ extern "C" {
 #define GAD_ROW_BYTES 128  /* one cache row: 2 KV heads x 64 E4M3 codes */
 #define GAD_MAX_L 8        /* longest verify block           */
 #define GAD_MAX_B 4096     /* most requests in one call      */
+#define GAD_NOALLOC_SCRATCH_BYTES (16u << 20) /* built-in scratch of gad_attn_decode_noalloc */
 
 /* Return codes (0 = success). */
 typedef enum {
@@ -129,6 +130,37 @@ int gad_attn_decode_timed(const void* qkv, const int64_t* positions, const int32
                           int L, int max_pages, int64_t num_rows, int page_size, int window,
                           int use_rope, void* out, void* workspace, size_t workspace_bytes,
                           void* stream, void* const* events);
+
+/*
+ * Allocation-free variant of gad_attn_decode.  The page has no counterpart:
+ * this is a library convenience for callers that cannot provide device
+ * scratch memory, e.g. code inside a framework whose memory pool owns every
+ * device allocation, plugins that must not call cudaMalloc (it can
+ * synchronise the device and is refused while a graph capture is running),
+ * or plain C hosts with no device allocator.
+ *
+ * Same arguments and results as gad_attn_decode, minus the workspace: the
+ * step's scratch is a fixed device array of GAD_NOALLOC_SCRATCH_BYTES
+ * (16 MiB) inside the library, which every GPU that loads the library holds
+ * until the process exits.  The caller still passes all inputs and outputs.
+ *   - Sizes whose scratch (gad_attn_workspace_bytes(B, L)) exceeds 16 MiB are
+ *     rejected with GAD_ERR_WORKSPACE before anything is launched; on a
+ *     148-SM B200 that admits L = 1 steps up to B = 2474 and L = 8 steps up
+ *     to B = 135 (use gad_attn_decode beyond that).
+ *   - It never allocates (no cudaMalloc, cudaFree or allocating library
+ *     call).  The first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress) with that device current and caches it;
+ *     make that first call before any stream capture on that device.
+ *   - Every call on a device shares the one array.  Nothing in it needs to
+ *     start at zero (each call writes every scratch byte it later reads), but
+ *     calls that overlap on the GPU (different streams, or graphs replayed
+ *     concurrently) race on it and give wrong results: serialise them.
+ */
+int gad_attn_decode_noalloc(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                            const int32_t* page_table, const int64_t* cache_loc,
+                            uint8_t* k_cache, uint8_t* v_cache, const float* k_scale,
+                            const float* v_scale, int B, int L, int max_pages, int64_t num_rows,
+                            int page_size, int window, int use_rope, void* out, void* stream);
 
 /* Message for the last nonzero status returned on this host thread. */
 const char* gad_last_error(void);

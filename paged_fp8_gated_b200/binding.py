@@ -34,6 +34,8 @@ _lib.gad_attn_decode.argtypes = [
     _vp, _vp, ctypes.c_size_t, _vp]                         # out, workspace, bytes, stream
 _lib.gad_attn_decode_timed.restype = ctypes.c_int
 _lib.gad_attn_decode_timed.argtypes = list(_lib.gad_attn_decode.argtypes) + [_vp]
+_lib.gad_attn_decode_noalloc.restype = ctypes.c_int
+_lib.gad_attn_decode_noalloc.argtypes = list(_lib.gad_attn_decode.argtypes[:17]) + [_vp]
 _lib.gad_last_error.restype = ctypes.c_char_p
 _lib.gad_last_error.argtypes = []
 _lib.gad_status_string.restype = ctypes.c_char_p
@@ -42,8 +44,9 @@ _lib.gad_status_string.argtypes = [ctypes.c_int]
 HQ, HKV, D = 16, 2, 64
 QKV_COLS, OUT_COLS, ROW_BYTES = 2304, 1024, 128
 
-EXPORTED = ("gad_attn_decode", "gad_attn_decode_timed", "gad_attn_workspace_bytes",
-            "gad_last_error", "gad_status_string")
+EXPORTED = ("gad_attn_decode", "gad_attn_decode_timed", "gad_attn_decode_noalloc",
+            "gad_attn_workspace_bytes", "gad_last_error", "gad_status_string")
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class GadError(RuntimeError):
@@ -148,6 +151,38 @@ def attn_decode(qkv: torch.Tensor, positions: torch.Tensor, seq_lens: torch.Tens
         st = _lib.gad_attn_decode_timed(*args, arr)
     if st != 0:
         raise GadError(st, "gad_attn_decode")
+    return out
+
+
+def attn_decode_noalloc(qkv: torch.Tensor, positions: torch.Tensor,
+                        seq_lens: torch.Tensor | None, page_table: torch.Tensor,
+                        cache_loc: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                        k_scale: torch.Tensor, v_scale: torch.Tensor, page_size: int, window: int,
+                        use_rope: bool, L: int = 1, out: torch.Tensor | None = None,
+                        stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """The step through gad_attn_decode_noalloc: no workspace argument, the library's
+    built-in 16 MiB device scratch is used instead (for callers that cannot allocate
+    device memory themselves).  Calls on one device must not overlap on the GPU."""
+    for t, n, dt in ((qkv, "qkv", torch.bfloat16), (positions, "positions", torch.int64),
+                     (page_table, "page_table", torch.int32), (cache_loc, "cache_loc", torch.int64),
+                     (k_cache, "k_cache", torch.uint8), (v_cache, "v_cache", torch.uint8),
+                     (k_scale, "k_scale", torch.float32), (v_scale, "v_scale", torch.float32)):
+        _need(t, n, dt)
+    B, max_pages = page_table.shape
+    T = qkv.shape[0]
+    if qkv.shape[1] != QKV_COLS or T != B * L:
+        raise ValueError(f"qkv must be [B*L={B * L}, {QKV_COLS}], got {tuple(qkv.shape)}")
+    num_rows = k_cache.numel() // ROW_BYTES
+    if out is None:
+        out = torch.empty(B, L, OUT_COLS, dtype=torch.bfloat16, device=qkv.device)
+    s = (stream or torch.cuda.current_stream(qkv.device)).cuda_stream
+    st = _lib.gad_attn_decode_noalloc(
+        _ptr(qkv), _ptr(positions), _ptr(seq_lens), _ptr(page_table), _ptr(cache_loc),
+        _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), int(B), int(L),
+        int(max_pages), int(num_rows), int(page_size), int(window), int(bool(use_rope)),
+        _ptr(out), ctypes.c_void_p(s))
+    if st != 0:
+        raise GadError(st, "gad_attn_decode_noalloc")
     return out
 
 

@@ -283,3 +283,61 @@ int gad_attn_decode_timed(const void* qkv, const int64_t* positions, const int32
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant.
+//
+// Some callers cannot hand the library a device workspace: code running
+// inside a framework whose memory pool owns every device allocation, plugins
+// that may not call cudaMalloc (which can synchronise the device and is not
+// allowed while another thread captures a CUDA graph), and plain C hosts with
+// no device allocator of their own.  For them the step's scratch lives in one
+// fixed, file-scope device array that the library carries.  Every GPU that
+// loads this library holds GAD_NOALLOC_SCRATCH_BYTES of it until the process
+// exits.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[GAD_NOALLOC_SCRATCH_BYTES];
+
+static std::atomic<void*> g_noalloc_addr[kMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+static int noalloc_scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", dev);
+    void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return fail(GAD_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+        g_noalloc_addr[dev].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return GAD_OK;
+}
+
+extern "C" int gad_attn_decode_noalloc(const void* qkv, const int64_t* positions,
+                                       const int32_t* seq_lens, const int32_t* page_table,
+                                       const int64_t* cache_loc, uint8_t* k_cache,
+                                       uint8_t* v_cache, const float* k_scale,
+                                       const float* v_scale, int B, int L, int max_pages,
+                                       int64_t num_rows, int page_size, int window, int use_rope,
+                                       void* out, void* stream) {
+    (void)seq_lens;
+    const size_t need = gad_attn_workspace_bytes(B, L);
+    if (need == 0) return B < 1 || B > GAD_MAX_B || L < 1 || L > GAD_MAX_L ? GAD_ERR_SHAPE : GAD_ERR_CUDA;
+    if (need > static_cast<size_t>(GAD_NOALLOC_SCRATCH_BYTES))
+        return fail(GAD_ERR_WORKSPACE,
+                    "B=%d, L=%d needs %zu B of scratch but the built-in scratch holds %zu B; "
+                    "call gad_attn_decode with a caller workspace instead",
+                    B, L, need, static_cast<size_t>(GAD_NOALLOC_SCRATCH_BYTES));
+    void* scratch = nullptr;
+    const int st = noalloc_scratch_address(&scratch);
+    if (st != GAD_OK) return st;
+    return run_step(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale, B,
+                    L, max_pages, num_rows, page_size, window, use_rope, out, scratch,
+                    static_cast<size_t>(GAD_NOALLOC_SCRATCH_BYTES), stream, nullptr);
+}
