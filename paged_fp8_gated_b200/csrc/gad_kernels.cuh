@@ -37,7 +37,7 @@ constexpr int TILE = 64;                    // keys per pipeline stage
 constexpr int STAGE_BYTES = 2 * TILE * ROWB;  // K tile then V tile: 16 KB
 constexpr int DEC_THREADS = 256;
 constexpr int PREP_THREADS = (HQ + HKV) * 32;
-constexpr int COMB_THREADS = HQ * 32;
+constexpr int COMB_THREADS = 256;
 
 struct StepParams {
     const __nv_bfloat16* qkv;
@@ -55,9 +55,17 @@ struct StepParams {
     __half* q_ws;    // [T][16][64]  normalised (rotated) queries
     float* part_o;   // [slots][lt][16][64]  un-normalised partial outputs
     float* part_ml;  // [slots][lt][16][2]   (running max in log2 units, sum)
-    int* meta;       // [0] total tiles, [1] tiles per CTA, [2 .. 2+B] tile prefix
+    int* meta;       // see META_*: tile count, tiles per CTA, error word, tile prefix
     int lt;          // token capacity of one partial slot (1 or 8)
+    int tl;          // tile lanes: partials per (CTA, request) and KV-head group
 };
+
+// Layout of StepParams::meta (ints).
+constexpr int META_TOTAL = 0;    // tiles in the step
+constexpr int META_PER = 1;      // tiles per CTA
+constexpr int META_ERROR = 2;    // nonzero: a bounded wait in the decode kernel timed out
+constexpr int META_PREFIX = 3;   // [B + 1] tile prefix over requests
+constexpr int META_INTS = 4;     // + B
 
 // ---------------------------------------------------------------------------
 // Kernel 1: split + QK-norm + RoPE + E4M3 quantise-and-scatter.
@@ -70,6 +78,7 @@ struct StepParams {
 __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) {
     pdl_launch_dependents();
     const int t = blockIdx.x;
+    if (t == 0 && threadIdx.x == 0) p.meta[META_ERROR] = 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const __nv_bfloat16* row = p.qkv + static_cast<size_t>(t) * QKV_COLS;
     const bool is_q = warp < HQ;
@@ -151,6 +160,57 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) 
 // runs its own online softmax over its keys; key groups are merged in shared
 // memory at the end of each segment.
 // ---------------------------------------------------------------------------
+// Per-request key ranges [lo_b, hi_b] (union over the request's tokens), the
+// prefix of 64-key tile counts over requests, and this CTA's share of the tile
+// list [t0, t1).  Every thread of the block must call it.  CTA 0 also writes the
+// list to the workspace for the combine kernel.
+__device__ __forceinline__ void build_tile_list(const StepParams& p, int* tpre, int* rlo, int* rhi,
+                                                int nthreads, int& total, int& per, int& t0,
+                                                int& t1) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int B = p.B, L = p.L;
+    for (int b = tid; b < B; b += nthreads) {
+        int lo = INT_MAX, hi = -1;
+        for (int j = 0; j < L; ++j) {
+            const int pos = static_cast<int>(p.positions[static_cast<size_t>(b) * L + j]);
+            const int l = p.window > 0 ? max(0, pos - p.window + 1) : 0;
+            lo = min(lo, l);
+            hi = max(hi, pos);
+        }
+        rlo[b] = lo;
+        rhi[b] = hi;
+        tpre[b + 1] = (hi >= lo && hi >= 0) ? (hi / TILE - lo / TILE + 1) : 0;
+    }
+    if (tid == 0) tpre[0] = 0;
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        for (int base = 1; base <= B; base += 32) {
+            const int i = base + lane;
+            int v = i <= B ? tpre[i] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += n;
+            }
+            if (i <= B) tpre[i] = v + carry;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    __syncthreads();
+    total = tpre[B];
+    per = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+    t0 = static_cast<int>(blockIdx.x) * per;
+    t1 = min(t0 + per, total);
+    if (blockIdx.x == 0) {
+        for (int i = tid; i <= B; i += nthreads) p.meta[META_PREFIX + i] = tpre[i];
+        if (tid == 0) {
+            p.meta[META_TOTAL] = total;
+            p.meta[META_PER] = per;
+        }
+    }
+}
+
 template <int LT, int KG, int NS>
 struct DecodeCfg {
     static constexpr int WARPS = DEC_THREADS / 32;
@@ -198,46 +258,8 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
     const int B = p.B, L = p.L;
 
     // ---- request key ranges and the tile list (reads inputs only) ----
-    for (int b = tid; b < B; b += DEC_THREADS) {
-        int lo = INT_MAX, hi = -1;
-        for (int j = 0; j < L; ++j) {
-            const int pos = static_cast<int>(p.positions[static_cast<size_t>(b) * L + j]);
-            const int l = p.window > 0 ? max(0, pos - p.window + 1) : 0;
-            lo = min(lo, l);
-            hi = max(hi, pos);
-        }
-        rlo[b] = lo;
-        rhi[b] = hi;
-        tpre[b + 1] = (hi >= lo && hi >= 0) ? (hi / TILE - lo / TILE + 1) : 0;
-    }
-    if (tid == 0) tpre[0] = 0;
-    __syncthreads();
-    if (warp == 0) {
-        int carry = 0;
-        for (int base = 1; base <= B; base += 32) {
-            const int i = base + lane;
-            int v = i <= B ? tpre[i] : 0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += n;
-            }
-            if (i <= B) tpre[i] = v + carry;
-            carry += __shfl_sync(0xffffffffu, v, 31);
-        }
-    }
-    __syncthreads();
-    const int total = tpre[B];
-    const int per = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
-    const int t0 = static_cast<int>(blockIdx.x) * per;
-    const int t1 = min(t0 + per, total);
-    if (blockIdx.x == 0) {
-        for (int i = tid; i <= B; i += DEC_THREADS) p.meta[2 + i] = tpre[i];
-        if (tid == 0) {
-            p.meta[0] = total;
-            p.meta[1] = per;
-        }
-    }
+    int total, per, t0, t1;
+    build_tile_list(p, tpre, rlo, rhi, DEC_THREADS, total, per, t0, t1);
     // q and this step's cache rows come from the prep kernel
     pdl_wait_primary();
     if (t0 >= t1) return;
@@ -518,7 +540,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
             __syncthreads();
         }
         if (kg == 0) {
-            const size_t slot = static_cast<size_t>(blockIdx.x) + b;
+            const size_t slot = (static_cast<size_t>(blockIdx.x) + b) * p.tl;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int j = rg * NT + nt;
@@ -583,48 +605,97 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
 
 // ---------------------------------------------------------------------------
 // Kernel 3: merge the partials of each (token, head) and apply the gated
-// output norm.  One block per token, one warp per head, two dims per lane.
+// output norm.  One block per (token, head).  A request covered by many CTAs
+// has many partial slots (a single 80K-key request spreads over ~300), so the
+// slots are read in parallel: thread (sl, dq) accumulates dims 4dq..4dq+3 over
+// slots sl, sl+16, ..., then the 16 slot lanes are summed in shared memory.
 // ---------------------------------------------------------------------------
+constexpr int COMB_SLOT_LANES = 16;
+
 __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams p) {
     pdl_wait_primary();
-    const int t = blockIdx.x;
-    const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ float red_o[COMB_SLOT_LANES][HD];
+    __shared__ float red_l[COMB_SLOT_LANES];
+    __shared__ float red_m[COMB_THREADS / 32];
+    __shared__ float red_ss[4];
+    const int t = blockIdx.x / HQ, h = blockIdx.x % HQ;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = t / p.L, j = t % p.L;
-    const int tp = p.meta[2 + b];
-    const int n = p.meta[3 + b] - tp;
-    const int per = p.meta[1];
-    const int d0 = 2 * lane;
-    float y0 = NAN, y1 = NAN;
-    if (n > 0 && per > 0) {
-        const int c_lo = tp / per, c_hi = (tp + n - 1) / per;
-        float M = -INFINITY;
-        for (int c = c_lo; c <= c_hi; ++c) {
-            const size_t base = (static_cast<size_t>(c + b) * p.lt + j) * HQ + h;
-            M = fmaxf(M, p.part_ml[base * 2]);
-        }
-        float l = 0.f, o0 = 0.f, o1 = 0.f;
-        for (int c = c_lo; c <= c_hi; ++c) {
-            const size_t base = (static_cast<size_t>(c + b) * p.lt + j) * HQ + h;
-            const float ms = p.part_ml[base * 2], ls = p.part_ml[base * 2 + 1];
-            const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-            const float2 o = *reinterpret_cast<const float2*>(p.part_o + base * HD + d0);
-            l += w * ls;
-            o0 += w * o.x;
-            o1 += w * o.y;
-        }
-        const float vs = __ldg(p.v_scale);
-        const float a0 = o0 / l * vs, a1 = o1 / l * vs;
-        float ss = a0 * a0 + a1 * a1;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float rinv = 1.0f / sqrtf(ss * (1.0f / 64.0f) + 1e-6f);
-        const __nv_bfloat16* gate = p.qkv + static_cast<size_t>(t) * QKV_COLS + G_OFF + h * HD + d0;
-        const float g0 = __bfloat162float(gate[0]), g1 = __bfloat162float(gate[1]);
-        y0 = a0 * rinv / (1.0f + expf(-g0));
-        y1 = a1 * rinv / (1.0f + expf(-g1));
+    const int tp = p.meta[META_PREFIX + b];
+    const int n = p.meta[META_PREFIX + b + 1] - tp;
+    const int per = p.meta[META_PER];
+    __nv_bfloat16* outp = p.out + static_cast<size_t>(t) * OUT_COLS + h * HD;
+    if (n <= 0 || per <= 0) {  // no key in range (positions outside the contract)
+        if (tid < HD) outp[tid] = __float2bfloat16(NAN);
+        return;
     }
-    *reinterpret_cast<__nv_bfloat162*>(p.out + static_cast<size_t>(t) * OUT_COLS + h * HD + d0) =
-        __floats2bfloat162_rn(y0, y1);
+    const int c_lo = tp / per, c_hi = (tp + n - 1) / per;
+    const int TL = p.tl;
+    const int ns = (c_hi - c_lo + 1) * TL;
+    // Partial s = (CTA c_lo + s / TL, tile lane s % TL).  Tile lane tl of CTA c
+    // holds a partial for this request only if one of the request's tiles in
+    // CTA c's share has a local index congruent to tl modulo TL.
+    auto slot_base = [&](int s) {
+        const int c = c_lo + s / TL, tl = s % TL;
+        return ((static_cast<size_t>(c + b) * TL + tl) * p.lt + j) * HQ + h;
+    };
+    auto slot_used = [&](int s) {
+        const int c = c_lo + s / TL, tl = s % TL;
+        const int i0 = max(tp, c * per) - c * per;
+        const int i1 = min(tp + n, (c + 1) * per) - c * per;
+        const int cnt = i1 - i0;
+        return cnt >= TL || (((tl - i0) % TL + TL) % TL) < cnt;
+    };
+    // 1. global max over the slots
+    float mx = -INFINITY;
+    for (int s = tid; s < ns; s += COMB_THREADS)
+        if (slot_used(s)) mx = fmaxf(mx, p.part_ml[slot_base(s) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red_m[warp] = mx;
+    __syncthreads();
+    float M = red_m[0];
+#pragma unroll
+    for (int w = 1; w < COMB_THREADS / 32; ++w) M = fmaxf(M, red_m[w]);
+    // 2. weighted sums: thread (sl, dq) over slots sl, sl + 16, ...
+    const int sl = tid / 16, dq = tid % 16;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lsum = 0.f;
+    for (int s = sl; s < ns; s += COMB_SLOT_LANES) {
+        if (!slot_used(s)) continue;
+        const size_t base = slot_base(s);
+        const float ms = p.part_ml[base * 2];
+        if (ms == -INFINITY) continue;
+        const float w = exp2f(ms - M);
+        const float4 o = *reinterpret_cast<const float4*>(p.part_o + base * HD + 4 * dq);
+        acc.x += w * o.x;
+        acc.y += w * o.y;
+        acc.z += w * o.z;
+        acc.w += w * o.w;
+        lsum += w * p.part_ml[base * 2 + 1];
+    }
+    *reinterpret_cast<float4*>(&red_o[sl][4 * dq]) = acc;
+    if (dq == 0) red_l[sl] = lsum;
+    __syncthreads();
+    // 3. threads 0..63: one output dim each
+    if (tid < HD) {
+        float o = 0.f, l = 0.f;
+#pragma unroll
+        for (int k = 0; k < COMB_SLOT_LANES; ++k) {
+            o += red_o[k][tid];
+            l += red_l[k];
+        }
+        const float a = o / l * __ldg(p.v_scale);
+        float ss = a * a;
+#pragma unroll
+        for (int q = 16; q > 0; q >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, q);
+        if (lane == 0) red_ss[warp] = ss;
+        asm volatile("bar.sync 1, 64;\n" ::: "memory");
+        const float tot = red_ss[0] + red_ss[1];
+        const float rinv = 1.0f / sqrtf(tot * (1.0f / 64.0f) + 1e-6f);
+        const float g = __bfloat162float(p.qkv[static_cast<size_t>(t) * QKV_COLS + G_OFF + h * HD + tid]);
+        outp[tid] = __float2bfloat16(a * rinv / (1.0f + expf(-g)));
+    }
 }
 
 }  // namespace gad

@@ -160,6 +160,11 @@ def named(name: str, seed: int = 0) -> Spec:
                               seed=seed + 2),
         "decode32_sliding": Spec("decode32_sliding", B=32, L=1, ctx_range=(40000, 80000),
                                  window=2048, use_rope=True, seed=seed + 21),
+        # diagnostics for the gather pattern: same step with sequential rows, or 64-key pages
+        "decode32_full_seq": Spec("decode32_full_seq", B=32, L=1, ctx_range=(40000, 80000),
+                                  permute=False, seed=seed + 2),
+        "decode32_full_p64": Spec("decode32_full_p64", B=32, L=1, ctx_range=(40000, 80000),
+                                  page_size=64, seed=seed + 2),
         # 16 requests, 8-token causal verify blocks at 80,000 cached keys
         "verify16_sliding": Spec("verify16_sliding", B=16, L=8, ctx=80000, window=2048,
                                  use_rope=True, seed=seed + 31),

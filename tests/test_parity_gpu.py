@@ -41,6 +41,10 @@ SMALL = [
       seed=118),
     S("gate_std2_s64", B=2, L=8, ctx=1500, page_size=64, kv_scale=1 / 64, gate_std=2.0, seed=119),
     S("spare_pages", B=2, seq_lens=[333, 777], page_size=64, spare_pages=5, seed=120),
+    # more requests than the single-token kernel keeps tables for (other kernel)
+    S("b1100_decode_p1", B=1100, ctx_range=(0, 300), seed=123),
+    S("b1100_decode_p64_sliding", B=1100, ctx_range=(0, 400), window=100, use_rope=True,
+      page_size=64, seed=124),
 ]
 
 
