@@ -145,8 +145,8 @@ int gad_attn_decode_timed(const void* qkv, const int64_t* positions, const int32
  * until the process exits.  The caller still passes all inputs and outputs.
  *   - Sizes whose scratch (gad_attn_workspace_bytes(B, L)) exceeds 16 MiB are
  *     rejected with GAD_ERR_WORKSPACE before anything is launched; on a
- *     148-SM B200 that admits L = 1 steps with B <= 753 or 1025 <= B <= 2474
- *     and L = 8 steps up to B = 135 (use gad_attn_decode beyond that).
+ *     148-SM B200 that admits L = 1 steps up to B = 621 and L = 8 steps up to
+ *     B = 135 (use gad_attn_decode beyond that).
  *   - It never allocates (no cudaMalloc, cudaFree or allocating library
  *     call).  The first call on each device looks up the array's device
  *     address (cudaGetSymbolAddress) with that device current and caches it;

@@ -2,9 +2,13 @@
 // the three launches (prep -> decode -> combine, chained with programmatic
 // dependent launch so each kernel's launch latency hides behind the previous
 // kernel's tail).
-#include <cuda.h>
+//
+// Decode kernel choice (measured on B200, decode-32 full attention, KV 463 MB):
+// cp.async gathers from every warp of two CTAs per SM into 128-key stages run
+// at 76.6% (page size 1) / 78.8% (page size 64) of the measured HBM copy rate;
+// a warp-specialised variant with one producer warp issuing 2D TMA page loads
+// reached 64%, and producer-warp cp.async gathers about 55%.
 #include <cuda_runtime.h>
-#include <cudaTypedefs.h>
 
 #include <atomic>
 #include <cstdarg>
@@ -13,7 +17,6 @@
 #include <string>
 
 #include "gad_attn.h"
-#include "gad_decode2.cuh"
 #include "gad_kernels.cuh"
 
 namespace {
@@ -36,46 +39,27 @@ constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Kernel choice per step (shapes only):
-//   L == 1, page size 64, B <= kDecode2MaxB   decode2_kernel (TMA pages, one CTA
-//                                            per SM, kDecode2TileLanes partials
-//                                            per CTA and request)
-//   everything else                          decode_kernel (cp.async gathers, up
-//                                            to kMaxCtasPerSm CTAs per SM, one
-//                                            merged partial per CTA and request)
-#ifndef GAD_D2_TILE_LANES
-#define GAD_D2_TILE_LANES 4
-#endif
-#ifndef GAD_D2_STAGES
-#define GAD_D2_STAGES 10
-#endif
-#ifndef GAD_V1_STAGES
-#define GAD_V1_STAGES 4
-#endif
-constexpr int kDecode2TileLanes = GAD_D2_TILE_LANES;
-constexpr int kDecode2Stages = GAD_D2_STAGES;
-constexpr int kDecode2MaxB = 1024;  // its per-request tables live in shared memory
-
-bool use_decode2(int B, int L, int page_size) {
-    return L == 1 && page_size == 64 && B <= kDecode2MaxB;
-}
+// decode_kernel configurations: (tokens, key groups, stages, CTAs per SM, keys
+// per stage, merge key groups in the CTA)
+//   single-token steps: 128-key stages, 3 of them, two CTAs per SM (so 128 KB of
+//   loads in flight per SM); each key group writes its own partial (no merge
+//   buffer, so the stages fit)
+//   verify blocks:      64-key stages, 4 of them, one CTA per SM, merged
+constexpr int kV1SingleKG = 4, kV1SingleNS = 3, kV1SingleTK = 128;
+constexpr int kV1VerifyKG = 2, kV1VerifyNS = 4, kV1VerifyTK = 64;
 
 struct WsLayout {
     size_t q_off, po_off, pml_off, meta_off, total;
     int lt;
 };
 
-// One layout serves both kernels of a shape (the page size is not an argument
-// of gad_attn_workspace_bytes): partial units = max over the kernels of
-// (CTAs + B) * partials per (CTA, request).
+// Partial slots: (CTAs + B) * partials per (CTA, request), each holding lt
+// tokens x 16 heads x (64 values + max + sum).
 WsLayout ws_layout(int B, int L, int sms) {
     WsLayout w{};
     w.lt = L == 1 ? 1 : GAD_MAX_L;
-    size_t units = static_cast<size_t>(sms) * kMaxCtasPerSm + B;
-    if (L == 1 && B <= kDecode2MaxB) {
-        const size_t u2 = (static_cast<size_t>(sms) + B) * kDecode2TileLanes;
-        if (u2 > units) units = u2;
-    }
+    const size_t units =
+        (static_cast<size_t>(sms) * kMaxCtasPerSm + B) * (L == 1 ? kV1SingleKG : 1);
     const size_t T = static_cast<size_t>(B) * L;
     const size_t parts = units * w.lt * GAD_HQ;
     size_t off = 0;
@@ -91,77 +75,6 @@ WsLayout ws_layout(int B, int L, int sms) {
     return w;
 }
 
-cudaLaunchAttribute pdl_attr() {
-    cudaLaunchAttribute a;
-    std::memset(&a, 0, sizeof(a));
-    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    a.val.programmaticStreamSerializationAllowed = 1;
-    return a;
-}
-
-// 2D tensor map over a cache viewed as [num_rows, 128] bytes, box 64 rows x 128
-// bytes (one 64-key page), 128-byte swizzle, zero fill out of bounds.
-int make_page_map(CUtensorMap* map, const uint8_t* base, int64_t num_rows) {
-    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-    if (encode == nullptr) {
-        void* fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
-            return fail(GAD_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
-        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    }
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(GAD_ROW_BYTES), static_cast<cuuint64_t>(num_rows)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(GAD_ROW_BYTES)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(GAD_ROW_BYTES), static_cast<cuuint32_t>(gad::TILE)};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(GAD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-    return GAD_OK;
-}
-
-int launch_decode2(const gad::StepParams& prm, int sms, int tiles_upper, cudaStream_t stream,
-                   bool pdl) {
-    constexpr int PS = 64, NS = kDecode2Stages;
-    using C = gad::Decode2Cfg<PS, kDecode2TileLanes, NS>;
-    auto kern = gad::decode2_kernel<PS, kDecode2TileLanes, NS>;
-    static std::atomic<bool> attr_done[kMaxDevices];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", dev);
-    if (!attr_done[dev].load(std::memory_order_acquire)) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(C::smem_bytes(kDecode2MaxB)));
-        if (e != cudaSuccess)
-            return fail(GAD_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        attr_done[dev].store(true, std::memory_order_release);
-    }
-    CUtensorMap mk, mv;
-    int st = make_page_map(&mk, prm.k_cache, prm.num_rows);
-    if (st != GAD_OK) return st;
-    st = make_page_map(&mv, prm.v_cache, prm.num_rows);
-    if (st != GAD_OK) return st;
-    long long grid = sms;
-    if (grid > tiles_upper) grid = tiles_upper;
-    if (grid < 1) grid = 1;
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(C::THREADS);
-    cfg.dynamicSmemBytes = C::smem_bytes(prm.B);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr = pdl_attr();
-    cfg.attrs = &attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kern, prm, mk, mv);
-    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-    return GAD_OK;
-}
-
 int current_device_sms(int* sms, int* major) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -175,12 +88,19 @@ int current_device_sms(int* sms, int* major) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+cudaLaunchAttribute pdl_attr() {
+    cudaLaunchAttribute a;
+    std::memset(&a, 0, sizeof(a));
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+    return a;
+}
 
-template <int LT, int PS, int KG, int NS, int MINB>
+template <int LT, int PS, int KG, int NS, int MINB, int TK, bool MERGE>
 int launch_decode(const gad::StepParams& prm, int sms, int tiles_upper, cudaStream_t stream,
                   bool pdl) {
-    using C = gad::DecodeCfg<LT, KG, NS>;
-    auto kern = gad::decode_kernel<LT, PS, KG, NS, MINB>;
+    using C = gad::DecodeCfg<LT, KG, NS, TK, MERGE>;
+    auto kern = gad::decode_kernel<LT, PS, KG, NS, MINB, TK, MERGE>;
     const size_t smem = C::smem_bytes(prm.B);
     // Raise the kernel's dynamic shared-memory limit once per device, to the
     // largest size any B needs, so no attribute call happens during capture.
@@ -307,7 +227,7 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     prm.part_ml = reinterpret_cast<float*>(ws + w.pml_off);
     prm.meta = reinterpret_cast<int*>(ws + w.meta_off);
     prm.lt = w.lt;
-    prm.tl = use_decode2(B, L, page_size) ? kDecode2TileLanes : 1;
+    prm.tl = L == 1 ? kV1SingleKG : 1;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int T = B * L;
@@ -330,14 +250,14 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
     if (timed) cudaEventRecord(static_cast<cudaEvent_t>(events[1]), s);
 
-    if (use_decode2(B, L, page_size)) {
-        st = launch_decode2(prm, sms, tiles_upper, s, !timed);
-    } else if (L == 1) {
-        st = page_size == 1 ? launch_decode<1, 1, 4, GAD_V1_STAGES, 2>(prm, sms, tiles_upper, s, !timed)
-                            : launch_decode<1, 64, 4, GAD_V1_STAGES, 2>(prm, sms, tiles_upper, s, !timed);
+    if (L == 1) {
+        st = page_size == 1
+                 ? launch_decode<1, 1, kV1SingleKG, kV1SingleNS, 2, kV1SingleTK, false>(prm, sms, tiles_upper, s, !timed)
+                 : launch_decode<1, 64, kV1SingleKG, kV1SingleNS, 2, kV1SingleTK, false>(prm, sms, tiles_upper, s, !timed);
     } else {
-        st = page_size == 1 ? launch_decode<8, 1, 2, 4, 1>(prm, sms, tiles_upper, s, !timed)
-                            : launch_decode<8, 64, 2, 4, 1>(prm, sms, tiles_upper, s, !timed);
+        st = page_size == 1
+                 ? launch_decode<8, 1, kV1VerifyKG, kV1VerifyNS, 1, kV1VerifyTK, true>(prm, sms, tiles_upper, s, !timed)
+                 : launch_decode<8, 64, kV1VerifyKG, kV1VerifyNS, 1, kV1VerifyTK, true>(prm, sms, tiles_upper, s, !timed);
     }
     if (st != GAD_OK) return st;
     if (timed) cudaEventRecord(static_cast<cudaEvent_t>(events[2]), s);
@@ -345,12 +265,17 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>(T) * gad::HQ);
-    cfg.blockDim = dim3(gad::COMB_THREADS);
     cfg.stream = s;
     cudaLaunchAttribute attr = pdl_attr();
     cfg.attrs = &attr;
     cfg.numAttrs = timed ? 0 : 1;
-    e = cudaLaunchKernelEx(&cfg, gad::combine_kernel, prm);
+    if (T <= 16) {
+        cfg.blockDim = dim3(1024);
+        e = cudaLaunchKernelEx(&cfg, gad::combine_kernel<1024>, prm);
+    } else {
+        cfg.blockDim = dim3(256);
+        e = cudaLaunchKernelEx(&cfg, gad::combine_kernel<256>, prm);
+    }
     if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
     if (timed) {
         e = cudaEventRecord(static_cast<cudaEvent_t>(events[3]), s);

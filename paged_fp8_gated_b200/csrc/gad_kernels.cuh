@@ -37,7 +37,6 @@ constexpr int TILE = 64;                    // keys per pipeline stage
 constexpr int STAGE_BYTES = 2 * TILE * ROWB;  // K tile then V tile: 16 KB
 constexpr int DEC_THREADS = 256;
 constexpr int PREP_THREADS = (HQ + HKV) * 32;
-constexpr int COMB_THREADS = 256;
 
 struct StepParams {
     const __nv_bfloat16* qkv;
@@ -57,7 +56,7 @@ struct StepParams {
     float* part_ml;  // [slots][lt][16][2]   (running max in log2 units, sum)
     int* meta;       // see META_*: tile count, tiles per CTA, error word, tile prefix
     int lt;          // token capacity of one partial slot (1 or 8)
-    int tl;          // tile lanes: partials per (CTA, request) and KV-head group
+    int tl;          // partials per (CTA, request) and KV-head group
 };
 
 // Layout of StepParams::meta (ints).
@@ -161,9 +160,10 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) 
 // memory at the end of each segment.
 // ---------------------------------------------------------------------------
 // Per-request key ranges [lo_b, hi_b] (union over the request's tokens), the
-// prefix of 64-key tile counts over requests, and this CTA's share of the tile
+// prefix of TK-key tile counts over requests (tiles aligned to multiples of TK), and this CTA's share of the tile
 // list [t0, t1).  Every thread of the block must call it.  CTA 0 also writes the
 // list to the workspace for the combine kernel.
+template <int TK>
 __device__ __forceinline__ void build_tile_list(const StepParams& p, int* tpre, int* rlo, int* rhi,
                                                 int nthreads, int& total, int& per, int& t0,
                                                 int& t1) {
@@ -179,7 +179,7 @@ __device__ __forceinline__ void build_tile_list(const StepParams& p, int* tpre, 
         }
         rlo[b] = lo;
         rhi[b] = hi;
-        tpre[b + 1] = (hi >= lo && hi >= 0) ? (hi / TILE - lo / TILE + 1) : 0;
+        tpre[b + 1] = (hi >= lo && hi >= 0) ? (hi / TK - lo / TK + 1) : 0;
     }
     if (tid == 0) tpre[0] = 0;
     __syncthreads();
@@ -211,24 +211,28 @@ __device__ __forceinline__ void build_tile_list(const StepParams& p, int* tpre, 
     }
 }
 
-template <int LT, int KG, int NS>
+template <int LT, int KG, int NS, int TK, bool MERGE>
 struct DecodeCfg {
     static constexpr int WARPS = DEC_THREADS / 32;
     static constexpr int RG = WARPS / (HKV * KG);
     static constexpr int NT = LT / RG;              // tokens per warp (MMA N tiles)
-    static constexpr int MT = (TILE / 16) / KG;     // 16-key groups per warp per tile
+    static constexpr int MT = (TK / 16) / KG;       // 16-key groups per warp per tile
+    static constexpr int STAGE = 2 * TK * ROWB;     // K tile then V tile
     static constexpr int IDX_SLOTS = 2 * NS;
-    static constexpr int MERGE_WARPS = (KG - 1) * HKV * RG;
+    static constexpr int MERGE_WARPS = MERGE ? (KG - 1) * HKV * RG : 0;
     static constexpr int MERGE_FLOATS_PER_WARP = NT * 32 * 20;
-    static constexpr size_t KV_BYTES = static_cast<size_t>(NS) * STAGE_BYTES;
-    static constexpr size_t IDX_BYTES = static_cast<size_t>(IDX_SLOTS) * TILE * 4;
+    // partials per (CTA, request): one after the in-CTA merge, else one per key group
+    static constexpr int PARTS = MERGE ? 1 : KG;
+    static constexpr size_t KV_BYTES = static_cast<size_t>(NS) * STAGE;
+    static constexpr size_t IDX_BYTES = static_cast<size_t>(IDX_SLOTS) * TK * 4;
     static constexpr size_t MERGE_BYTES =
         static_cast<size_t>(MERGE_WARPS) * MERGE_FLOATS_PER_WARP * 4;
     static size_t smem_bytes(int B) {
         return KV_BYTES + IDX_BYTES + MERGE_BYTES + static_cast<size_t>(3 * B + 1) * 4;
     }
     static_assert(RG >= 1 && RG * HKV * KG == WARPS, "warp split");
-    static_assert(NT * RG == LT && MT * KG == TILE / 16, "tile split");
+    static_assert(NT * RG == LT && MT * KG == TK / 16, "tile split");
+    static_assert(TK % 64 == 0 && TK <= DEC_THREADS, "tile size");
 };
 
 // Row (within a 16-key group) holding the MMA's logical key l.
@@ -238,9 +242,9 @@ __device__ __forceinline__ int kappa(int l) {
     return (l & 8) | s;
 }
 
-template <int LT, int PS, int KG, int NS, int MINB>
+template <int LT, int PS, int KG, int NS, int MINB, int TK, bool MERGE>
 __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepParams p) {
-    using C = DecodeCfg<LT, KG, NS>;
+    using C = DecodeCfg<LT, KG, NS, TK, MERGE>;
     constexpr int NT = C::NT, MT = C::MT, RG = C::RG;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* kv_smem = smem;
@@ -259,7 +263,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
 
     // ---- request key ranges and the tile list (reads inputs only) ----
     int total, per, t0, t1;
-    build_tile_list(p, tpre, rlo, rhi, DEC_THREADS, total, per, t0, t1);
+    build_tile_list<TK>(p, tpre, rlo, rhi, DEC_THREADS, total, per, t0, t1);
     // q and this step's cache rows come from the prep kernel
     pdl_wait_primary();
     if (t0 >= t1) return;
@@ -280,47 +284,51 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
         ++tau;
         while (b < B - 1 && tau >= tpre[b + 1]) ++b;
     };
-    auto tile_k0 = [&](int tau, int b) { return (rlo[b] / TILE + (tau - tpre[b])) * TILE; };
+    auto tile_k0 = [&](int tau, int b) { return (rlo[b] / TK + (tau - tpre[b])) * TK; };
 
     // ---- async loads ----
     auto issue_idx = [&](int tau, int b) {
         if (tau >= t1) return;
         const int k0 = tile_k0(tau, b);
-        int* dst = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TILE;
+        int* dst = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
         const int32_t* pt = p.page_table + static_cast<size_t>(b) * p.max_pages;
         if (PS == 1) {
-            if (tid < TILE) {
+            if (tid < TK) {
                 const int k = k0 + tid;
                 if (k >= rlo[b] && k <= rhi[b] && k < p.max_pages) cp_async4(smem_addr(dst + tid), pt + k);
                 else dst[tid] = -1;
             }
         } else {
-            if (tid == 0) {
-                const int pg = k0 / PS;
-                if (pg < p.max_pages) cp_async4(smem_addr(dst), pt + pg);
-                else dst[0] = -1;
+            if (tid < TK / PS) {  // the tile's pages
+                const int pg = k0 / PS + tid;
+                if (pg < p.max_pages) cp_async4(smem_addr(dst + tid), pt + pg);
+                else dst[tid] = -1;
             }
         }
     };
     auto issue_kv = [&](int tau, int b) {
         if (tau >= t1) return;
         const int k0 = tile_k0(tau, b);
-        const int* ix = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TILE;
-        const uint32_t base = smem_addr(kv_smem + ((tau - t0) % NS) * STAGE_BYTES);
+        const int* ix = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
+        const uint32_t base = smem_addr(kv_smem + ((tau - t0) % NS) * C::STAGE);
         const int lo = rlo[b], hi = rhi[b];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < TK / 32; ++i) {
             const int r = (tid >> 3) + 32 * i;  // tile row
             const int j = tid & 7;              // 16-byte chunk
             const int k = k0 + r;
             int64_t crow;
-            if (PS == 1) crow = ix[r];
-            else crow = ix[0] >= 0 ? static_cast<int64_t>(ix[0]) * PS + r : -1;
+            if (PS == 1) {
+                crow = ix[r];
+            } else {
+                const int pg = ix[r / PS];
+                crow = pg >= 0 ? static_cast<int64_t>(pg) * PS + r % PS : -1;
+            }
             const bool ok = k >= lo && k <= hi && crow >= 0 && crow < p.num_rows;
             const size_t off = ok ? static_cast<size_t>(crow) * ROWB + j * 16 : 0;
             const uint32_t d = base + r * ROWB + ((j ^ (r & 7)) << 4);
             cp_async16(d, p.k_cache + off, ok ? 16 : 0);
-            cp_async16(d + TILE * ROWB, p.v_cache + off, ok ? 16 : 0);
+            cp_async16(d + TK * ROWB, p.v_cache + off, ok ? 16 : 0);
         }
     };
 
@@ -375,9 +383,9 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
     };
 
     auto compute_tile = [&](int slot, int k0) {
-        const uint32_t kbase = smem_addr(kv_smem + slot * STAGE_BYTES);
-        const uint32_t vbase = kbase + TILE * ROWB;
-        const bool need_mask = !(k0 >= req_lo_max && k0 + TILE - 1 <= req_hi_min);
+        const uint32_t kbase = smem_addr(kv_smem + slot * C::STAGE);
+        const uint32_t vbase = kbase + TK * ROWB;
+        const bool need_mask = !(k0 >= req_lo_max && k0 + TK - 1 <= req_hi_min);
         float s[MT][NT][4];
         // S^T = K . Q^T
 #pragma unroll
@@ -494,7 +502,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
                 l += __shfl_xor_sync(0xffffffffu, l, 16);
                 l_run[nt][e] = l;
             }
-        if (KG > 1) {
+        if (MERGE && KG > 1) {
             if (kg > 0) {
                 float* buf = merge_smem +
                              static_cast<size_t>(((kg - 1) * HKV * RG + g * RG + rg) * NT) * 640;
@@ -539,8 +547,8 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
             }
             __syncthreads();
         }
-        if (kg == 0) {
-            const size_t slot = (static_cast<size_t>(blockIdx.x) + b) * p.tl;
+        if (!MERGE || kg == 0) {
+            const size_t slot = (static_cast<size_t>(blockIdx.x) + b) * C::PARTS + (MERGE ? 0 : kg);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int j = rg * NT + nt;
@@ -606,13 +614,15 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
 // ---------------------------------------------------------------------------
 // Kernel 3: merge the partials of each (token, head) and apply the gated
 // output norm.  One block per (token, head).  A request covered by many CTAs
-// has many partial slots (a single 80K-key request spreads over ~300), so the
-// slots are read in parallel: thread (sl, dq) accumulates dims 4dq..4dq+3 over
-// slots sl, sl+16, ..., then the 16 slot lanes are summed in shared memory.
+// has many partials (a single 80K-key request spreads over ~1,200), so they
+// are read in parallel: thread (sl, dq) accumulates dims 4dq..4dq+3 over
+// partials sl, sl + lanes, ..., then the slot lanes are summed in shared memory.
 // ---------------------------------------------------------------------------
-constexpr int COMB_SLOT_LANES = 16;
-
+// Block width: 1024 threads (64 slot lanes) for steps with few tokens, whose
+// requests are spread over many CTAs; 256 (16 slot lanes) otherwise.
+template <int COMB_THREADS>
 __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams p) {
+    constexpr int COMB_SLOT_LANES = COMB_THREADS / 16;
     pdl_wait_primary();
     __shared__ float red_o[COMB_SLOT_LANES][HD];
     __shared__ float red_l[COMB_SLOT_LANES];
@@ -632,24 +642,16 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams 
     const int c_lo = tp / per, c_hi = (tp + n - 1) / per;
     const int TL = p.tl;
     const int ns = (c_hi - c_lo + 1) * TL;
-    // Partial s = (CTA c_lo + s / TL, tile lane s % TL).  Tile lane tl of CTA c
-    // holds a partial for this request only if one of the request's tiles in
-    // CTA c's share has a local index congruent to tl modulo TL.
+    // Partial s = (CTA c_lo + s / TL, lane s % TL); every CTA that covered some
+    // of the request's tiles wrote all its lanes (a lane that saw no key of the
+    // request has max -inf and is skipped).
     auto slot_base = [&](int s) {
         const int c = c_lo + s / TL, tl = s % TL;
         return ((static_cast<size_t>(c + b) * TL + tl) * p.lt + j) * HQ + h;
     };
-    auto slot_used = [&](int s) {
-        const int c = c_lo + s / TL, tl = s % TL;
-        const int i0 = max(tp, c * per) - c * per;
-        const int i1 = min(tp + n, (c + 1) * per) - c * per;
-        const int cnt = i1 - i0;
-        return cnt >= TL || (((tl - i0) % TL + TL) % TL) < cnt;
-    };
     // 1. global max over the slots
     float mx = -INFINITY;
-    for (int s = tid; s < ns; s += COMB_THREADS)
-        if (slot_used(s)) mx = fmaxf(mx, p.part_ml[slot_base(s) * 2]);
+    for (int s = tid; s < ns; s += COMB_THREADS) mx = fmaxf(mx, p.part_ml[slot_base(s) * 2]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if (lane == 0) red_m[warp] = mx;
@@ -661,8 +663,8 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams 
     const int sl = tid / 16, dq = tid % 16;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.f;
+#pragma unroll 2
     for (int s = sl; s < ns; s += COMB_SLOT_LANES) {
-        if (!slot_used(s)) continue;
         const size_t base = slot_base(s);
         const float ms = p.part_ml[base * 2];
         if (ms == -INFINITY) continue;
@@ -680,7 +682,7 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams 
     // 3. threads 0..63: one output dim each
     if (tid < HD) {
         float o = 0.f, l = 0.f;
-#pragma unroll
+#pragma unroll 8
         for (int k = 0; k < COMB_SLOT_LANES; ++k) {
             o += red_o[k][tid];
             l += red_l[k];

@@ -93,73 +93,3 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 
 }  // namespace gad
 
-namespace gad {
-
-// ---- mbarrier (shared::cta) ----
-__device__ __forceinline__ void mbar_init(uint32_t addr, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(addr), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t addr) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(addr) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t addr, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(addr), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_timer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
-    return t;
-}
-// try_wait that lets the hardware suspend the thread (up to `hint_ns`) until
-// the phase completes, instead of spinning and taking issue slots.
-__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t addr, uint32_t parity,
-                                                      uint32_t hint_ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(addr), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
-}
-
-// Wait for the barrier phase with the given parity, for at most about
-// `limit_ns`.  Returns false on timeout (the caller records an error and stops).
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity, uint64_t limit_ns) {
-    if (mbar_try_wait(addr, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-#pragma unroll 1
-        for (int k = 0; k < 64; ++k)
-            if (mbar_try_wait_suspend(addr, parity, 100000u)) return true;
-        if (global_timer_ns() - t0 > limit_ns) return false;
-    }
-}
-
-// 2D TMA tile load global -> shared, completion counted on an mbarrier.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y,
-                                            uint32_t mbar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(mbar)
-        : "memory");
-}
-
-}  // namespace gad
-
