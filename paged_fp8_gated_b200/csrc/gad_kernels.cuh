@@ -160,25 +160,28 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) 
 // memory at the end of each segment.
 // ---------------------------------------------------------------------------
 // Per-request key ranges [lo_b, hi_b] (union over the request's tokens), the
+// first key this step writes (rnew_b), the
 // prefix of TK-key tile counts over requests (tiles aligned to multiples of TK), and this CTA's share of the tile
 // list [t0, t1).  Every thread of the block must call it.  CTA 0 also writes the
 // list to the workspace for the combine kernel.
 template <int TK>
 __device__ __forceinline__ void build_tile_list(const StepParams& p, int* tpre, int* rlo, int* rhi,
-                                                int nthreads, int& total, int& per, int& t0,
-                                                int& t1) {
+                                                int* rnew, int nthreads, int& total, int& per,
+                                                int& t0, int& t1) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int B = p.B, L = p.L;
     for (int b = tid; b < B; b += nthreads) {
-        int lo = INT_MAX, hi = -1;
+        int lo = INT_MAX, hi = -1, first = INT_MAX;
         for (int j = 0; j < L; ++j) {
             const int pos = static_cast<int>(p.positions[static_cast<size_t>(b) * L + j]);
             const int l = p.window > 0 ? max(0, pos - p.window + 1) : 0;
             lo = min(lo, l);
             hi = max(hi, pos);
+            first = min(first, pos);
         }
         rlo[b] = lo;
         rhi[b] = hi;
+        rnew[b] = first;  // keys at or above this one are written by this step
         tpre[b + 1] = (hi >= lo && hi >= 0) ? (hi / TK - lo / TK + 1) : 0;
     }
     if (tid == 0) tpre[0] = 0;
@@ -228,7 +231,7 @@ struct DecodeCfg {
     static constexpr size_t MERGE_BYTES =
         static_cast<size_t>(MERGE_WARPS) * MERGE_FLOATS_PER_WARP * 4;
     static size_t smem_bytes(int B) {
-        return KV_BYTES + IDX_BYTES + MERGE_BYTES + static_cast<size_t>(3 * B + 1) * 4;
+        return KV_BYTES + IDX_BYTES + MERGE_BYTES + static_cast<size_t>(4 * B + 1) * 4;
     }
     static_assert(RG >= 1 && RG * HKV * KG == WARPS, "warp split");
     static_assert(NT * RG == LT && MT * KG == TK / 16, "tile split");
@@ -253,6 +256,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
     int* tpre = reinterpret_cast<int*>(smem + C::KV_BYTES + C::IDX_BYTES + C::MERGE_BYTES);
     int* rlo = tpre + p.B + 1;
     int* rhi = rlo + p.B;
+    int* rnew = rhi + p.B;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gid = lane >> 2, tig = lane & 3;
@@ -263,10 +267,20 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
 
     // ---- request key ranges and the tile list (reads inputs only) ----
     int total, per, t0, t1;
-    build_tile_list<TK>(p, tpre, rlo, rhi, DEC_THREADS, total, per, t0, t1);
-    // q and this step's cache rows come from the prep kernel
-    pdl_wait_primary();
+    build_tile_list<TK>(p, tpre, rlo, rhi, rnew, DEC_THREADS, total, per, t0, t1);
     if (t0 >= t1) return;
+    // The normalised q and this step's new cache rows come from the prep kernel,
+    // which may still be running (programmatic dependent launch): wait for it
+    // only before the first q load or the first gather of a tile holding new
+    // keys, so the tile list and the first gathers overlap it.  The condition is
+    // the same for every thread of the CTA.
+    bool prep_done = false;
+    auto ensure_prep = [&]() {
+        if (!prep_done) {
+            pdl_wait_primary();
+            prep_done = true;
+        }
+    };
 
     const float C2 = __ldg(p.k_scale) * 0.125f * 1.4426950408889634f;  // raw score -> log2 units
 
@@ -309,6 +323,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
     auto issue_kv = [&](int tau, int b) {
         if (tau >= t1) return;
         const int k0 = tile_k0(tau, b);
+        if (k0 + TK - 1 >= rnew[b]) ensure_prep();
         const int* ix = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
         const uint32_t base = smem_addr(kv_smem + ((tau - t0) % NS) * C::STAGE);
         const int lo = rlo[b], hi = rhi[b];
@@ -343,6 +358,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
     const int vrow0 = kappa(2 * tig), vrow1 = kappa(2 * tig + 1);  // PV: + 0 and + 8
 
     auto begin_request = [&](int b) {
+        ensure_prep();
         req_lo_max = 0;
         req_hi_min = INT_MAX;
         for (int j = 0; j < L; ++j) {
