@@ -197,9 +197,8 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from paged_fp8_gated_b200 import replicas
+    rank, world, local_rank = replicas.rank_info()
 
     if args.impl == "reference":
         run_reference(args, rank, world)
@@ -217,7 +216,7 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
-    spec = W.named(args.workload, seed=1000 * rank)
+    spec = W.named(args.workload, seed=replicas.replica_seed(0, rank))
     inp = W.make_inputs(spec)
     B, L, ps = inp["B"], inp["L"], inp["page_size"]
     T = B * L
@@ -256,15 +255,10 @@ def main():
     torch.cuda.synchronize(dev)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        replicas.barrier(world)
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(x, world, dev)
 
     # ---- device-timed steps: graph replay, cold L2 before each ----
     for _ in range(args.warmup):
@@ -349,7 +343,7 @@ def main():
     traffic = TRAFFIC.get((args.workload, kernel_source_hash()))
     line = {
         "metric": METRIC,
-        "value": round(world * kv_bytes / (mean_ms * 1e-3) / 1e9, 2),
+        "value": round(replicas.job_rate(kv_bytes, world, mean_ms * 1e-3) / 1e9, 2),
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,

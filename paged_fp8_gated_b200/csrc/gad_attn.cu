@@ -44,9 +44,10 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 //   single-token steps: 128-key stages, 3 of them, two CTAs per SM (so 128 KB of
 //   loads in flight per SM); each key group writes its own partial (no merge
 //   buffer, so the stages fit)
-//   verify blocks:      64-key stages, 4 of them, one CTA per SM, merged
+//   verify blocks:      64-key stages, 4 of them, two CTAs per SM; each warp
+//   covers all keys of a tile for two tokens of one KV head (one key group)
 constexpr int kV1SingleKG = 4, kV1SingleNS = 3, kV1SingleTK = 128;
-constexpr int kV1VerifyKG = 2, kV1VerifyNS = 4, kV1VerifyTK = 64;
+constexpr int kV1VerifyKG = 1, kV1VerifyNS = 4, kV1VerifyTK = 64;
 
 struct WsLayout {
     size_t q_off, po_off, pml_off, meta_off, total;
@@ -256,8 +257,8 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
                  : launch_decode<1, 64, kV1SingleKG, kV1SingleNS, 2, kV1SingleTK, false>(prm, sms, tiles_upper, s, !timed);
     } else {
         st = page_size == 1
-                 ? launch_decode<8, 1, kV1VerifyKG, kV1VerifyNS, 1, kV1VerifyTK, true>(prm, sms, tiles_upper, s, !timed)
-                 : launch_decode<8, 64, kV1VerifyKG, kV1VerifyNS, 1, kV1VerifyTK, true>(prm, sms, tiles_upper, s, !timed);
+                 ? launch_decode<8, 1, kV1VerifyKG, kV1VerifyNS, 2, kV1VerifyTK, true>(prm, sms, tiles_upper, s, !timed)
+                 : launch_decode<8, 64, kV1VerifyKG, kV1VerifyNS, 2, kV1VerifyTK, true>(prm, sms, tiles_upper, s, !timed);
     }
     if (st != GAD_OK) return st;
     if (timed) cudaEventRecord(static_cast<cudaEvent_t>(events[2]), s);

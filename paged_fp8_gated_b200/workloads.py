@@ -48,6 +48,7 @@ class Spec:
     gate_std: float = 1.0
     seed: int = 0
     spare_pages: int = 0       # unused pages in the pool
+    dist: str = "normal"       # "normal", "coherent" or "edges" (see make_inputs)
     extra: dict = field(default_factory=dict)
 
 
@@ -116,6 +117,35 @@ def make_inputs(spec: Spec) -> dict:
         vx = torch.randn(r1 - r0, HKV, D, generator=gen)
         k_cache[r0:r1] = _to_e4m3_codes(kx * inv)
         v_cache[r0:r1] = _to_e4m3_codes(vx * inv)
+
+    if spec.dist == "coherent":
+        # Keys of each KV head share a direction (so attention spreads over many
+        # keys) and values share one too: the page's "dist coherent" loads.
+        u = _unit_rms(torch.randn(1, HKV, D, generator=gen))
+        vdir = torch.randn(1, HKV, D, generator=gen)
+        for r0 in range(0, rows, chunk):
+            r1 = min(rows, r0 + chunk)
+            kx = _unit_rms(u + 0.35 * torch.randn(r1 - r0, HKV, D, generator=gen))
+            vx = vdir + 0.5 * torch.randn(r1 - r0, HKV, D, generator=gen)
+            k_cache[r0:r1] = _to_e4m3_codes(kx * inv)
+            v_cache[r0:r1] = _to_e4m3_codes(vx * inv)
+    elif spec.dist == "edges":
+        # Large-logit keys at the window's edges: for every token, the oldest key
+        # inside its window and the newest key just outside it copy the token's
+        # raw query direction (mean over the KV head's 8 query heads), scaled up.
+        # Meant for layers without RoPE, where that raw direction is the one the
+        # scores see; a window off by one key changes the output completely.
+        assert spec.window > 0, "edges needs a sliding window"
+        qraw = qkv.float()[:, :HQ * D].view(T, HKV, HQ // HKV, D).mean(2)  # [T, 2, 64]
+        for t in range(T):
+            b = t // L
+            for key in (int(positions[t]) - spec.window + 1, int(positions[t]) - spec.window):
+                if 0 <= key < int(seq[b]):   # cached keys only
+                    row = int(page_table[b, key // ps]) * ps + key % ps
+                    kdir = _unit_rms(qraw[t])
+                    k_cache[row] = _to_e4m3_codes(kdir * (3.0 * inv))
+    elif spec.dist != "normal":
+        raise ValueError(f"unknown dist {spec.dist!r}")
 
     return dict(
         name=spec.name,

@@ -41,10 +41,19 @@ SMALL = [
       seed=118),
     S("gate_std2_s64", B=2, L=8, ctx=1500, page_size=64, kv_scale=1 / 64, gate_std=2.0, seed=119),
     S("spare_pages", B=2, seq_lens=[333, 777], page_size=64, spare_pages=5, seed=120),
-    # more requests than the single-token kernel keeps tables for (other kernel)
+    # many requests
     S("b1100_decode_p1", B=1100, ctx_range=(0, 300), seed=123),
     S("b1100_decode_p64_sliding", B=1100, ctx_range=(0, 400), window=100, use_rope=True,
       page_size=64, seed=124),
+    # the page's stress distributions (section "Correctness")
+    S("coherent_full", B=4, ctx=6000, dist="coherent", seed=125),
+    S("coherent_full_v8_p64", B=2, L=8, ctx=20000, page_size=64, dist="coherent", seed=126),
+    S("coherent_sliding_rope", B=3, L=8, ctx=5000, window=2048, use_rope=True, dist="coherent",
+      seed=127),
+    S("edges_sliding", B=4, ctx=6000, window=2048, dist="edges", seed=128),
+    S("edges_sliding_v8", B=4, L=8, ctx=6000, window=2048, dist="edges", seed=129),
+    S("edges_sliding_v8_p64_s64", B=3, L=8, ctx=4000, window=2048, page_size=64,
+      kv_scale=1 / 64, dist="edges", seed=130),
 ]
 
 
