@@ -24,7 +24,6 @@ rank's time.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import os
@@ -42,16 +41,29 @@ BYTES_PER_KEY = 256          # K and V rows: 2 KV heads x 64 E4M3 codes each
 PT_BYTES_PER_KEY = {1: 4, 64: 4 / 64}   # page-table bytes read per key
 FALLBACK_HBM_GBS = 6650.0
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one decode-kernel launch on the
-# default workload, from the ncu capture summarised in profiles/, keyed by the
-# hash of the kernel sources it was taken on (null once the sources change).
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of the step's main
+# kernel on a workload, from the ncu captures summarised in profiles/, keyed by
+# the hash of that kernel's sources when the counters were taken (null once the
+# sources change).
 TRAFFIC = {("decode32_full", "2fdd59b5ca40957d"): 474552832}
 
+# Sources of the step's main kernel: decode_kernel for single-token steps,
+# verify_tc_kernel for verify blocks (the launch code is in gad_attn.cu).
+_CSRC = os.path.join(ROOT, "paged_fp8_gated_b200", "csrc")
+KERNEL_SOURCES = {
+    "decode_kernel": ["gad_kernels.cuh", "gad_ptx.cuh"],
+    "verify_tc_kernel": ["gad_kernels.cuh", "gad_ptx.cuh", "gad_tc.cuh", "gad_verify_tc.cuh"],
+}
 
-def kernel_source_hash() -> str:
+
+def main_kernel(L: int) -> str:
+    return "decode_kernel" if L == 1 else "verify_tc_kernel"
+
+
+def kernel_source_hash(kernel: str = "decode_kernel") -> str:
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "paged_fp8_gated_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(_CSRC, name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
@@ -340,7 +352,9 @@ def main():
 
     peaks = measured_peaks()
     achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
-    traffic = TRAFFIC.get((args.workload, kernel_source_hash()))
+    kname = main_kernel(L)
+    ksrc = kernel_source_hash(kname)
+    traffic = TRAFFIC.get((args.workload, ksrc))
     line = {
         "metric": METRIC,
         "value": round(replicas.job_rate(kv_bytes, world, mean_ms * 1e-3) / 1e9, 2),
@@ -368,7 +382,7 @@ def main():
                           "page table device-resident",
         },
         "roofline": {
-            "kernel": "decode_kernel", "bound": "hbm", "achieved": round(achieved, 1),
+            "kernel": kname, "bound": "hbm", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4),
             "traffic": traffic,
@@ -383,7 +397,7 @@ def main():
         "clocks": clocks,
         "wall_s_timed_region": round(wall, 4),
         "cpu_baseline": cpu,
-        "kernel_sources": kernel_source_hash(),
+        "kernel_sources": ksrc,
     }
     print(json.dumps(line), flush=True)
 

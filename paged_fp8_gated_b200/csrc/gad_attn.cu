@@ -18,6 +18,7 @@
 
 #include "gad_attn.h"
 #include "gad_kernels.cuh"
+#include "gad_verify_tc.cuh"
 
 namespace {
 
@@ -39,15 +40,11 @@ constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// decode_kernel configurations: (tokens, key groups, stages, CTAs per SM, keys
-// per stage, merge key groups in the CTA)
-//   single-token steps: 128-key stages, 3 of them, two CTAs per SM (so 128 KB of
-//   loads in flight per SM); each key group writes its own partial (no merge
-//   buffer, so the stages fit)
-//   verify blocks:      64-key stages, 4 of them, two CTAs per SM; each warp
-//   covers all keys of a tile for two tokens of one KV head (one key group)
+// decode_kernel configuration for single-token steps: 128-key stages, 3 of
+// them, two CTAs per SM (so 128 KB of loads in flight per SM); each of the 4
+// key groups writes its own partial (no merge buffer, so the stages fit).
+// Verify blocks (L > 1) run verify_tc_kernel (tcgen05), one CTA per SM.
 constexpr int kV1SingleKG = 4, kV1SingleNS = 3, kV1SingleTK = 128;
-constexpr int kV1VerifyKG = 1, kV1VerifyNS = 4, kV1VerifyTK = 64;
 
 struct WsLayout {
     size_t q_off, po_off, pml_off, meta_off, total;
@@ -138,6 +135,52 @@ int launch_decode(const gad::StepParams& prm, int sms, int tiles_upper, cudaStre
     e = cudaLaunchKernelEx(&cfg, kern, prm);
     if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     return GAD_OK;
+}
+
+// Verify blocks (L > 1) on the tcgen05 kernel: one CTA per SM; as many raw
+// stages as the shared memory leaves room for next to the per-request tables.
+template <int PS, int NS>
+int launch_verify_tc(const gad::StepParams& prm, int sms, int tiles_upper, cudaStream_t stream,
+                     bool pdl) {
+    using C = gad::vtc::Cfg<NS>;
+    auto kern = gad::verify_tc_kernel<PS, NS>;
+    const size_t smem = C::smem_bytes(prm.B);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", dev);
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        int optin = 0;
+        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess)
+            return fail(GAD_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+        if (e != cudaSuccess)
+            return fail(GAD_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    long long grid = sms;
+    if (grid > tiles_upper) grid = tiles_upper;
+    if (grid < 1) grid = 1;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(gad::vtc::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr = pdl_attr();
+    cfg.attrs = &attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, prm);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "verify launch: %s", cudaGetErrorString(e));
+    return GAD_OK;
+}
+
+// Largest B for which the 8-stage verify kernel fits in `optin` bytes of shared memory.
+constexpr int kVtcDeepStages = 8, kVtcShallowStages = 4;
+bool verify_deep_fits(int B, int optin) {
+    return gad::vtc::Cfg<kVtcDeepStages>::smem_bytes(B) <= static_cast<size_t>(optin);
 }
 
 }  // namespace
@@ -256,9 +299,17 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
                  ? launch_decode<1, 1, kV1SingleKG, kV1SingleNS, 2, kV1SingleTK, false>(prm, sms, tiles_upper, s, !timed)
                  : launch_decode<1, 64, kV1SingleKG, kV1SingleNS, 2, kV1SingleTK, false>(prm, sms, tiles_upper, s, !timed);
     } else {
-        st = page_size == 1
-                 ? launch_decode<8, 1, kV1VerifyKG, kV1VerifyNS, 2, kV1VerifyTK, true>(prm, sms, tiles_upper, s, !timed)
-                 : launch_decode<8, 64, kV1VerifyKG, kV1VerifyNS, 2, kV1VerifyTK, true>(prm, sms, tiles_upper, s, !timed);
+        int optin = 0, dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return fail(GAD_ERR_CUDA, "shared-memory opt-in query failed");
+        const bool deep = verify_deep_fits(B, optin);
+        if (page_size == 1)
+            st = deep ? launch_verify_tc<1, kVtcDeepStages>(prm, sms, tiles_upper, s, !timed)
+                      : launch_verify_tc<1, kVtcShallowStages>(prm, sms, tiles_upper, s, !timed);
+        else
+            st = deep ? launch_verify_tc<64, kVtcDeepStages>(prm, sms, tiles_upper, s, !timed)
+                      : launch_verify_tc<64, kVtcShallowStages>(prm, sms, tiles_upper, s, !timed);
     }
     if (st != GAD_OK) return st;
     if (timed) cudaEventRecord(static_cast<cudaEvent_t>(events[2]), s);
