@@ -18,24 +18,19 @@
 // output is 128 rows x (64 dims of head 0 | 64 dims of head 1); row r keeps
 // the half of its own KV head.
 //
-// Warp roles (one CTA per SM, 17 warps):
-//   loader warps 8-15   cp.async gathers of raw E4M3 rows into an NS-stage ring
-//                       (as decode_kernel), then E4M3 -> fp16 into a 128-byte-
-//                       swizzled tile (K and V, double-buffered); at a request's
-//                       first tile they also write its A operand into tensor
-//                       memory.
-//   MMA warp 16         S(i) = A . K(i)^T into tensor memory (double-buffered),
-//                       then O += P(i-1) . V(i-1) with P read from tensor memory,
-//                       and the row sums l += P(i-1) . 1 (an N = 16 MMA against
-//                       an all-ones tile), so l sums exactly the fp16 P that O
-//                       sums.
-//   softmax warps 0-7   warp w serves rows 32 (w % 4) .. +31 and keys
-//                       32 (w / 4) .. +31 of each tile; the two warps of a row
-//                       exchange their partial maxima through shared memory.
-//                       Online softmax with lazy rescaling (O is rescaled in
-//                       tensor memory only when the running max grows by more
-//                       than 2^8); P as fp16 back into the S columns; at a
-//                       request's last tile, O's row half -> partial.
+// Data flow per tile (all in one CTA per SM):
+//   loader warps 4-7  cp.async gathers of raw E4M3 rows into an NS-stage ring
+//                     (as decode_kernel), then E4M3 -> fp16 into a 128-byte-
+//                     swizzled tile (K and V, double-buffered); at a request's
+//                     first tile they also write its A operand into tensor
+//                     memory.
+//   MMA warp 8        S(i) = A . K(i)^T into tensor memory (double-buffered),
+//                     then O += P(i-1) . V(i-1) with P read from tensor memory.
+//   softmax warps 0-3 one thread per row: S from tensor memory, mask, online
+//                     softmax with lazy rescaling (O is rescaled in tensor
+//                     memory only when the running max grows by more than
+//                     2^8), P as fp16 back into the S columns; at a request's
+//                     last tile, O's row half -> partial.
 // Synchronisation by mbarriers; every wait is bounded (an expired wait sets
 // the step's error word and the CTA winds down, waits for its MMAs and frees
 // its tensor memory).
@@ -48,12 +43,10 @@ namespace gad {
 namespace vtc {
 
 constexpr int TK = 64;                        // keys per tile
-constexpr int SOFT_WARPS = 8;
-constexpr int SOFT = SOFT_WARPS * 32;         // 256 softmax threads
-constexpr int LOAD_T0 = SOFT;                 // first loader thread (warp 8)
-constexpr int LOADERS = 256;
-constexpr int MMA_WARP = (SOFT + LOADERS) / 32;  // warp 16
-constexpr int THREADS = SOFT + LOADERS + 32;     // 544
+constexpr int THREADS = 288;                  // 9 warps
+constexpr int LOAD_T0 = 128;                  // first loader thread (warp 4)
+constexpr int LOADERS = 128;
+constexpr int MMA_WARP = 8;
 constexpr int RAW_STAGE = 2 * TK * ROWB;      // 16 KB: 64 K rows then 64 V rows (E4M3)
 constexpr int HALF_TILE = TK * 128;           // one head of a converted tile: 64 keys x 64 fp16
 constexpr int F16_TILE = 2 * HALF_TILE;       // both heads: 16 KB
@@ -62,65 +55,47 @@ constexpr uint32_t TM_COLS = 512;             // tensor-memory columns allocated
 constexpr uint32_t TM_Q = 0;                  // A operand (fp16 pairs): 64 columns
 constexpr uint32_t TM_S = 64;                 // S buffer b at TM_S + 64 b (P aliases its first 32)
 constexpr uint32_t TM_O = 256;                // O: 128 columns (head 0 dims | head 1 dims)
-constexpr uint32_t TM_L = 384;                // row sums of P: 16 equal columns
-constexpr int ONES_BYTES = 16 * 128;          // B operand of the row-sum MMA: 16 x 64 fp16 ones
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr float RESCALE_LOG2 = 8.f;           // lazy rescale threshold (P stays <= 2^8)
 
-// named barriers (0 is __syncthreads)
-constexpr int NB_LOADERS = 1;
-constexpr int NB_PAIR0 = 2;                   // + w % 4: the two softmax warps of a row block
-
-// mbarrier indices ([2]: by tile parity)
-constexpr int BAR_K_READY = 0;    // [2] converted K tile (and A operand) ready  (loader arrivals)
-constexpr int BAR_V_READY = 2;    // [2] converted V tile ready                  (loader arrivals)
-constexpr int BAR_PV_DONE = 4;    // [2] PV of the tile done: V buffer free      (MMA commit)
-constexpr int BAR_S_FULL = 6;     // [2] S of the tile done: K buffer free       (MMA commit)
-constexpr int BAR_P_FULL = 8;     // [2] P of the tile in tensor memory          (softmax arrivals)
-constexpr int BAR_O_FREE = 10;    // O read out at a request's last tile         (softmax arrivals)
-constexpr int BAR_MMA_DONE = 11;  // teardown: all MMAs done                     (MMA commit)
-constexpr int NBARS = 12;
-
-// control block: barriers, tensor-memory base, abort flag, then the softmax
-// exchange array (per-half row maxima by tile parity)
-constexpr int CTRL_XMAX = 128;                          // float [2][2][128]
-constexpr int CTRL_BYTES = CTRL_XMAX + 2 * 2 * 128 * 4;
+// mbarrier indices
+constexpr int BAR_KV_READY = 0;   // [2] converted tile (and A operand) ready   (128 loader arrivals)
+constexpr int BAR_KV_FREE = 2;    // [2] PV of the tile done: buffers free       (MMA commit)
+constexpr int BAR_S_FULL = 4;     // [2] S of the tile in tensor memory          (MMA commit)
+constexpr int BAR_P_FULL = 6;     // [2] P of the tile in tensor memory          (128 softmax arrivals)
+constexpr int BAR_O_FREE = 8;     // O read out at a request's last tile         (128 softmax arrivals)
+constexpr int BAR_MMA_DONE = 9;   // teardown: all MMAs done                     (MMA commit)
+constexpr int NBARS = 10;
 
 template <int NS>
 struct Cfg {
-    static constexpr size_t F16_BYTES = 2 * F16_BUF + ONES_BYTES;
+    static constexpr size_t F16_BYTES = 2 * F16_BUF;
     static constexpr size_t RAW_BYTES = static_cast<size_t>(NS) * RAW_STAGE;
     static constexpr int IDX_SLOTS = 2 * NS;
     static constexpr size_t IDX_BYTES = static_cast<size_t>(IDX_SLOTS) * TK * 4;
+    static constexpr size_t CTRL_BYTES = 128;  // barriers, tensor-memory base, abort flag
     // + 1024 so the swizzled tiles can start on a 1024-byte boundary
     static size_t smem_bytes(int B) {
         return 1024 + F16_BYTES + RAW_BYTES + IDX_BYTES + CTRL_BYTES +
                static_cast<size_t>(4 * B + 1) * 4;
     }
     static_assert(NS >= 3, "stages");
-    static_assert(NBARS * 8 + 8 <= CTRL_XMAX, "control block");
+    static_assert(NBARS * 8 + 8 <= static_cast<int>(CTRL_BYTES), "control block");
 };
 
 // Wait for phase `parity` of `bar`, giving up after WAIT_LIMIT_NS or as soon
 // as another thread has flagged an abort.  Returns false on giving up (and
 // raises the abort flag).
-// The flag and the clock are looked at every 32nd poll only, so a waiting warp
-// spends few issue slots.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                              bool stop_on_abort = true) {
     if (mbar_try_wait(bar, parity)) return true;
-    uint64_t t0 = 0;
-    for (uint32_t n = 1;; ++n) {
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((n & 31u) == 0) {
-            if (stop_on_abort && *abort_flag) return false;
-            const uint64_t t = global_timer_ns();
-            if (t0 == 0) {
-                t0 = t;
-            } else if (t - t0 > WAIT_LIMIT_NS) {
-                *abort_flag = 1;
-                return false;
-            }
+        if (stop_on_abort && *abort_flag) return false;
+        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+            *abort_flag = 1;
+            return false;
         }
     }
 }
@@ -141,19 +116,17 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
     const uint32_t raw_addr = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
     uint8_t* f16 = smem;                                     // [2][K,V][head][64 keys][128 B]
-    uint8_t* ones = smem + 2 * F16_BUF;                      // [16][128 B] fp16 1.0
     uint8_t* raw = smem + C::F16_BYTES;                      // [NS][K rows, V rows]
     int* idx_smem = reinterpret_cast<int*>(raw + C::RAW_BYTES);
     uint8_t* ctrl = reinterpret_cast<uint8_t*>(idx_smem) + C::IDX_BYTES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + NBARS * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + NBARS * 8 + 4);
-    float* xmax = reinterpret_cast<float*>(ctrl + CTRL_XMAX);   // [parity][half][row]
-    int* tpre = reinterpret_cast<int*>(ctrl + CTRL_BYTES);
+    int* tpre = reinterpret_cast<int*>(ctrl + C::CTRL_BYTES);
     int* rlo = tpre + p.B + 1;
     int* rhi = rlo + p.B;
     int* rnew = rhi + p.B;
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
     const int B = p.B, L = p.L;
 
     int total, per, t0, t1;
@@ -163,17 +136,15 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
     const uint32_t bar0 = smem_addr(ctrl);
     auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
     if (tid == 0) {
-        mbar_init(BAR(BAR_K_READY), LOADERS);
-        mbar_init(BAR(BAR_K_READY + 1), LOADERS);
-        mbar_init(BAR(BAR_V_READY), LOADERS);
-        mbar_init(BAR(BAR_V_READY + 1), LOADERS);
-        mbar_init(BAR(BAR_PV_DONE), 1);
-        mbar_init(BAR(BAR_PV_DONE + 1), 1);
+        mbar_init(BAR(BAR_KV_READY), LOADERS);
+        mbar_init(BAR(BAR_KV_READY + 1), LOADERS);
+        mbar_init(BAR(BAR_KV_FREE), 1);
+        mbar_init(BAR(BAR_KV_FREE + 1), 1);
         mbar_init(BAR(BAR_S_FULL), 1);
         mbar_init(BAR(BAR_S_FULL + 1), 1);
-        mbar_init(BAR(BAR_P_FULL), SOFT);
-        mbar_init(BAR(BAR_P_FULL + 1), SOFT);
-        mbar_init(BAR(BAR_O_FREE), SOFT);
+        mbar_init(BAR(BAR_P_FULL), 128);
+        mbar_init(BAR(BAR_P_FULL + 1), 128);
+        mbar_init(BAR(BAR_O_FREE), 128);
         mbar_init(BAR(BAR_MMA_DONE), 1);
         *abort_flag = 0;
         mbar_fence_init();
@@ -182,9 +153,6 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
         tc_alloc(smem_addr(tmem_slot), TM_COLS);
         tc_relinquish();
     }
-    for (int i = tid; i < ONES_BYTES / 16; i += THREADS)
-        reinterpret_cast<uint4*>(ones)[i] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -207,7 +175,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
     auto tile_k0 = [&](int tau, int b) { return (rlo[b] / TK + (tau - tpre[b])) * TK; };
     const float C2 = __ldg(p.k_scale) * 0.125f * 1.4426950408889634f;  // raw score -> log2 units
 
-    if (warp >= SOFT_WARPS && warp < MMA_WARP) {
+    if (warp >= 4 && warp < 8) {
         // =================== loaders: gather, convert, A operand ===================
         const int ltid = tid - LOAD_T0;
         bool prep_done = false;
@@ -274,11 +242,9 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 cp_async16(d + TK * ROWB, p.v_cache + off[i], nbytes[i]);
             }
         };
-        // A operand of request b's S MMA, written by the loaders of warps 8-11:
-        // row q = [q | 0] (KV head 0) or [0 | q] (KV head 1).
+        // A operand of request b's S MMA: row ltid = [q | 0] (KV head 0) or [0 | q].
         auto write_q = [&](int b) {
             ensure_prep();
-            if (ltid >= 128) return;
             const int g = ltid >> 6, j = (ltid >> 3) & 7, hh = ltid & 7;
             uint32_t q[32], z[32];
 #pragma unroll
@@ -298,110 +264,84 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
 #pragma unroll
                 for (int c = 0; c < 32; ++c) q[c] = 0u;
             }
-            const uint32_t ta = tmem + TM_Q + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+            const uint32_t ta = tmem + TM_Q + (static_cast<uint32_t>(32 * (warp - 4)) << 16);
             tc_st32(ta + (g == 0 ? 0u : 32u), q);
             tc_st32(ta + (g == 0 ? 32u : 0u), z);
-            tc_wait_st();
         };
-        // raw stage -> fp16 tile, K or V part (kv = 0 / 1).  Thread = (row r, KV head
-        // h, chunk pair cp): 2 chunks of 16 codes, each to two 16-byte fp16 chunks.
-        // The (h, cp) lanes of a row walk their chunks in different orders so no
-        // two lanes of an 8-lane phase meet in one bank group.
-        auto convert = [&](int stage, int buf, int kv) {
-            const int r = ltid >> 2, h = (ltid >> 1) & 1, cp = ltid & 1;
+        // raw stage -> fp16 tile: thread = (K or V, row r); 16 codes -> two 16-byte fp16 chunks.
+        auto convert = [&](int stage, int buf) {
+            const int kv = ltid >> 6, r = ltid & 63;
             const uint32_t src = smem_addr(raw + stage * RAW_STAGE) + kv * TK * ROWB + r * ROWB;
-            const uint32_t dst = smem_addr(f16 + buf * F16_BUF) + kv * F16_TILE + h * HALF_TILE + r * 128;
-            uint4 w[2];
+            const uint32_t dst = smem_addr(f16 + buf * F16_BUF) + kv * F16_TILE + r * 128;
+            uint4 w[8];
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int jx = 2 * cp + (jj ^ h);  // code chunk within the head: 0..3
-                w[jj] = lds128(src + (((4 * h + jx) ^ (r & 7)) << 4));
-            }
+            for (int j = 0; j < 8; ++j) w[j] = lds128(src + ((j ^ (r & 7)) << 4));
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int c0 = 2 * (2 * cp + (jj ^ h));
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t row = dst + (j >> 2) * HALF_TILE;
+                const int c0 = 2 * (j & 3);
                 uint4 a, b;
-                a.x = e4m3x2_to_f16x2(w[jj].x);
-                a.y = e4m3x2_to_f16x2(w[jj].x >> 16);
-                a.z = e4m3x2_to_f16x2(w[jj].y);
-                a.w = e4m3x2_to_f16x2(w[jj].y >> 16);
-                b.x = e4m3x2_to_f16x2(w[jj].z);
-                b.y = e4m3x2_to_f16x2(w[jj].z >> 16);
-                b.z = e4m3x2_to_f16x2(w[jj].w);
-                b.w = e4m3x2_to_f16x2(w[jj].w >> 16);
-                sts128(dst + ((c0 ^ (r & 7)) << 4), a);
-                sts128(dst + (((c0 + 1) ^ (r & 7)) << 4), b);
+                a.x = e4m3x2_to_f16x2(w[j].x);
+                a.y = e4m3x2_to_f16x2(w[j].x >> 16);
+                a.z = e4m3x2_to_f16x2(w[j].y);
+                a.w = e4m3x2_to_f16x2(w[j].y >> 16);
+                b.x = e4m3x2_to_f16x2(w[j].z);
+                b.y = e4m3x2_to_f16x2(w[j].z >> 16);
+                b.z = e4m3x2_to_f16x2(w[j].w);
+                b.w = e4m3x2_to_f16x2(w[j].w >> 16);
+                sts128(row + ((c0 ^ (r & 7)) << 4), a);
+                sts128(row + (((c0 + 1) ^ (r & 7)) << 4), b);
             }
         };
 
-        // Pipeline.  Iteration i converts K(i) and V(i - 1), then gathers tile
-        // i + NS - 2 into the stage of tile i - 2 (fully consumed by then); page-
-        // table entries are fetched 2 NS - 4 tiles ahead.  Tile i's copies are in
-        // commit group i + 1.
         int xt = t0, xb = find_req(t0);
         int kt = t0, kb = xb;
         int ct = t0, cb = xb;
-        for (int d = 0; d < 2 * NS - 4; ++d) {
+        for (int d = 0; d < NS - 1; ++d) {
             issue_idx(xt, xb);
             advance(xt, xb);
         }
         cp_async_commit();
         cp_async_wait<0>();
-        bar_red_or(NB_LOADERS, LOADERS, false);
-        for (int d = 0; d < NS - 2; ++d) {
+        bar_red_or(1, LOADERS, false);
+        for (int d = 0; d < NS - 1; ++d) {
             issue_kv(kt, kb);
             advance(kt, kb);
+            issue_idx(xt, xb);
+            advance(xt, xb);
             cp_async_commit();
         }
         int seg_b = -1;
-        int i = 0;
-        bool aborted = false;
-        for (; ct < t1; ++i) {
-            cp_async_wait<NS - 3>();
+        for (int i = 0; ct < t1; ++i) {
+            cp_async_wait<NS - 2>();
             const bool seg_start = cb != seg_b;
             bool bad = false;
-            // K buffer i & 1: free once S(i - 2) is done; the A operand may be
-            // replaced once S(i - 1) is done (every earlier S MMA is then done too)
-            if (seg_start && i >= 1) bad = !wait_bounded(BAR(BAR_S_FULL + ((i - 1) & 1)), ((i - 1) >> 1) & 1, abort_flag);
-            else if (i >= 2) bad = !wait_bounded(BAR(BAR_S_FULL + (i & 1)), ((i - 2) >> 1) & 1, abort_flag);
-            // V buffer (i - 1) & 1: free once PV(i - 3) is done
-            if (i >= 3 && !bad) bad = !wait_bounded(BAR(BAR_PV_DONE + ((i - 1) & 1)), ((i - 3) >> 1) & 1, abort_flag);
-            // past this barrier: tile i landed for every loader, and every loader is
-            // done with tile i - 2's stage
-            if (bar_red_or(NB_LOADERS, LOADERS, bad)) {
-                aborted = true;
-                break;
-            }
+            // buffers i & 1 are free once PV(i - 2) is done (which also means every
+            // S MMA up to tile i - 1 is done, so the A operand may be replaced)
+            if (i >= 2) bad = !wait_bounded(BAR(BAR_KV_FREE + (i & 1)), ((i - 2) >> 1) & 1, abort_flag);
+            if (i == 1 && seg_start && !bad) bad = !wait_bounded(BAR(BAR_S_FULL), 0, abort_flag);
+            // past this barrier: tile i landed for every loader, and every loader
+            // has converted tile i - 1, so its raw stage may be refilled
+            if (bar_red_or(1, LOADERS, bad)) break;
             if (seg_start) {
                 write_q(cb);
                 seg_b = cb;
             }
-            convert(i % NS, i & 1, 0);
+            convert(i % NS, i & 1);
             fence_proxy_async_smem();
-            if (seg_start) tc_fence_before();
-            mbar_arrive(BAR(BAR_K_READY + (i & 1)));
-            if (i >= 1) {
-                convert((i - 1) % NS, (i - 1) & 1, 1);
-                fence_proxy_async_smem();
-                mbar_arrive(BAR(BAR_V_READY + ((i - 1) & 1)));
+            if (seg_start) {
+                tc_wait_st();
+                tc_fence_before();
             }
+            mbar_arrive(BAR(BAR_KV_READY + (i & 1)));
+            // gathers for tile i + NS - 1 (into the stage of tile i - 1), off the
+            // path from "buffer free" to "tile ready"
             issue_kv(kt, kb);
             advance(kt, kb);
             issue_idx(xt, xb);
             advance(xt, xb);
             cp_async_commit();
             advance(ct, cb);
-        }
-        if (!aborted && i >= 1) {
-            // the last tile's V
-            const int k = i - 1;
-            bool bad = false;
-            if (k >= 2) bad = !wait_bounded(BAR(BAR_PV_DONE + (k & 1)), ((k - 2) >> 1) & 1, abort_flag);
-            if (!bar_red_or(NB_LOADERS, LOADERS, bad)) {
-                convert(k % NS, k & 1, 1);
-                fence_proxy_async_smem();
-                mbar_arrive(BAR(BAR_V_READY + (k & 1)));
-            }
         }
         cp_async_wait<0>();
     }
@@ -411,12 +351,10 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
         // MMA and commit instructions is warp-uniform.
         constexpr uint32_t ID_S = idesc_f16_f32(128, TK, 0);  // S: A . K^T, K-major B
         constexpr uint32_t ID_O = idesc_f16_f32(128, 64, 1);  // O: P . V, MN-major B
-        constexpr uint32_t ID_L = idesc_f16_f32(128, 16, 0);  // row sums: P . ones^T
         const uint32_t f16_base = smem_addr(f16);
         // O += P(k) . V(k), as two N = 64 MMAs (one per KV head's dims).
         auto issue_pv = [&](int k, bool first, int seg) {
             if (!wait_warp(BAR(BAR_P_FULL + (k & 1)), (k >> 1) & 1, abort_flag)) return false;
-            if (!wait_warp(BAR(BAR_V_READY + (k & 1)), (k >> 1) & 1, abort_flag)) return false;
             if (first && seg >= 1 && !wait_warp(BAR(BAR_O_FREE), (seg - 1) & 1, abort_flag)) return false;
             tc_fence_after();
             const uint32_t vbuf = f16_base + (k & 1) * F16_BUF + F16_TILE;
@@ -428,11 +366,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                     tc_mma_ts(tmem + TM_O + 64u * h, pa + 8u * ks,
                               smem_desc_sw128(vbuf + h * HALF_TILE + ks * 2048), ID_O,
                               (ks > 0 || !first) ? 1u : 0u);
-#pragma unroll
-            for (int ks = 0; ks < TK / 16; ++ks)
-                tc_mma_ts(tmem + TM_L, pa + 8u * ks, smem_desc_sw128(smem_addr(ones) + ks * 32), ID_L,
-                          (ks > 0 || !first) ? 1u : 0u);
-            tc_commit(BAR(BAR_PV_DONE + (k & 1)));
+            tc_commit(BAR(BAR_KV_FREE + (k & 1)));
             return true;
         };
         int ct = t0, cb = find_req(t0);
@@ -447,7 +381,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 seg_b = cb;
                 ++seg;
             }
-            if (!wait_warp(BAR(BAR_K_READY + (i & 1)), (i >> 1) & 1, abort_flag)) {
+            if (!wait_warp(BAR(BAR_KV_READY + (i & 1)), (i >> 1) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -471,18 +405,17 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
         if (ok && i > 0) issue_pv(i - 1, prev_first, prev_seg);
         // every MMA this warp issued is done before the tensor memory is freed
         tc_commit(BAR(BAR_MMA_DONE));
-        wait_bounded(BAR(BAR_MMA_DONE), 0, abort_flag, false);
+        const bool done = wait_bounded(BAR(BAR_MMA_DONE), 0, abort_flag, false);
         __syncwarp();
+        (void)done;
     } else {
-        // =================== softmax: a row per lane, half the keys per warp ===================
-        const int sp = warp & 3, hc = warp >> 2;   // sub-partition (row block), key half
-        const int r = 32 * sp + lane;
+        // =================== softmax: one thread per row ===================
+        const int r = tid;
         const int g = r >> 6, j = (r >> 3) & 7, qh = g * GRP + (r & 7);
-        const uint32_t lane_base = static_cast<uint32_t>(32 * sp) << 16;
-        const int pair_bar = NB_PAIR0 + sp;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
         int ct = t0, cb = find_req(t0);
         int seg_b = -1, seg_t1 = 0, k0 = 0;  // current request, end of its tiles here, tile key
-        float m_run = -INFINITY;
+        float m_run = -INFINITY, l_run = 0.f;
         int lo_j = INT_MAX, hi_j = -1;
         for (int i = 0; ct < t1; ++i) {
             const bool seg_start = cb != seg_b;
@@ -491,6 +424,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 seg_t1 = min(t1, tpre[cb + 1]);
                 k0 = tile_k0(ct, cb);
                 m_run = -INFINITY;
+                l_run = 0.f;
                 if (j < L) {
                     const int pos = static_cast<int>(p.positions[static_cast<size_t>(cb) * L + j]);
                     hi_j = pos;
@@ -503,116 +437,97 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 k0 += TK;
             }
             const bool seg_end = ct + 1 >= seg_t1;
+
+            if (!wait_warp(BAR(BAR_S_FULL + (i & 1)), (i >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
             const uint32_t sbuf = tmem + TM_S + 64u * (i & 1) + lane_base;
-
-            // S half-row, mask, partial max, exchange with the other half's warp
-            bool bad = !wait_warp(BAR(BAR_S_FULL + (i & 1)), (i >> 1) & 1, abort_flag);
-            float s[32];
-            float mh = -INFINITY;
-            if (!bad) {
-                tc_fence_after();
-                uint32_t sr[32];
-                tc_ld32(sbuf + 32u * hc, sr);
-                tc_wait_ld();
-                const int cmin = (lo_j == INT_MAX ? TK : lo_j - k0) - 32 * hc;
-                const int cmax = hi_j - k0 - 32 * hc;
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                if (cmin <= 0 && cmax >= 31) {
+            uint32_t sr[64];
+            tc_ld32(sbuf, sr);
+            tc_ld32(sbuf + 32u, sr + 32);
+            tc_wait_ld();
+            float s[64];
+            const int cmin = lo_j == INT_MAX ? TK : lo_j - k0;
+            const int cmax = hi_j - k0;
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (cmin <= 0 && cmax >= TK - 1) {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        s[c] = __uint_as_float(sr[c]);
-                        m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        s[c] = (c < cmin || c > cmax) ? -INFINITY : __uint_as_float(sr[c]);
-                        m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-                    }
+                for (int c = 0; c < 64; ++c) {
+                    s[c] = __uint_as_float(sr[c]);
+                    m4[c & 3] = fmaxf(m4[c & 3], s[c]);
                 }
-                mh = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-                xmax[((i & 1) * 2 + hc) * 128 + r] = mh;
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    s[c] = (c < cmin || c > cmax) ? -INFINITY : __uint_as_float(sr[c]);
+                    m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+                }
             }
-            if (bar_red_or(pair_bar, 64, bad)) break;
-            const float mx = fmaxf(mh, xmax[((i & 1) * 2 + (1 - hc)) * 128 + r]);
-
-            // lazy rescale: O (in tensor memory) is corrected only when the max grows a
-            // lot; both warps of a row take the same decision from the same numbers
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            // lazy rescale: O (in tensor memory) is corrected only when the max grows a lot
             const float m_new = fmaxf(m_run, mx);
             bool corr = false;
             if (m_new > m_run) {
-                if (m_run == -INFINITY || (m_new - m_run) * C2 <= RESCALE_LOG2) {
-                    if (m_run == -INFINITY) m_run = m_new;
+                if (m_run == -INFINITY || seg_start || (m_new - m_run) * C2 <= RESCALE_LOG2) {
+                    if (m_run == -INFINITY || seg_start) m_run = m_new;
                 } else {
                     corr = true;
                 }
             }
             if (__any_sync(0xffffffffu, corr)) {
                 // PV(i - 1) of this request must be done before O is touched
-                bad = !wait_warp(BAR(BAR_PV_DONE + ((i - 1) & 1)), ((i - 1) >> 1) & 1, abort_flag);
-                if (!bad) {
-                    tc_fence_after();
-                    const float alpha = corr ? fast_exp2((m_run - m_new) * C2) : 1.f;
-                    const uint32_t oa = tmem + TM_O + 64u * g + 32u * hc + lane_base;
-                    uint32_t o[32];
-                    tc_ld32(oa, o);
+                if (!wait_warp(BAR(BAR_KV_FREE + ((i - 1) & 1)), ((i - 1) >> 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                const float alpha = corr ? fast_exp2((m_run - m_new) * C2) : 1.f;
+                const uint32_t oa = tmem + TM_O + 64u * g + lane_base;
+                uint32_t o[32];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    tc_ld32(oa + 32u * half, o);
                     tc_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                    tc_st32(oa, o);
-                    if (hc == 0) {  // the row sum, once per row
-                        uint32_t lv;
-                        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n"
-                                     : "=r"(lv) : "r"(tmem + TM_L + lane_base));
-                        tc_wait_ld();
-                        lv = __float_as_uint(__uint_as_float(lv) * alpha);
-                        asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};\n"
-                                     :: "r"(tmem + TM_L + lane_base), "r"(lv) : "memory");
-                    }
-                    tc_wait_st();
-                    if (corr) m_run = m_new;
+                    tc_st32(oa + 32u * half, o);
                 }
-                if (bar_red_or(pair_bar, 64, bad)) break;
+                tc_wait_st();
+                if (corr) {
+                    l_run *= alpha;
+                    m_run = m_new;
+                }
             }
-
-            // P = 2^(s C2 - m C2) as fp16 into the first 32 columns of the S buffer
             const float mc = m_run == -INFINITY ? 0.f : m_run * C2;
-            uint32_t pk[16];
+            uint32_t pk[32];
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
+            for (int c = 0; c < 32; ++c) {
                 const float p0 = fast_exp2(fmaf(s[2 * c], C2, -mc));
                 const float p1 = fast_exp2(fmaf(s[2 * c + 1], C2, -mc));
+                l4[c & 3] += p0 + p1;
                 pk[c] = pack_f16x2(p0, p1);
             }
-            tc_st16(sbuf + 16u * hc, pk);
+            l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            tc_st32(sbuf, pk);
             tc_wait_st();
             tc_fence_before();
             mbar_arrive(BAR(BAR_P_FULL + (i & 1)));
 
             if (seg_end) {
-                // PV(i) done -> this request's O row (a quarter per warp) -> partial
-                bad = !wait_warp(BAR(BAR_PV_DONE + (i & 1)), (i >> 1) & 1, abort_flag);
-                if (bar_red_or(pair_bar, 64, bad)) break;
+                if (!wait_warp(BAR(BAR_KV_FREE + (i & 1)), (i >> 1) & 1, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t oa = tmem + TM_O + 64u * g + 32u * hc + lane_base;
-                uint32_t o[32], lv;
+                const uint32_t oa = tmem + TM_O + 64u * g + lane_base;
+                uint32_t o[64];
                 tc_ld32(oa, o);
-                asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n"
-                             : "=r"(lv) : "r"(tmem + TM_L + lane_base));
+                tc_ld32(oa + 32u, o + 32);
                 tc_wait_ld();
-                const float l_tot = __uint_as_float(lv);
                 if (j < L) {
                     const size_t slot = static_cast<size_t>(blockIdx.x) + cb;
                     const size_t base = (slot * p.lt + j) * HQ + qh;
-                    float4* dst = reinterpret_cast<float4*>(p.part_o + base * HD + 32 * hc);
+                    float4* dst = reinterpret_cast<float4*>(p.part_o + base * HD);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
+                    for (int q = 0; q < 16; ++q)
                         dst[q] = make_float4(__uint_as_float(o[4 * q]), __uint_as_float(o[4 * q + 1]),
                                              __uint_as_float(o[4 * q + 2]), __uint_as_float(o[4 * q + 3]));
-                    if (hc == 0) {
-                        p.part_ml[base * 2 + 0] = m_run * C2;
-                        p.part_ml[base * 2 + 1] = l_tot;
-                    }
+                    p.part_ml[base * 2 + 0] = m_run * C2;
+                    p.part_ml[base * 2 + 1] = l_run;
                 }
                 tc_fence_before();
                 mbar_arrive(BAR(BAR_O_FREE));
