@@ -45,7 +45,8 @@ FALLBACK_HBM_GBS = 6650.0
 # kernel on a workload, from the ncu captures summarised in profiles/, keyed by
 # the hash of that kernel's sources when the counters were taken (null once the
 # sources change).
-TRAFFIC = {("decode32_full", "2fdd59b5ca40957d"): 474552832}
+TRAFFIC = {("decode32_full", "64c5ab721f0a7f48"): 474521600,
+           ("verify16_full", "9c1a1c537fa1f9f0"): 337947136}
 
 # Sources of the step's main kernel: decode_kernel for single-token steps,
 # verify_tc_kernel for verify blocks (the launch code is in gad_attn.cu).
