@@ -20,6 +20,8 @@ is weak and the job value is the sum of the ranks' KV bytes over the slowest
 rank's time.
 
 --impl reference times the CPU oracle itself as the reference arm.
+--suite times the page's twelve scored loads (decode and verify at B = 1, 16,
+32, sliding and full) against the page's floor model instead.
 """
 from __future__ import annotations
 
@@ -198,6 +200,97 @@ def run_reference(args, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
+def token_keys(inp: dict) -> int:
+    """Sum over tokens of the keys each token attends (p - lo + 1)."""
+    pos = inp["positions"].numpy()
+    W_ = inp["window"]
+    lo = (pos - W_ + 1).clip(min=0) if W_ > 0 else 0 * pos
+    return int((pos - lo + 1).sum())
+
+
+def run_suite(args):
+    """The page's twelve scored loads (section "Shapes" of the task page): per
+    load the graph-replayed step time (cold L2 before each replay) against the
+    page's floor model, max(bytes / 4.8 TB/s, flops / 989 TFLOP/s), applied to
+    this step's own bytes and flops; the score is the geometric mean of
+    floor / time weighted 46 (sliding) and 16 (full) as on the page."""
+    import math
+    import torch
+    from paged_fp8_gated_b200 import binding
+    from paged_fp8_gated_b200 import workloads as W
+
+    dev = torch.device("cuda", 0)
+    peaks = measured_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sink = torch.empty((), dtype=torch.int64, device=dev)
+    rows, num, den = [], 0.0, 0.0
+    for load, layer, name in W.LOAD_SET:
+        inp = W.make_inputs(W.named(name))
+        B, L = inp["B"], inp["L"]
+        T = B * L
+        d = {k: inp[k].to(dev) for k in ("qkv", "positions", "seq_lens", "page_table", "cache_loc",
+                                           "k_cache", "v_cache")}
+        ks = torch.tensor([inp["k_scale"]], dtype=torch.float32, device=dev)
+        vs = torch.tensor([inp["v_scale"]], dtype=torch.float32, device=dev)
+        out = torch.empty(B, L, 1024, dtype=torch.bfloat16, device=dev)
+        ws = binding.alloc_workspace(B, L, dev)
+
+        def step():
+            binding.attn_decode(d["qkv"], d["positions"], d["seq_lens"], d["page_table"], d["cache_loc"],
+                                d["k_cache"], d["v_cache"], ks, vs, inp["page_size"], inp["window"],
+                                inp["use_rope"], L=L, out=out, workspace=ws)
+
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            step()
+        side.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            step()
+        torch.cuda.synchronize(dev)
+
+        def cold():
+            flush.fill_(1)
+            torch.sum(flush.view(torch.int64), dim=0, out=sink)
+
+        for _ in range(args.warmup):
+            cold()
+            graph.replay()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for a, b in evs:
+            cold()
+            a.record()
+            graph.replay()
+            b.record()
+        torch.cuda.synchronize(dev)
+        us = statistics.median(a.elapsed_time(b) * 1e3 for a, b in evs)
+        keys = W.keys_attended(inp)
+        kv = keys * BYTES_PER_KEY
+        moved = kv + T * (2304 + 1024) * 2 + T * BYTES_PER_KEY   # KV read, qkv in, out, new rows
+        flops = 4096 * token_keys(inp)
+        floor_us = max(moved / 4.8e12, flops / 989e12) * 1e6
+        frac = floor_us / us
+        w = W.LAYER_WEIGHT[layer]
+        num += w * math.log(frac)
+        den += w
+        rows.append({"load": load, "layer": layer, "workload": name, "B": B, "L": L, "keys": keys,
+                     "us_per_step": round(us, 2), "kv_gbs": round(kv / (us * 1e-6) / 1e9, 1),
+                     "hbm_frac": round(kv / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                     "floor_us_page_model": round(floor_us, 2), "floor_over_time": round(frac, 4),
+                     "weight": w})
+        del graph, d, out, ws
+        torch.cuda.empty_cache()
+    line = {"metric": "page load set: weighted geometric mean of floor/time (floor = page's model on "
+                      "this step's bytes and flops)",
+            "value": round(math.exp(num / den), 4), "unit": "ratio", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "data": "synthetic",
+            "timing": "CUDA-graph replay, 256 MiB write+read before every step, median of steps",
+            "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"], "loads": rows}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -206,9 +299,14 @@ def main():
     ap.add_argument("--workload", default="decode32_full")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--suite", action="store_true",
+                    help="time the page's twelve scored loads instead (one GPU, one JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.suite:
+        run_suite(args)
+        return
 
     from paged_fp8_gated_b200 import replicas
     rank, world, local_rank = replicas.rank_info()

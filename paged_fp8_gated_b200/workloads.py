@@ -195,6 +195,18 @@ def named(name: str, seed: int = 0) -> Spec:
                                   permute=False, seed=seed + 2),
         "decode32_full_p64": Spec("decode32_full_p64", B=32, L=1, ctx_range=(40000, 80000),
                                   page_size=64, seed=seed + 2),
+        # the page's load table (section "Shapes"): decode and verify at B = 1, 16,
+        # 32, sliding and full; requests of B > 1 loads draw contexts uniformly
+        # from [40000, 80000] like decode32_full
+        "decode16_full": Spec("decode16_full", B=16, L=1, ctx_range=(40000, 80000), seed=seed + 51),
+        "decode16_sliding": Spec("decode16_sliding", B=16, L=1, ctx_range=(40000, 80000),
+                                 window=2048, use_rope=True, seed=seed + 52),
+        "verify1_full": Spec("verify1_full", B=1, L=8, ctx=80000, seed=seed + 53),
+        "verify1_sliding": Spec("verify1_sliding", B=1, L=8, ctx=80000, window=2048,
+                                use_rope=True, seed=seed + 54),
+        "verify32_full": Spec("verify32_full", B=32, L=8, ctx_range=(40000, 80000), seed=seed + 55),
+        "verify32_sliding": Spec("verify32_sliding", B=32, L=8, ctx_range=(40000, 80000),
+                                 window=2048, use_rope=True, seed=seed + 56),
         # 16 requests, 8-token causal verify blocks at 80,000 cached keys
         "verify16_sliding": Spec("verify16_sliding", B=16, L=8, ctx=80000, window=2048,
                                  use_rope=True, seed=seed + 31),
@@ -210,3 +222,15 @@ def named(name: str, seed: int = 0) -> Spec:
 
 NAMED = ["pr1", "decode1_sliding", "decode1_full", "decode32_full", "decode32_sliding",
          "verify16_sliding", "verify16_full", "paged_full", "paged_sliding"]
+
+# The page's twelve scored loads (load, layer) -> workload, and the weight the
+# page gives each layer kind in its geometric-mean score.
+LOAD_SET = [
+    ("decode 1", "sliding", "decode1_sliding"), ("decode 1", "full", "decode1_full"),
+    ("decode 16", "sliding", "decode16_sliding"), ("decode 16", "full", "decode16_full"),
+    ("decode 32", "sliding", "decode32_sliding"), ("decode 32", "full", "decode32_full"),
+    ("verify 1", "sliding", "verify1_sliding"), ("verify 1", "full", "verify1_full"),
+    ("verify 16", "sliding", "verify16_sliding"), ("verify 16", "full", "verify16_full"),
+    ("verify 32", "sliding", "verify32_sliding"), ("verify 32", "full", "verify32_full"),
+]
+LAYER_WEIGHT = {"sliding": 46.0, "full": 16.0}

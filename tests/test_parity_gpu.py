@@ -84,8 +84,12 @@ def test_long_ctx_1m_sampled(cuda_dev):
 
 
 FULL = ["pr1", "decode1_sliding", "decode1_full", "decode32_full", "decode32_sliding",
-        "verify16_sliding", "verify16_full", "paged_full", "paged_sliding"]
-SAMPLED = {"decode32_full": 24, "verify16_full": 24, "paged_full": 32}
+        "verify16_sliding", "verify16_full", "paged_full", "paged_sliding",
+        # the rest of the page's twelve scored loads
+        "decode16_full", "decode16_sliding", "verify1_full", "verify1_sliding",
+        "verify32_full", "verify32_sliding"]
+SAMPLED = {"decode32_full": 24, "verify16_full": 24, "paged_full": 32, "decode16_full": 24,
+           "verify1_full": 24, "verify32_full": 24, "verify32_sliding": 48}
 
 
 @pytest.mark.slow
