@@ -27,8 +27,14 @@
  *   - rmsnorm: eps 1e-6, unit weights, over each 64-wide head.
  *   - rope: NeoX half-split pairs (i, i+32), angle p * 10000^(-2i/64).
  *   - window W: token at position p attends keys i with p-W < i <= p.
- *   - q head h reads KV head h / 8.
- *   - qkv columns: q[0,1024) | k[1024,1152) | v[1152,1280) | gate[1280,2304).
+ *   - q head h reads KV head h / (hq / hkv); with 16 and 2 heads, h / 8.
+ *   - qkv columns, for hq query and hkv KV heads of 64 dims:
+ *     q[0, 64hq) | k[64hq, 64(hq+hkv)) | v[.., 64(hq+2hkv)) | gate[.., 64(2hq+2hkv)),
+ *     i.e. q[0,1024) | k[1024,1152) | v[1152,1280) | gate[1280,2304) at 16 and 2.
+ *   - "heads tp8" is 16 query and 2 KV heads per GPU (the page's section
+ *     "Shapes"); "heads dp" gives each GPU all heads of the layer, 8 times
+ *     as many: 128 and 16.  The step itself is the same formula.
+ *   - a cache row holds the hkv heads' 64 codes each: 64 * hkv bytes.
  *   - cache scale: stored code = E4M3(x / scale), dequantised = code * scale.
  *   - fp8(): double -> float (round to nearest even), then float -> E4M3
  *     (round to nearest even, saturating to +-448, NaN kept).
@@ -44,15 +50,9 @@
 #include <stdlib.h>
 #include <string.h>
 
-#define GADO_HQ 16
-#define GADO_HKV 2
+#define GADO_HQ 16   /* query heads of the page's per-GPU shapes ("heads tp8") */
+#define GADO_HKV 2   /* key/value heads of those shapes */
 #define GADO_D 64
-#define GADO_QKV_COLS (GADO_HQ * GADO_D + 2 * GADO_HKV * GADO_D + GADO_HQ * GADO_D) /* 2304 */
-#define GADO_Q_OFF 0
-#define GADO_K_OFF (GADO_HQ * GADO_D)                    /* 1024 */
-#define GADO_V_OFF (GADO_K_OFF + GADO_HKV * GADO_D)      /* 1152 */
-#define GADO_G_OFF (GADO_V_OFF + GADO_HKV * GADO_D)      /* 1280 */
-#define GADO_ROW_BYTES (GADO_HKV * GADO_D)               /* 128 bytes per cache row */
 
 /* ------------------------------------------------------------------------- */
 /* Number formats                                                             */
@@ -177,9 +177,10 @@ typedef struct {
     const uint16_t* qkv;
     double k_scale, v_scale;
     int B, L, max_pages, page_size, window;
+    int hq, hkv;            /* query heads, key/value heads */
     int64_t num_rows;
     const uint8_t* want;
-    const double* qn;       /* [T, 16, 64] normalised (and rotated) queries */
+    const double* qn;       /* [T, hq, 64] normalised (and rotated) queries */
     /* outputs */
     uint16_t* out;
     double* out_exact;
@@ -203,7 +204,9 @@ static int gado_row(const gado_job* J, int b, int64_t i, int64_t* row) {
 /* softmax(q.K^T/8).V for one (token, query head), then the gated output norm. */
 static int gado_one_head(gado_job* J, int t, int h, double* logits, int64_t cap) {
     const int b = t / J->L;
-    const int g = h / (GADO_HQ / GADO_HKV);
+    const int hq = J->hq, hkv = J->hkv;
+    const int g = h / (hq / hkv);
+    const int64_t row_bytes = (int64_t)hkv * GADO_D;
     const int64_t p = J->positions[t];
     int64_t lo = 0;
     if (J->window > 0) {
@@ -212,7 +215,7 @@ static int gado_one_head(gado_job* J, int t, int h, double* logits, int64_t cap)
     }
     const int64_t n = p - lo + 1;
     if (n <= 0 || n > cap) return GADO_ERR_ARG;
-    const double* q = J->qn + ((int64_t)t * GADO_HQ + h) * GADO_D;
+    const double* q = J->qn + ((int64_t)t * hq + h) * GADO_D;
 
     /* logits s_i = q . K_i / 8, K_i dequantised from the cache */
     double smax = -INFINITY;
@@ -220,7 +223,7 @@ static int gado_one_head(gado_job* J, int t, int h, double* logits, int64_t cap)
         int64_t row;
         int st = gado_row(J, b, i, &row);
         if (st) return st;
-        const uint8_t* kr = J->k_cache + row * GADO_ROW_BYTES + g * GADO_D;
+        const uint8_t* kr = J->k_cache + row * row_bytes + g * GADO_D;
         double dot = 0.0;
         for (int d = 0; d < GADO_D; ++d) dot += q[d] * (gado_e4m3_decode(kr[d]) * J->k_scale);
         double s = dot / 8.0;
@@ -232,9 +235,9 @@ static int gado_one_head(gado_job* J, int t, int h, double* logits, int64_t cap)
     for (int d = 0; d < GADO_D; ++d) a[d] = 0.0;
     double den = 0.0;
     for (int64_t i = lo; i <= p; ++i) {
-        int64_t row;
-        gado_row(J, b, i, &row);
-        const uint8_t* vr = J->v_cache + row * GADO_ROW_BYTES + g * GADO_D;
+        int64_t row = 0;
+        gado_row(J, b, i, &row);  /* checked by the first pass over the keys */
+        const uint8_t* vr = J->v_cache + row * row_bytes + g * GADO_D;
         double w = exp(logits[i - lo] - smax);
         den += w;
         for (int d = 0; d < GADO_D; ++d) a[d] += w * (gado_e4m3_decode(vr[d]) * J->v_scale);
@@ -244,11 +247,13 @@ static int gado_one_head(gado_job* J, int t, int h, double* logits, int64_t cap)
     /* out = rmsnorm(a) * sigmoid(gate) */
     double an[GADO_D];
     gado_rmsnorm(a, an, GADO_D, 1e-6);
-    const uint16_t* row_qkv = J->qkv + (int64_t)t * GADO_QKV_COLS;
+    const int64_t qkv_cols = (int64_t)(2 * hq + 2 * hkv) * GADO_D;
+    const int64_t gate_off = (int64_t)(hq + 2 * hkv) * GADO_D;
+    const uint16_t* row_qkv = J->qkv + (int64_t)t * qkv_cols;
     for (int d = 0; d < GADO_D; ++d) {
-        double gate = gado_bf16_decode(row_qkv[GADO_G_OFF + h * GADO_D + d]);
+        double gate = gado_bf16_decode(row_qkv[gate_off + h * GADO_D + d]);
         double y = an[d] * gado_sigmoid(gate);
-        int64_t o = (int64_t)t * (GADO_HQ * GADO_D) + h * GADO_D + d;
+        int64_t o = (int64_t)t * ((int64_t)hq * GADO_D) + h * GADO_D + d;
         J->out[o] = gado_bf16_encode(y);
         if (J->out_exact) J->out_exact[o] = y;
         if (J->attn_out) J->attn_out[o] = a[d];
@@ -271,9 +276,9 @@ static void* gado_worker(void* arg) {
         J->status = GADO_ERR_NOMEM;
         return NULL;
     }
-    for (int w = J->tid; w < T * GADO_HQ; w += J->nthreads) {
+    for (int64_t w = J->tid; w < (int64_t)T * J->hq; w += J->nthreads) {
         if (J->want && !J->want[w]) continue;
-        int st = gado_one_head(J, w / GADO_HQ, w % GADO_HQ, logits, cap);
+        int st = gado_one_head(J, (int)(w / J->hq), (int)(w % J->hq), logits, cap);
         if (st) {
             J->status = st;
             break;
@@ -284,43 +289,49 @@ static void* gado_worker(void* arg) {
 }
 
 /*
- * The whole step on host memory.
- *   qkv        bf16 bits [T, 2304], T = B * L, token t = b * L + j
+ * The whole step on host memory, for hq query heads and hkv key/value heads
+ * of 64 dims (hq a positive multiple of hkv).
+ *   qkv        bf16 bits [T, 64 * (2 hq + 2 hkv)], T = B * L, token t = b * L + j
  *   positions  [T]   position p of each token (attends keys lo..p)
  *   page_table [B, max_pages]
  *   cache_loc  [T]   cache row receiving token t's k and v
- *   k_cache, v_cache [num_rows, 2, 64] E4M3 codes; rows cache_loc[] are written
+ *   k_cache, v_cache [num_rows, hkv, 64] E4M3 codes; rows cache_loc[] are written
  *   k_scale, v_scale  the cache scales (float, as the device holds them)
  *   window     > 0: sliding window size; <= 0: full attention
  *   use_rope   1: rotate q and k by their positions
- *   want       [T * 16] or NULL: compute only (t, h) with want[t*16+h] != 0
- *   out        bf16 bits [T, 1024]
- *   out_exact  [T, 1024] or NULL: the output before bf16 rounding
- *   attn_out   [T, 1024] or NULL: a = softmax(...) . V before the output norm
+ *   want       [T * hq] or NULL: compute only (t, h) with want[t*hq+h] != 0
+ *   out        bf16 bits [T, 64 * hq]
+ *   out_exact  [T, 64 * hq] or NULL: the output before bf16 rounding
+ *   attn_out   [T, 64 * hq] or NULL: a = softmax(...) . V before the output norm
  * Returns 0, or a negative GADO_ERR_* code.
  */
-int gado_attn_decode(const uint16_t* qkv, const int64_t* positions, const int32_t* page_table,
-                     const int64_t* cache_loc, uint8_t* k_cache, uint8_t* v_cache, float k_scale,
-                     float v_scale, int B, int L, int max_pages, int64_t num_rows, int page_size,
-                     int window, int use_rope, const uint8_t* want, uint16_t* out, double* out_exact,
-                     double* attn_out, int nthreads) {
+int gado_attn_decode_heads(const uint16_t* qkv, const int64_t* positions, const int32_t* page_table,
+                           const int64_t* cache_loc, uint8_t* k_cache, uint8_t* v_cache,
+                           float k_scale, float v_scale, int B, int L, int hq, int hkv,
+                           int max_pages, int64_t num_rows, int page_size, int window,
+                           int use_rope, const uint8_t* want, uint16_t* out, double* out_exact,
+                           double* attn_out, int nthreads) {
     if (B <= 0 || L <= 0 || max_pages <= 0 || num_rows <= 0 || page_size <= 0) return GADO_ERR_ARG;
+    if (hq <= 0 || hkv <= 0 || hq % hkv != 0) return GADO_ERR_ARG;
     if (!(k_scale > 0.0f) || !(v_scale > 0.0f)) return GADO_ERR_ARG;
     if (nthreads < 1) nthreads = 1;
     const int T = B * L;
     const double ks = (double)k_scale, vs = (double)v_scale;
+    const int64_t qkv_cols = (int64_t)(2 * hq + 2 * hkv) * GADO_D;
+    const int64_t k_off = (int64_t)hq * GADO_D, v_off = (int64_t)(hq + hkv) * GADO_D;
+    const int64_t row_bytes = (int64_t)hkv * GADO_D;
 
-    double* qn = (double*)malloc(sizeof(double) * (size_t)T * GADO_HQ * GADO_D);
+    double* qn = (double*)malloc(sizeof(double) * (size_t)T * hq * GADO_D);
     if (!qn) return GADO_ERR_NOMEM;
 
     /* Pass 1: split, QK-norm, RoPE, quantise and write this step's k, v. */
     for (int t = 0; t < T; ++t) {
-        const uint16_t* row_qkv = qkv + (int64_t)t * GADO_QKV_COLS;
+        const uint16_t* row_qkv = qkv + (int64_t)t * qkv_cols;
         const double p = (double)positions[t];
         double u[GADO_D];
-        for (int h = 0; h < GADO_HQ; ++h) {
-            for (int d = 0; d < GADO_D; ++d) u[d] = gado_bf16_decode(row_qkv[GADO_Q_OFF + h * GADO_D + d]);
-            double* qh = qn + ((int64_t)t * GADO_HQ + h) * GADO_D;
+        for (int h = 0; h < hq; ++h) {
+            for (int d = 0; d < GADO_D; ++d) u[d] = gado_bf16_decode(row_qkv[h * GADO_D + d]);
+            double* qh = qn + ((int64_t)t * hq + h) * GADO_D;
             gado_rmsnorm(u, qh, GADO_D, 1e-6);
             for (int d = 0; d < GADO_D; ++d) qh[d] *= 5.473;
             if (use_rope) gado_rope_neox(qh, GADO_D, p, 10000.0);
@@ -330,15 +341,15 @@ int gado_attn_decode(const uint16_t* qkv, const int64_t* positions, const int32_
             free(qn);
             return GADO_ERR_ROW;
         }
-        for (int g = 0; g < GADO_HKV; ++g) {
+        for (int g = 0; g < hkv; ++g) {
             double kh[GADO_D];
-            for (int d = 0; d < GADO_D; ++d) u[d] = gado_bf16_decode(row_qkv[GADO_K_OFF + g * GADO_D + d]);
+            for (int d = 0; d < GADO_D; ++d) u[d] = gado_bf16_decode(row_qkv[k_off + g * GADO_D + d]);
             gado_rmsnorm(u, kh, GADO_D, 1e-6);
             if (use_rope) gado_rope_neox(kh, GADO_D, p, 10000.0);
             for (int d = 0; d < GADO_D; ++d) {
-                double vv = gado_bf16_decode(row_qkv[GADO_V_OFF + g * GADO_D + d]);
-                k_cache[row * GADO_ROW_BYTES + g * GADO_D + d] = gado_e4m3_encode((float)(kh[d] / ks));
-                v_cache[row * GADO_ROW_BYTES + g * GADO_D + d] = gado_e4m3_encode((float)(vv / vs));
+                double vv = gado_bf16_decode(row_qkv[v_off + g * GADO_D + d]);
+                k_cache[row * row_bytes + g * GADO_D + d] = gado_e4m3_encode((float)(kh[d] / ks));
+                v_cache[row * row_bytes + g * GADO_D + d] = gado_e4m3_encode((float)(vv / vs));
             }
         }
     }
@@ -366,6 +377,8 @@ int gado_attn_decode(const uint16_t* qkv, const int64_t* positions, const int32_
         J->max_pages = max_pages;
         J->page_size = page_size;
         J->window = window;
+        J->hq = hq;
+        J->hkv = hkv;
         J->num_rows = num_rows;
         J->want = want;
         J->qn = qn;
@@ -389,4 +402,15 @@ int gado_attn_decode(const uint16_t* qkv, const int64_t* positions, const int32_
     free(th);
     free(qn);
     return status;
+}
+
+/* The page's per-GPU shapes: 16 query heads and 2 key/value heads. */
+int gado_attn_decode(const uint16_t* qkv, const int64_t* positions, const int32_t* page_table,
+                     const int64_t* cache_loc, uint8_t* k_cache, uint8_t* v_cache, float k_scale,
+                     float v_scale, int B, int L, int max_pages, int64_t num_rows, int page_size,
+                     int window, int use_rope, const uint8_t* want, uint16_t* out, double* out_exact,
+                     double* attn_out, int nthreads) {
+    return gado_attn_decode_heads(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale,
+                                  v_scale, B, L, GADO_HQ, GADO_HKV, max_pages, num_rows, page_size,
+                                  window, use_rope, want, out, out_exact, attn_out, nthreads);
 }

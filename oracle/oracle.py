@@ -23,8 +23,13 @@ _SRC = os.path.join(_HERE, "gad_oracle.c")
 _BUILD = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_BUILD, "libgad_oracle.so")
 
-HQ, HKV, D = 16, 2, 64
+HQ, HKV, D = 16, 2, 64   # the page's per-GPU shapes ("heads tp8")
 QKV_COLS = 2304
+
+
+def qkv_cols(hq: int, hkv: int) -> int:
+    """Columns of one qkv row: q (hq heads) | k (hkv) | v (hkv) | gate (hq), 64 each."""
+    return (2 * hq + 2 * hkv) * D
 
 
 def build(force: bool = False) -> str:
@@ -66,6 +71,11 @@ def lib() -> ctypes.CDLL:
             vp, vp, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp,
             ctypes.c_int]
+        L.gado_attn_decode_heads.restype = ctypes.c_int
+        L.gado_attn_decode_heads.argtypes = [
+            vp, vp, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, vp, vp, vp, vp, ctypes.c_int]
     return _lib
 
 
@@ -111,9 +121,9 @@ def rope_neox(u, pos: float, theta: float = 10000.0) -> np.ndarray:
 
 @dataclass
 class OracleResult:
-    out: np.ndarray        # uint16 bf16 bits [T, 1024]
-    out_exact: np.ndarray  # float64 [T, 1024], before bf16 rounding
-    attn: np.ndarray       # float64 [T, 1024], a before the output norm
+    out: np.ndarray        # uint16 bf16 bits [T, 64 hq]
+    out_exact: np.ndarray  # float64 [T, 64 hq], before bf16 rounding
+    attn: np.ndarray       # float64 [T, 64 hq], a before the output norm
     k_cache: np.ndarray    # uint8, after this step's writes
     v_cache: np.ndarray
 
@@ -126,37 +136,37 @@ def _np(x, dtype):
 
 def attn_decode(qkv_bits, positions, page_table, cache_loc, k_cache, v_cache, k_scale: float,
                 v_scale: float, page_size: int, window: int, use_rope: bool, want=None,
-                nthreads: int | None = None) -> OracleResult:
+                nthreads: int | None = None, hq: int = HQ, hkv: int = HKV) -> OracleResult:
     """Run the oracle on host arrays.  The caches are copied, not mutated.
 
-    qkv_bits: uint16 [T, 2304] (bf16 bit patterns); positions, cache_loc: int64 [T];
-    page_table: int32 [B, max_pages]; caches: uint8 [..., 128] (any leading shape).
-    want: optional bool [T, 16] selecting the (token, head) outputs to compute;
-    outputs that are not computed are left as 0.
+    qkv_bits: uint16 [T, qkv_cols(hq, hkv)] (bf16 bit patterns); positions,
+    cache_loc: int64 [T]; page_table: int32 [B, max_pages]; caches: uint8
+    [..., 64 hkv] (any leading shape).  want: optional bool [T, hq] selecting
+    the (token, head) outputs to compute; outputs not computed are left as 0.
     """
-    qkv = _np(qkv_bits, np.uint16).reshape(-1, QKV_COLS)
+    qkv = _np(qkv_bits, np.uint16).reshape(-1, qkv_cols(hq, hkv))
     pos = _np(positions, np.int64).reshape(-1)
     pt = _np(page_table, np.int32)
     B, max_pages = pt.shape
     cl = _np(cache_loc, np.int64).reshape(-1)
-    kc = np.array(_np(k_cache, np.uint8).reshape(-1, HKV * D), copy=True)
-    vc = np.array(_np(v_cache, np.uint8).reshape(-1, HKV * D), copy=True)
+    kc = np.array(_np(k_cache, np.uint8).reshape(-1, hkv * D), copy=True)
+    vc = np.array(_np(v_cache, np.uint8).reshape(-1, hkv * D), copy=True)
     T = qkv.shape[0]
     assert T % B == 0 and pos.size == T and cl.size == T
     L = T // B
     want_arr = None
     if want is not None:
-        want_arr = np.ascontiguousarray(np.asarray(want, dtype=bool).reshape(T, HQ), dtype=np.uint8)
-    out = np.zeros((T, HQ * D), np.uint16)
-    out_exact = np.zeros((T, HQ * D), np.float64)
-    attn = np.zeros((T, HQ * D), np.float64)
+        want_arr = np.ascontiguousarray(np.asarray(want, dtype=bool).reshape(T, hq), dtype=np.uint8)
+    out = np.zeros((T, hq * D), np.uint16)
+    out_exact = np.zeros((T, hq * D), np.float64)
+    attn = np.zeros((T, hq * D), np.float64)
     if nthreads is None:
         nthreads = os.cpu_count() or 1
     vp = lambda a: None if a is None else a.ctypes.data_as(ctypes.c_void_p)
-    st = lib().gado_attn_decode(
+    st = lib().gado_attn_decode_heads(
         vp(qkv), vp(pos), vp(pt), vp(cl), vp(kc), vp(vc), float(k_scale), float(v_scale), B, L,
-        max_pages, kc.shape[0], int(page_size), int(window), int(bool(use_rope)), vp(want_arr),
-        vp(out), vp(out_exact), vp(attn), int(nthreads))
+        int(hq), int(hkv), max_pages, kc.shape[0], int(page_size), int(window),
+        int(bool(use_rope)), vp(want_arr), vp(out), vp(out_exact), vp(attn), int(nthreads))
     if st != 0:
         raise RuntimeError(f"oracle gado_attn_decode failed with status {st}")
     return OracleResult(out, out_exact, attn, kc, vc)

@@ -385,6 +385,89 @@ def test_want_mask_computes_only_selected_heads():
 
 
 # ----------------------------------------------------------------------------
+# "heads dp": every head of the layer on one GPU (128 query, 16 KV heads)
+# ----------------------------------------------------------------------------
+
+DP_HQ, DP_HKV = 128, 16
+
+
+def _dp_tiny(seq_len, L=1, window=0, rope=False, seed=0):
+    rng = np.random.default_rng(seed)
+    total = seq_len + L
+    qkv = rng.normal(size=(L, O.qkv_cols(DP_HQ, DP_HKV))).astype(np.float32)
+    kc = _codes(rng.normal(size=(total, DP_HKV, 64)))
+    vc = _codes(rng.normal(size=(total, DP_HKV, 64)))
+    pt = np.arange(((total + 3) // 4) * 4, dtype=np.int32)[None, :]
+    pos = np.arange(seq_len, seq_len + L, dtype=np.int64)
+    return dict(qkv=qkv, kc=kc, vc=vc, pt=pt, pos=pos, cl=pos.copy(), window=window, rope=rope,
+                s=1.0)
+
+
+def _dp_run(c):
+    return O.attn_decode(_bf16_bits(c["qkv"]), c["pos"], c["pt"], c["cl"], c["kc"], c["vc"],
+                         c["s"], c["s"], 1, c["window"], c["rope"], nthreads=2, hq=DP_HQ,
+                         hkv=DP_HKV)
+
+
+@pytest.mark.parametrize("L,window,rope", [(1, 0, False), (8, 0, False), (8, 16, True)])
+def test_heads_dp_step_is_eight_tp8_steps(L, window, rope):
+    """Query heads 8k..8k+7 only ever meet KV head k, so a step over 128/16
+    heads must equal eight 16/2-head steps on the matching column slices:
+    q and gate columns 1024 g.. (16 heads), k and v columns 128 g.. (2 heads)
+    of their own sections, cache bytes 128 g.. of each row."""
+    c = _dp_tiny(29, L=L, window=window, rope=rope, seed=21)
+    dp = _dp_run(c)
+    q_sec, k_sec = 0, DP_HQ * 64
+    v_sec, g_sec = k_sec + DP_HKV * 64, k_sec + 2 * DP_HKV * 64
+    for g in range(DP_HKV // 2):
+        sub = dict(c)
+        sub["qkv"] = np.concatenate(
+            [c["qkv"][:, q_sec + 1024 * g:q_sec + 1024 * (g + 1)],
+             c["qkv"][:, k_sec + 128 * g:k_sec + 128 * (g + 1)],
+             c["qkv"][:, v_sec + 128 * g:v_sec + 128 * (g + 1)],
+             c["qkv"][:, g_sec + 1024 * g:g_sec + 1024 * (g + 1)]], axis=1)
+        sub["kc"] = np.ascontiguousarray(c["kc"][:, 2 * g:2 * g + 2])
+        sub["vc"] = np.ascontiguousarray(c["vc"][:, 2 * g:2 * g + 2])
+        tp = _run(sub)
+        assert np.array_equal(dp.out[:, 1024 * g:1024 * (g + 1)], tp.out)
+        assert np.array_equal(dp.k_cache[:, 128 * g:128 * (g + 1)], tp.k_cache)
+        assert np.array_equal(dp.v_cache[:, 128 * g:128 * (g + 1)], tp.v_cache)
+
+
+def test_heads_dp_query_head_reads_kv_head_h_div_8():
+    """Two keys per KV head: for even KV heads the cached key wins, for odd
+    ones the new key; the winning value is +-(k+1)/4 on KV head k (exact in
+    E4M3 and bf16), so each query head's a names the KV head it read."""
+    c = _dp_tiny(1, seed=22)
+    ks, vs = DP_HQ * 64, DP_HQ * 64 + DP_HKV * 64
+    c["qkv"][:, 0:ks] = 1.0                                   # q = ones on every head
+    for k in range(DP_HKV):
+        sign = 1.0 if k % 2 else -1.0                         # new key +ones wins on odd heads
+        c["qkv"][:, ks + 64 * k:ks + 64 * (k + 1)] = sign
+        c["kc"][0, k] = 0xB8 if k % 2 else 0x38               # cached key: the other sign
+        c["vc"][0, k] = _codes(np.full(64, (k + 1) / 4))      # cached value +(k+1)/4
+        c["qkv"][:, vs + 64 * k:vs + 64 * (k + 1)] = -(k + 1) / 4  # new value -(k+1)/4
+    r = _dp_run(c)
+    for h in range(DP_HQ):
+        k = h // 8
+        want = -(k + 1) / 4 if k % 2 else (k + 1) / 4
+        assert np.allclose(r.attn[0, 64 * h:64 * (h + 1)], want, rtol=1e-12, atol=0), h
+
+
+def test_heads_dp_gate_columns():
+    """A gate of -inf-like size on one query head zeroes that head's output
+    alone; the gate section starts at column 64 (hq + 2 hkv) = 10240."""
+    c = _dp_tiny(5, seed=23)
+    gs = (DP_HQ + 2 * DP_HKV) * 64
+    c["qkv"][:, gs + 64 * 77:gs + 64 * 78] = -200.0
+    r = _dp_run(c)
+    vals = O.bf16_bits_to_float(r.out[0]).reshape(DP_HQ, 64)
+    assert (vals[77] == 0).all()                              # +-0 after bf16 rounding
+    others = np.delete(vals, 77, axis=0)
+    assert (others != 0).sum(axis=1).min() > 32
+
+
+# ----------------------------------------------------------------------------
 # The page's own numbers: the floor column of the load table
 # ----------------------------------------------------------------------------
 
