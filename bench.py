@@ -145,22 +145,23 @@ def oracle_cpu_rate(inp: dict, max_key_heads: float = 40e6) -> dict:
         lo = max(0, int(pos[b, 0]) - W_ + 1) if W_ > 0 else 0
         keys.append(int(pos[b, -1]) - lo + 1)
     nb, kh = 0, 0.0
-    while nb < B and (nb == 0 or kh + keys[nb] * 16 * L <= max_key_heads):
-        kh += keys[nb] * 16 * L
+    hq, hkv = inp.get("hq", 16), inp.get("hkv", 2)
+    while nb < B and (nb == 0 or kh + keys[nb] * hq * L <= max_key_heads):
+        kh += keys[nb] * hq * L
         nb += 1
     T = nb * L
     qkv = inp["qkv"][:T].view(torch.int16).numpy().astype(np.uint16)
     threads = os.cpu_count() or 1
     t = time.perf_counter()
     O.attn_decode(qkv, inp["positions"][:T], inp["page_table"][:nb], inp["cache_loc"][:T],
-                  inp["k_cache"].reshape(-1, 128), inp["v_cache"].reshape(-1, 128),
+                  inp["k_cache"].reshape(-1, 64 * hkv), inp["v_cache"].reshape(-1, 64 * hkv),
                   inp["k_scale"], inp["v_scale"], inp["page_size"], inp["window"],
-                  inp["use_rope"], nthreads=threads)
+                  inp["use_rope"], nthreads=threads, hq=hq, hkv=hkv)
     dt = time.perf_counter() - t
-    kv = sum(keys[:nb]) * BYTES_PER_KEY
+    kv = sum(keys[:nb]) * 2 * 64 * hkv
     return {"value": kv / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "seconds": dt,
-            "sample": f"requests 0..{nb - 1} of {B} ({sum(keys[:nb])} keys, all 16 heads x {L} "
+            "sample": f"requests 0..{nb - 1} of {B} ({sum(keys[:nb])} keys, all {hq} heads x {L} "
                       f"tokens), FP64 C oracle incl. its cache copy"}
 
 
@@ -330,17 +331,19 @@ def main():
     spec = W.named(args.workload, seed=replicas.replica_seed(0, rank))
     inp = W.make_inputs(spec)
     B, L, ps = inp["B"], inp["L"], inp["page_size"]
+    hq, hkv = inp["hq"], inp["hkv"]
     T = B * L
     keys = W.keys_attended(inp)
-    kv_bytes = keys * BYTES_PER_KEY
-    alg_bytes = keys * (BYTES_PER_KEY + PT_BYTES_PER_KEY[ps])   # decode kernel, per launch
+    bpk = BYTES_PER_KEY * hkv // 2                               # K and V bytes per key
+    kv_bytes = keys * bpk
+    alg_bytes = keys * (bpk + PT_BYTES_PER_KEY[ps])              # decode kernel, per launch
 
     d = {k: inp[k].to(dev) for k in ("qkv", "positions", "seq_lens", "page_table", "cache_loc",
                                        "k_cache", "v_cache")}
     k_scale = torch.tensor([inp["k_scale"]], dtype=torch.float32, device=dev)
     v_scale = torch.tensor([inp["v_scale"]], dtype=torch.float32, device=dev)
-    out = torch.empty(B, L, 1024, dtype=torch.bfloat16, device=dev)
-    ws = binding.alloc_workspace(B, L, dev)
+    out = torch.empty(B, L, 64 * hq, dtype=torch.bfloat16, device=dev)
+    ws = binding.alloc_workspace(B, L, dev, hq, hkv)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # 256 MiB > 126 MB L2
     flush_sink = torch.empty((), dtype=torch.int64, device=dev)
 
@@ -348,7 +351,7 @@ def main():
         binding.attn_decode(d["qkv"], d["positions"], d["seq_lens"], d["page_table"],
                             d["cache_loc"], d["k_cache"], d["v_cache"], k_scale, v_scale, ps,
                             inp["window"], inp["use_rope"], L=L, out=out, workspace=ws,
-                            events=events)
+                            events=events, hq=hq, hkv=hkv)
 
     def cold_l2():
         flush.fill_(1)                                     # write > L2 ...
@@ -413,7 +416,7 @@ def main():
     # Per-token step inputs come from the host every step; the KV cache and the
     # page table are device-resident state, as a serving stack keeps them.
     host = {k: inp[k].pin_memory() for k in ("qkv", "positions", "seq_lens", "cache_loc")}
-    out_host = torch.empty(B, L, 1024, dtype=torch.bfloat16).pin_memory()
+    out_host = torch.empty(B, L, 64 * hq, dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host.numel() * out_host.element_size()
 
@@ -471,7 +474,7 @@ def main():
         "dtype": "e4m3 cache, f16 MMA / f32 accumulate, bf16 out",
         "data": "synthetic",
         "config": {
-            "workload": args.workload, "B": B, "L": L, "page_size": ps,
+            "workload": args.workload, "B": B, "L": L, "heads": [hq, hkv], "page_size": ps,
             "window": inp["window"], "use_rope": inp["use_rope"],
             "keys_attended": keys, "kv_bytes_per_step": kv_bytes,
             "parallelism": f"replicas x{world}",

@@ -15,7 +15,9 @@
  *   out = rmsnorm(a) * sigmoid(gate)                   bf16
  *
  * Model shape (section "Shapes"): 16 query heads, 2 KV heads, head dim 64;
- * query head h reads KV head h / 8.  Readings of points the page leaves open:
+ * query head h reads KV head h / 8.  The page's tests also run "heads dp",
+ * read here as every head of the layer on one GPU (128 query, 16 KV heads);
+ * gad_attn_decode_heads takes such head counts.  Readings of points the page leaves open:
  * rmsnorm eps 1e-6 with unit weights; RoPE is the NeoX half-split rotation of
  * dims (i, i+32) by p * 10000^(-2i/64); a sliding window W attends keys i with
  * p - W < i <= p; stored code = E4M3(x / scale) with round-to-nearest-even and
@@ -37,7 +39,8 @@
 extern "C" {
 #endif
 
-/* Fixed model shape. */
+/* The page's per-GPU shape ("heads tp8"); gad_attn_decode_heads takes
+ * multiples of it. */
 #define GAD_HQ 16          /* query heads per GPU            */
 #define GAD_HKV 2          /* key/value heads per GPU        */
 #define GAD_HEAD_DIM 64
@@ -54,7 +57,8 @@ typedef enum {
     GAD_ERR_NULL = -1,        /* a required pointer is NULL                     */
     GAD_ERR_SHAPE = -2,       /* B, L, max_pages or num_rows out of range       */
     GAD_ERR_ALIGN = -3,       /* a pointer is not aligned as documented         */
-    GAD_ERR_UNSUPPORTED = -4, /* page_size not 1 or 64, or window < 0           */
+    GAD_ERR_UNSUPPORTED = -4, /* page_size not 1 or 64, window < 0, or head
+                                 counts other than hq = 8 hkv, hkv = 2, 4, 6 .. */
     GAD_ERR_WORKSPACE = -5,   /* workspace NULL or smaller than required        */
     GAD_ERR_CUDA = -6,        /* a CUDA call or kernel launch failed            */
     GAD_ERR_DEVICE = -7       /* current device is not compute capability 10.x  */
@@ -67,6 +71,15 @@ typedef enum {
  * device is present.  Host-only; launches nothing.
  */
 size_t gad_attn_workspace_bytes(int B, int L);
+
+/*
+ * Workspace bytes of gad_attn_decode_heads for B requests of L tokens with
+ * hq query and hkv KV heads, on the CURRENT device.  Returns 0 and sets
+ * gad_last_error() on the same conditions as gad_attn_workspace_bytes and on
+ * unsupported head counts.  gad_attn_workspace_bytes(B, L) equals
+ * gad_attn_workspace_bytes_heads(B, L, 16, 2).  Host-only.
+ */
+size_t gad_attn_workspace_bytes_heads(int B, int L, int hq, int hkv);
 
 /*
  * One step.  T = B * L tokens; token t = b * L + j is token j of request b.
@@ -115,6 +128,32 @@ int gad_attn_decode(const void* qkv, const int64_t* positions, const int32_t* se
                     void* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * gad_attn_decode for other head counts: hq query heads over hkv KV heads,
+ * with hkv a positive multiple of 2 and hq = 8 hkv (query head h reads KV
+ * head h / 8), e.g. hq = 128, hkv = 16 for the page's "heads dp" tests
+ * (section "Shapes" and its list of tests).  gad_attn_decode is this call
+ * with hq = 16, hkv = 2.  The layouts widen with the head counts:
+ *
+ *   qkv         bf16 [T, 64 (2 hq + 2 hkv)]: q heads [0, 64 hq), k heads
+ *               [64 hq, 64 (hq + hkv)), v heads [.., 64 (hq + 2 hkv)), gate
+ *               [.., 64 (2 hq + 2 hkv)); each head 64 contiguous values.
+ *   k_cache,    uint8 [num_rows, hkv, 64] E4M3 codes (64 hkv bytes per row).
+ *   v_cache
+ *   out         bf16 [T, 64 hq].
+ *   workspace   at least gad_attn_workspace_bytes_heads(B, L, hq, hkv) bytes.
+ *
+ * B * hkv / 2 may not exceed GAD_MAX_B (GAD_ERR_SHAPE).  Other head counts
+ * return GAD_ERR_UNSUPPORTED.  Every other argument, the error behaviour and
+ * the contract are those of gad_attn_decode.
+ */
+int gad_attn_decode_heads(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                          const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,
+                          uint8_t* v_cache, const float* k_scale, const float* v_scale, int B,
+                          int L, int hq, int hkv, int max_pages, int64_t num_rows, int page_size,
+                          int window, int use_rope, void* out, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/*
  * Profiling variant of gad_attn_decode: same arguments and semantics, plus
  * `events`, an array of four cudaEvent_t created by the caller.  It records
  * events[0] before the prep kernel, events[1] between prep and decode,
@@ -130,6 +169,18 @@ int gad_attn_decode_timed(const void* qkv, const int64_t* positions, const int32
                           int L, int max_pages, int64_t num_rows, int page_size, int window,
                           int use_rope, void* out, void* workspace, size_t workspace_bytes,
                           void* stream, void* const* events);
+
+/*
+ * Profiling variant of gad_attn_decode_heads: its arguments plus the four
+ * events of gad_attn_decode_timed, recorded the same way.
+ */
+int gad_attn_decode_heads_timed(const void* qkv, const int64_t* positions,
+                                const int32_t* seq_lens, const int32_t* page_table,
+                                const int64_t* cache_loc, uint8_t* k_cache, uint8_t* v_cache,
+                                const float* k_scale, const float* v_scale, int B, int L, int hq,
+                                int hkv, int max_pages, int64_t num_rows, int page_size,
+                                int window, int use_rope, void* out, void* workspace,
+                                size_t workspace_bytes, void* stream, void* const* events);
 
 /*
  * Allocation-free variant of gad_attn_decode.  The page has no counterpart:

@@ -32,6 +32,14 @@ _lib.gad_attn_decode.argtypes = [
     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,  # B, L, max_pages, num_rows
     ctypes.c_int, ctypes.c_int, ctypes.c_int,               # page_size, window, use_rope
     _vp, _vp, ctypes.c_size_t, _vp]                         # out, workspace, bytes, stream
+_lib.gad_attn_workspace_bytes_heads.restype = ctypes.c_size_t
+_lib.gad_attn_workspace_bytes_heads.argtypes = [ctypes.c_int] * 4
+_lib.gad_attn_decode_heads.restype = ctypes.c_int
+_lib.gad_attn_decode_heads.argtypes = (list(_lib.gad_attn_decode.argtypes[:11])
+                                       + [ctypes.c_int, ctypes.c_int]  # hq, hkv
+                                       + list(_lib.gad_attn_decode.argtypes[11:]))
+_lib.gad_attn_decode_heads_timed.restype = ctypes.c_int
+_lib.gad_attn_decode_heads_timed.argtypes = list(_lib.gad_attn_decode_heads.argtypes) + [_vp]
 _lib.gad_attn_decode_timed.restype = ctypes.c_int
 _lib.gad_attn_decode_timed.argtypes = list(_lib.gad_attn_decode.argtypes) + [_vp]
 _lib.gad_attn_decode_noalloc.restype = ctypes.c_int
@@ -44,8 +52,10 @@ _lib.gad_status_string.argtypes = [ctypes.c_int]
 HQ, HKV, D = 16, 2, 64
 QKV_COLS, OUT_COLS, ROW_BYTES = 2304, 1024, 128
 
-EXPORTED = ("gad_attn_decode", "gad_attn_decode_timed", "gad_attn_decode_noalloc",
-            "gad_attn_workspace_bytes", "gad_last_error", "gad_status_string")
+EXPORTED = ("gad_attn_decode", "gad_attn_decode_heads", "gad_attn_decode_timed",
+            "gad_attn_decode_heads_timed",
+            "gad_attn_decode_noalloc", "gad_attn_workspace_bytes",
+            "gad_attn_workspace_bytes_heads", "gad_last_error", "gad_status_string")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -61,16 +71,20 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
-def workspace_bytes(B: int, L: int) -> int:
-    n = _lib.gad_attn_workspace_bytes(int(B), int(L))
+def workspace_bytes(B: int, L: int, hq: int = HQ, hkv: int = HKV) -> int:
+    if (hq, hkv) == (HQ, HKV):
+        n = _lib.gad_attn_workspace_bytes(int(B), int(L))
+    else:
+        n = _lib.gad_attn_workspace_bytes_heads(int(B), int(L), int(hq), int(hkv))
     if n == 0:
         raise GadError(-2, "gad_attn_workspace_bytes")
     return int(n)
 
 
-def alloc_workspace(B: int, L: int, device=None) -> torch.Tensor:
+def alloc_workspace(B: int, L: int, device=None, hq: int = HQ, hkv: int = HKV) -> torch.Tensor:
     """Caller-owned scratch for gad_attn_decode (256-byte aligned by torch's allocator)."""
-    return torch.empty(workspace_bytes(B, L), dtype=torch.uint8, device=device or "cuda")
+    return torch.empty(workspace_bytes(B, L, hq, hkv), dtype=torch.uint8,
+                       device=device or "cuda")
 
 
 def _ptr(t: torch.Tensor | None):
@@ -96,14 +110,15 @@ def attn_decode(qkv: torch.Tensor, positions: torch.Tensor, seq_lens: torch.Tens
                 page_size: int, window: int, use_rope: bool, L: int = 1,
                 out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                 stream: torch.cuda.Stream | None = None,
-                events: list | None = None) -> torch.Tensor:
-    """One decode step (L = 1) or verify block (L <= 8); returns out bf16 [B, L, 1024].
+                events: list | None = None, hq: int = HQ, hkv: int = HKV) -> torch.Tensor:
+    """One decode step (L = 1) or verify block (L <= 8); returns out bf16 [B, L, 64 hq].
 
-    Shapes: qkv bf16 [B*L, 2304]; positions, cache_loc int64 [B*L]; seq_lens int32 [B]
-    (optional); page_table int32 [B, max_pages]; k_cache / v_cache uint8
-    [num_pages, page_size, 2, 64] (mutated in the rows cache_loc); k_scale / v_scale
-    float32 [1] on the device.  With ``events`` (four torch.cuda.Event with timing),
-    the profiling entry point records them around the three kernels.
+    Shapes: qkv bf16 [B*L, 64 (2 hq + 2 hkv)]; positions, cache_loc int64 [B*L];
+    seq_lens int32 [B] (optional); page_table int32 [B, max_pages]; k_cache / v_cache
+    uint8 [num_pages, page_size, hkv, 64] (mutated in the rows cache_loc); k_scale /
+    v_scale float32 [1] on the device.  hq, hkv: head counts (16, 2 by default; other
+    counts go through gad_attn_decode_heads).  With ``events`` (four torch.cuda.Event
+    with timing), the profiling entry point records them around the three kernels.
     """
     _need(qkv, "qkv", torch.bfloat16, 2)
     _need(positions, "positions", torch.int64, 1)
@@ -117,30 +132,34 @@ def attn_decode(qkv: torch.Tensor, positions: torch.Tensor, seq_lens: torch.Tens
         _need(seq_lens, "seq_lens", torch.int32, 1)
     B, max_pages = page_table.shape
     T = qkv.shape[0]
-    if qkv.shape[1] != QKV_COLS or T != B * L:
-        raise ValueError(f"qkv must be [B*L={B * L}, {QKV_COLS}], got {tuple(qkv.shape)}")
+    qkv_cols, out_cols, row_bytes = (2 * hq + 2 * hkv) * D, hq * D, hkv * D
+    if qkv.shape[1] != qkv_cols or T != B * L:
+        raise ValueError(f"qkv must be [B*L={B * L}, {qkv_cols}], got {tuple(qkv.shape)}")
     if positions.numel() != T or cache_loc.numel() != T:
         raise ValueError("positions and cache_loc need one entry per token")
-    if k_cache.shape != v_cache.shape or k_cache.numel() % ROW_BYTES:
-        raise ValueError("k_cache and v_cache must have the same shape, 128 bytes per row")
-    num_rows = k_cache.numel() // ROW_BYTES
+    if k_cache.shape != v_cache.shape or k_cache.numel() % row_bytes:
+        raise ValueError(f"k_cache and v_cache must have the same shape, {row_bytes} bytes per row")
+    num_rows = k_cache.numel() // row_bytes
     if out is None:
-        out = torch.empty(B, L, OUT_COLS, dtype=torch.bfloat16, device=qkv.device)
+        out = torch.empty(B, L, out_cols, dtype=torch.bfloat16, device=qkv.device)
     else:
         _need(out, "out", torch.bfloat16)
-        if out.numel() != T * OUT_COLS:
-            raise ValueError("out must hold B*L*1024 values")
+        if out.numel() != T * out_cols:
+            raise ValueError(f"out must hold B*L*{out_cols} values")
     if workspace is None:
-        workspace = alloc_workspace(B, L, qkv.device)
+        workspace = alloc_workspace(B, L, qkv.device, hq, hkv)
     else:
         _need(workspace, "workspace", torch.uint8)
     s = (stream or torch.cuda.current_stream(qkv.device)).cuda_stream
-    args = (_ptr(qkv), _ptr(positions), _ptr(seq_lens), _ptr(page_table), _ptr(cache_loc),
-            _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), int(B), int(L),
-            int(max_pages), int(num_rows), int(page_size), int(window), int(bool(use_rope)),
+    head = (_ptr(qkv), _ptr(positions), _ptr(seq_lens), _ptr(page_table), _ptr(cache_loc),
+            _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), int(B), int(L))
+    tail = (int(max_pages), int(num_rows), int(page_size), int(window), int(bool(use_rope)),
             _ptr(out), _ptr(workspace), int(workspace.numel()), ctypes.c_void_p(s))
+    args = head + tail
+    tp8 = (hq, hkv) == (HQ, HKV)
     if events is None:
-        st = _lib.gad_attn_decode(*args)
+        st = _lib.gad_attn_decode(*args) if tp8 else \
+            _lib.gad_attn_decode_heads(*head, int(hq), int(hkv), *tail)
     else:
         if len(events) != 4:
             raise ValueError("events must hold four torch.cuda.Event")
@@ -148,7 +167,8 @@ def attn_decode(qkv: torch.Tensor, positions: torch.Tensor, seq_lens: torch.Tens
             if ev.cuda_event == 0:
                 ev.record()
         arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(ev.cuda_event) for ev in events])
-        st = _lib.gad_attn_decode_timed(*args, arr)
+        st = _lib.gad_attn_decode_timed(*args, arr) if tp8 else \
+            _lib.gad_attn_decode_heads_timed(*head, int(hq), int(hkv), *tail, arr)
     if st != 0:
         raise GadError(st, "gad_attn_decode")
     return out
@@ -191,11 +211,13 @@ def raw_call(**kw) -> int:
     args = [kw.get(k) for k in ("qkv", "positions", "seq_lens", "page_table", "cache_loc",
                                 "k_cache", "v_cache", "k_scale", "v_scale")]
     args = [a if (a is None or isinstance(a, ctypes.c_void_p)) else ctypes.c_void_p(a) for a in args]
-    return _lib.gad_attn_decode(*args, kw.get("B", 1), kw.get("L", 1), kw.get("max_pages", 1),
-                                kw.get("num_rows", 1), kw.get("page_size", 1),
-                                kw.get("window", 0), kw.get("use_rope", 0), kw.get("out"),
-                                kw.get("workspace"), kw.get("workspace_bytes", 0),
-                                kw.get("stream"))
+    args += [kw.get("B", 1), kw.get("L", 1)]
+    rest = [kw.get("max_pages", 1), kw.get("num_rows", 1), kw.get("page_size", 1),
+            kw.get("window", 0), kw.get("use_rope", 0), kw.get("out"), kw.get("workspace"),
+            kw.get("workspace_bytes", 0), kw.get("stream")]
+    if "hq" in kw or "hkv" in kw:   # through gad_attn_decode_heads
+        return _lib.gad_attn_decode_heads(*args, kw.get("hq", HQ), kw.get("hkv", HKV), *rest)
+    return _lib.gad_attn_decode(*args, *rest)
 
 
 def last_error() -> str:

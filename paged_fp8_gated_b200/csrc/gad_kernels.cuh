@@ -25,14 +25,25 @@
 
 namespace gad {
 
-constexpr int HQ = 16;         // query heads
-constexpr int HKV = 2;         // key/value heads
+// Head groups.  The kernels work on groups of 16 query heads over 2 KV heads
+// (query head h of a group reads its KV head h / 8).  The page's "heads tp8"
+// shapes are one group; a step with ngrp groups (16 ngrp query heads, 2 ngrp
+// KV heads, e.g. 8 groups for "heads dp") is ngrp independent problems that
+// share positions, pages and cache rows.  Columns of a qkv row, for group c:
+//   q    c * 1024 + 64 h                    (section of 1024 ngrp columns)
+//   k    1024 ngrp + 128 c + 64 g           (section of 128 ngrp)
+//   v    1152 ngrp + 128 c + 64 g           (section of 128 ngrp)
+//   gate 1280 ngrp + 1024 c + 64 h          (section of 1024 ngrp)
+// a cache row holds 128 ngrp bytes (group c at byte 128 c), and an output row
+// 1024 ngrp values (group c at 1024 c).
+constexpr int HQ = 16;         // query heads of a group
+constexpr int HKV = 2;         // key/value heads of a group
 constexpr int HD = 64;         // head dim
 constexpr int GRP = HQ / HKV;  // query heads per KV head (8)
-constexpr int QKV_COLS = 2304;
-constexpr int K_OFF = 1024, V_OFF = 1152, G_OFF = 1280;
-constexpr int OUT_COLS = 1024;
-constexpr int ROWB = 128;                   // bytes per cache row: 2 KV heads x 64 codes
+constexpr int QKV_COLS = 2304; // qkv columns per group
+constexpr int K_OFF = 1024, V_OFF = 1152, G_OFF = 1280;  // section starts per group
+constexpr int OUT_COLS = 1024; // output columns per group
+constexpr int ROWB = 128;                   // cache bytes per row and group: 2 KV heads x 64 codes
 constexpr int TILE = 64;                    // keys per pipeline stage
 constexpr int STAGE_BYTES = 2 * TILE * ROWB;  // K tile then V tile: 16 KB
 constexpr int DEC_THREADS = 256;
@@ -49,40 +60,48 @@ struct StepParams {
     const float* v_scale;
     __nv_bfloat16* out;
     int B, L, max_pages, window, use_rope;
+    int ngrp;        // head groups (16 query + 2 KV heads each)
+    int NB;          // items of the tile list: B * ngrp; item i = (request i / ngrp, group i % ngrp)
     int64_t num_rows;
     // workspace views
-    __half* q_ws;    // [T][16][64]  normalised (rotated) queries
-    float* part_o;   // [slots][lt][16][64]  un-normalised partial outputs
+    __half* q_ws;    // [T][ngrp][16][64]  normalised (rotated) queries
+    float* part_o;   // [slots][lt][16][64]  un-normalised partial outputs (slot = CTA + item)
     float* part_ml;  // [slots][lt][16][2]   (running max in log2 units, sum)
-    int* meta;       // see META_*: tile count, tiles per CTA, error word, tile prefix
+    int* meta;       // see META_*: tile count, tiles per CTA, error word, tile prefix over items
     int lt;          // token capacity of one partial slot (1 or 8)
     int tl;          // partials per (CTA, request) and KV-head group
 };
+
+// List item -> (request, head group).  One group is the common case, kept
+// free of integer divisions.
+__device__ __forceinline__ int item_req(int b, int ng) { return ng == 1 ? b : b / ng; }
+__device__ __forceinline__ int item_grp(int b, int ng) { return ng == 1 ? 0 : b % ng; }
 
 // Layout of StepParams::meta (ints).
 constexpr int META_TOTAL = 0;    // tiles in the step
 constexpr int META_PER = 1;      // tiles per CTA
 constexpr int META_ERROR = 2;    // nonzero: a bounded wait in the decode kernel timed out
-constexpr int META_PREFIX = 3;   // [B + 1] tile prefix over requests
-constexpr int META_INTS = 4;     // + B
+constexpr int META_PREFIX = 3;   // [NB + 1] tile prefix over list items
+constexpr int META_INTS = 4;     // + NB
 
 // ---------------------------------------------------------------------------
 // Kernel 1: split + QK-norm + RoPE + E4M3 quantise-and-scatter.
-// One block per token; warp w < 16 handles query head w, warps 16 and 17 the
-// two KV heads.  Lane l owns the RoPE pair (l, l + 32).  Done in double so the
+// One block per (token, head group); warp w < 16 handles query head w of the
+// group, warps 16 and 17 its two KV heads.  Lane l owns the RoPE pair (l, l + 32).  Done in double so the
 // cache bytes match the double-precision definition exactly: the sum of squares
 // runs in index order with explicit round-to-nearest operations (no fused
 // multiply-add), as does the rotation.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) {
     pdl_launch_dependents();
-    const int t = blockIdx.x;
-    if (t == 0 && threadIdx.x == 0) p.meta[META_ERROR] = 0;
+    const int ng = p.ngrp;
+    const int t = blockIdx.x / ng, c = blockIdx.x % ng;
+    if (blockIdx.x == 0 && threadIdx.x == 0) p.meta[META_ERROR] = 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const __nv_bfloat16* row = p.qkv + static_cast<size_t>(t) * QKV_COLS;
+    const __nv_bfloat16* row = p.qkv + static_cast<size_t>(t) * QKV_COLS * ng;
     const bool is_q = warp < HQ;
     const int g = warp - HQ;
-    const int off = is_q ? warp * HD : K_OFF + g * HD;
+    const int off = is_q ? c * OUT_COLS + warp * HD : K_OFF * ng + c * ROWB + g * HD;
     const double x0 = static_cast<double>(__bfloat162float(row[off + lane]));
     const double x1 = static_cast<double>(__bfloat162float(row[off + lane + 32]));
 
@@ -112,7 +131,7 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) 
         u1 = r1;
     }
     if (is_q) {
-        __half* q = p.q_ws + (static_cast<size_t>(t) * HQ + warp) * HD;
+        __half* q = p.q_ws + (static_cast<size_t>(blockIdx.x) * HQ + warp) * HD;
         q[lane] = __double2half(u0);
         q[lane + 32] = __double2half(u1);
         return;
@@ -121,12 +140,14 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) 
     if (crow < 0 || crow >= p.num_rows) return;
     const double ks = static_cast<double>(__ldg(p.k_scale));
     const double vs = static_cast<double>(__ldg(p.v_scale));
-    uint8_t* kd = p.k_cache + crow * ROWB + g * HD;
-    uint8_t* vd = p.v_cache + crow * ROWB + g * HD;
+    const int64_t cofs = crow * (ROWB * ng) + c * ROWB + g * HD;
+    uint8_t* kd = p.k_cache + cofs;
+    uint8_t* vd = p.v_cache + cofs;
     kd[lane] = __nv_cvt_float_to_fp8(__double2float_rn(u0 / ks), __NV_SATFINITE, __NV_E4M3);
     kd[lane + 32] = __nv_cvt_float_to_fp8(__double2float_rn(u1 / ks), __NV_SATFINITE, __NV_E4M3);
-    const double v0 = static_cast<double>(__bfloat162float(row[V_OFF + g * HD + lane]));
-    const double v1 = static_cast<double>(__bfloat162float(row[V_OFF + g * HD + lane + 32]));
+    const int voff = V_OFF * ng + c * ROWB + g * HD;
+    const double v0 = static_cast<double>(__bfloat162float(row[voff + lane]));
+    const double v1 = static_cast<double>(__bfloat162float(row[voff + lane + 32]));
     vd[lane] = __nv_cvt_float_to_fp8(__double2float_rn(v0 / vs), __NV_SATFINITE, __NV_E4M3);
     vd[lane + 32] = __nv_cvt_float_to_fp8(__double2float_rn(v1 / vs), __NV_SATFINITE, __NV_E4M3);
 }
@@ -159,21 +180,24 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) 
 // runs its own online softmax over its keys; key groups are merged in shared
 // memory at the end of each segment.
 // ---------------------------------------------------------------------------
-// Per-request key ranges [lo_b, hi_b] (union over the request's tokens), the
-// first key this step writes (rnew_b), the
-// prefix of TK-key tile counts over requests (tiles aligned to multiples of TK), and this CTA's share of the tile
-// list [t0, t1).  Every thread of the block must call it.  CTA 0 also writes the
-// list to the workspace for the combine kernel.
-template <int TK>
+// Per-item key ranges [lo_i, hi_i] (union over the item's request's tokens),
+// the first key this step writes (rnew_i), the prefix of TK-key tile counts
+// over the list items (tiles aligned to multiples of TK), and this CTA's share
+// of the tile list [t0, t1).  Item i is request i / ngrp and head group
+// i % ngrp, so a request's groups are adjacent in the list and the CTAs that
+// share its pages run at about the same time.  Every thread of the block must
+// call it.  CTA 0 also writes the list to the workspace for the combine kernel.
+template <int TK, bool GROUPS>
 __device__ __forceinline__ void build_tile_list(const StepParams& p, int* tpre, int* rlo, int* rhi,
                                                 int* rnew, int nthreads, int& total, int& per,
                                                 int& t0, int& t1) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int B = p.B, L = p.L;
+    const int B = GROUPS ? p.NB : p.B, L = p.L, ng = GROUPS ? p.ngrp : 1;
     for (int b = tid; b < B; b += nthreads) {
+        const int req = item_req(b, ng);
         int lo = INT_MAX, hi = -1, first = INT_MAX;
         for (int j = 0; j < L; ++j) {
-            const int pos = static_cast<int>(p.positions[static_cast<size_t>(b) * L + j]);
+            const int pos = static_cast<int>(p.positions[static_cast<size_t>(req) * L + j]);
             const int l = p.window > 0 ? max(0, pos - p.window + 1) : 0;
             lo = min(lo, l);
             hi = max(hi, pos);
@@ -245,7 +269,9 @@ __device__ __forceinline__ int kappa(int l) {
     return (l & 8) | s;
 }
 
-template <int LT, int PS, int KG, int NS, int MINB, int TK, bool MERGE>
+// GROUPS: more than one head group (the one-group instantiation keeps the
+// list item equal to the request, with no index arithmetic for groups).
+template <int LT, int PS, int KG, int NS, int MINB, int TK, bool MERGE, bool GROUPS>
 __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepParams p) {
     using C = DecodeCfg<LT, KG, NS, TK, MERGE>;
     constexpr int NT = C::NT, MT = C::MT, RG = C::RG;
@@ -254,20 +280,22 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
     int* idx_smem = reinterpret_cast<int*>(smem + C::KV_BYTES);
     float* merge_smem = reinterpret_cast<float*>(smem + C::KV_BYTES + C::IDX_BYTES);
     int* tpre = reinterpret_cast<int*>(smem + C::KV_BYTES + C::IDX_BYTES + C::MERGE_BYTES);
-    int* rlo = tpre + p.B + 1;
-    int* rhi = rlo + p.B;
-    int* rnew = rhi + p.B;
+    int* rlo = tpre + p.NB + 1;
+    int* rhi = rlo + p.NB;
+    int* rnew = rhi + p.NB;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gid = lane >> 2, tig = lane & 3;
     const int g = warp % HKV;
     const int rg = (warp / HKV) % RG;
     const int kg = warp / (HKV * RG);
-    const int B = p.B, L = p.L;
+    // B counts list items (request, head group); b below is an item index.
+    const int B = GROUPS ? p.NB : p.B, L = p.L, ng = GROUPS ? p.ngrp : 1;
+    const size_t row_pitch = static_cast<size_t>(ROWB) * ng;  // cache bytes per row
 
     // ---- request key ranges and the tile list (reads inputs only) ----
     int total, per, t0, t1;
-    build_tile_list<TK>(p, tpre, rlo, rhi, rnew, DEC_THREADS, total, per, t0, t1);
+    build_tile_list<TK, GROUPS>(p, tpre, rlo, rhi, rnew, DEC_THREADS, total, per, t0, t1);
     if (t0 >= t1) return;
     // The normalised q and this step's new cache rows come from the prep kernel,
     // which may still be running (programmatic dependent launch): wait for it
@@ -305,7 +333,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
         if (tau >= t1) return;
         const int k0 = tile_k0(tau, b);
         int* dst = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
-        const int32_t* pt = p.page_table + static_cast<size_t>(b) * p.max_pages;
+        const int32_t* pt = p.page_table + static_cast<size_t>(item_req(b, ng)) * p.max_pages;
         if (PS == 1) {
             if (tid < TK) {
                 const int k = k0 + tid;
@@ -327,6 +355,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
         const int* ix = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
         const uint32_t base = smem_addr(kv_smem + ((tau - t0) % NS) * C::STAGE);
         const int lo = rlo[b], hi = rhi[b];
+        const size_t gofs = static_cast<size_t>(item_grp(b, ng)) * ROWB;
 #pragma unroll
         for (int i = 0; i < TK / 32; ++i) {
             const int r = (tid >> 3) + 32 * i;  // tile row
@@ -340,7 +369,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
                 crow = pg >= 0 ? static_cast<int64_t>(pg) * PS + r % PS : -1;
             }
             const bool ok = k >= lo && k <= hi && crow >= 0 && crow < p.num_rows;
-            const size_t off = ok ? static_cast<size_t>(crow) * ROWB + j * 16 : 0;
+            const size_t off = ok ? static_cast<size_t>(crow) * row_pitch + gofs + j * 16 : 0;
             const uint32_t d = base + r * ROWB + ((j ^ (r & 7)) << 4);
             cp_async16(d, p.k_cache + off, ok ? 16 : 0);
             cp_async16(d + TK * ROWB, p.v_cache + off, ok ? 16 : 0);
@@ -359,10 +388,11 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
 
     auto begin_request = [&](int b) {
         ensure_prep();
+        const int req = item_req(b, ng), grp = item_grp(b, ng);
         req_lo_max = 0;
         req_hi_min = INT_MAX;
         for (int j = 0; j < L; ++j) {
-            const int pos = static_cast<int>(p.positions[static_cast<size_t>(b) * L + j]);
+            const int pos = static_cast<int>(p.positions[static_cast<size_t>(req) * L + j]);
             const int l = p.window > 0 ? max(0, pos - p.window + 1) : 0;
             req_lo_max = max(req_lo_max, l);
             req_hi_min = min(req_hi_min, pos);
@@ -371,12 +401,12 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
         for (int nt = 0; nt < NT; ++nt) {
             const int j = rg * NT + nt;
             if (j < L) {
-                const size_t t = static_cast<size_t>(b) * L + j;
+                const size_t t = static_cast<size_t>(req) * L + j;
                 const int pos = static_cast<int>(p.positions[t]);
                 tok_hi[nt] = pos;
                 tok_lo[nt] = p.window > 0 ? max(0, pos - p.window + 1) : 0;
                 const uint4* q = reinterpret_cast<const uint4*>(
-                    p.q_ws + (t * HQ + g * GRP + gid) * HD + 16 * tig);
+                    p.q_ws + ((t * ng + grp) * HQ + g * GRP + gid) * HD + 16 * tig);
                 const uint4 a = q[0], c = q[1];
                 qf[nt][0] = a.x; qf[nt][1] = a.y; qf[nt][2] = a.z; qf[nt][3] = a.w;
                 qf[nt][4] = c.x; qf[nt][5] = c.y; qf[nt][6] = c.z; qf[nt][7] = c.w;
@@ -629,7 +659,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
 
 // ---------------------------------------------------------------------------
 // Kernel 3: merge the partials of each (token, head) and apply the gated
-// output norm.  One block per (token, head).  A request covered by many CTAs
+// output norm.  One block per (token, head), over all ngrp * 16 query heads.  A request covered by many CTAs
 // has many partials (a single 80K-key request spreads over ~1,200), so they
 // are read in parallel: thread (sl, dq) accumulates dims 4dq..4dq+3 over
 // partials sl, sl + lanes, ..., then the slot lanes are summed in shared memory.
@@ -644,13 +674,15 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams 
     __shared__ float red_l[COMB_SLOT_LANES];
     __shared__ float red_m[COMB_THREADS / 32];
     __shared__ float red_ss[4];
-    const int t = blockIdx.x / HQ, h = blockIdx.x % HQ;
+    const int ng = p.ngrp, hq_all = HQ * ng;
+    const int t = blockIdx.x / hq_all, hh = blockIdx.x % hq_all;  // hh = 16 * group + h
+    const int h = hh % HQ;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = t / p.L, j = t % p.L;
+    const int b = (t / p.L) * ng + hh / HQ, j = t % p.L;        // list item (request, group)
     const int tp = p.meta[META_PREFIX + b];
     const int n = p.meta[META_PREFIX + b + 1] - tp;
     const int per = p.meta[META_PER];
-    __nv_bfloat16* outp = p.out + static_cast<size_t>(t) * OUT_COLS + h * HD;
+    __nv_bfloat16* outp = p.out + static_cast<size_t>(t) * OUT_COLS * ng + hh * HD;
     if (n <= 0 || per <= 0) {  // no key in range (positions outside the contract)
         if (tid < HD) outp[tid] = __float2bfloat16(NAN);
         return;
@@ -711,7 +743,8 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams 
         asm volatile("bar.sync 1, 64;\n" ::: "memory");
         const float tot = red_ss[0] + red_ss[1];
         const float rinv = 1.0f / sqrtf(tot * (1.0f / 64.0f) + 1e-6f);
-        const float g = __bfloat162float(p.qkv[static_cast<size_t>(t) * QKV_COLS + G_OFF + h * HD + tid]);
+        const float g = __bfloat162float(
+            p.qkv[static_cast<size_t>(t) * QKV_COLS * ng + G_OFF * ng + hh * HD + tid]);
         outp[tid] = __float2bfloat16(a * rinv / (1.0f + expf(-g)));
     }
 }

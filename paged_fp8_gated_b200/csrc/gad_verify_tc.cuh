@@ -108,7 +108,8 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
 
 }  // namespace vtc
 
-template <int PS, int NS>
+// GROUPS: more than one head group (see decode_kernel).
+template <int PS, int NS, bool GROUPS>
 __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepParams p) {
     using namespace vtc;
     using C = Cfg<NS>;
@@ -122,15 +123,16 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + NBARS * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + NBARS * 8 + 4);
     int* tpre = reinterpret_cast<int*>(ctrl + C::CTRL_BYTES);
-    int* rlo = tpre + p.B + 1;
-    int* rhi = rlo + p.B;
-    int* rnew = rhi + p.B;
+    int* rlo = tpre + p.NB + 1;
+    int* rhi = rlo + p.NB;
+    int* rnew = rhi + p.NB;
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int B = p.B, L = p.L;
+    // B counts list items (request, head group); b below is an item index.
+    const int B = GROUPS ? p.NB : p.B, L = p.L, ng = GROUPS ? p.ngrp : 1;
 
     int total, per, t0, t1;
-    build_tile_list<TK>(p, tpre, rlo, rhi, rnew, THREADS, total, per, t0, t1);
+    build_tile_list<TK, GROUPS>(p, tpre, rlo, rhi, rnew, THREADS, total, per, t0, t1);
     if (t0 >= t1) return;
 
     const uint32_t bar0 = smem_addr(ctrl);
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // ---- tile cursors over the list (request b owns tiles [tpre[b], tpre[b+1])) ----
+    // ---- tile cursors over the list (item b owns tiles [tpre[b], tpre[b+1])) ----
     auto find_req = [&](int tau) {
         int lo = 0, hi = B;
         while (hi - lo > 1) {
@@ -189,7 +191,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
             if (tau >= t1) return;
             const int k0 = tile_k0(tau, b);
             int* dst = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
-            const int32_t* pt = p.page_table + static_cast<size_t>(b) * p.max_pages;
+            const int32_t* pt = p.page_table + static_cast<size_t>(item_req(b, ng)) * p.max_pages;
             if (PS == 1) {
                 if (ltid < TK) {
                     const int k = k0 + ltid;
@@ -211,6 +213,8 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
             const int* ix = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
             const uint32_t base = smem_addr(raw + ((tau - t0) % NS) * RAW_STAGE);
             const int lo = rlo[b], hi = rhi[b];
+            const size_t row_pitch = static_cast<size_t>(ROWB) * ng;
+            const size_t gofs = static_cast<size_t>(item_grp(b, ng)) * ROWB;
             constexpr int ROWS = TK * 8 / LOADERS;  // rows per thread
             const int j = ltid & 7;                 // 16-byte chunk
             // all page-table reads first, then the copies (the copies are ordered
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 if (PS == 1) crow = pix[i];
                 else crow = pix[i] >= 0 ? static_cast<int64_t>(pix[i]) * PS + r % PS : -1;
                 const bool ok = k >= lo && k <= hi && crow >= 0 && crow < p.num_rows;
-                off[i] = ok ? static_cast<size_t>(crow) * ROWB + j * 16 : 0;
+                off[i] = ok ? static_cast<size_t>(crow) * row_pitch + gofs + j * 16 : 0;
                 nbytes[i] = ok ? 16 : 0;
             }
 #pragma unroll
@@ -242,16 +246,17 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 cp_async16(d + TK * ROWB, p.v_cache + off[i], nbytes[i]);
             }
         };
-        // A operand of request b's S MMA: row ltid = [q | 0] (KV head 0) or [0 | q].
+        // A operand of item b's S MMA: row ltid = [q | 0] (KV head 0) or [0 | q].
         auto write_q = [&](int b) {
             ensure_prep();
             const int g = ltid >> 6, j = (ltid >> 3) & 7, hh = ltid & 7;
+            const size_t req = static_cast<size_t>(item_req(b, ng)), grp = static_cast<size_t>(item_grp(b, ng));
             uint32_t q[32], z[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) z[c] = 0u;
             if (j < L) {
                 const uint4* src = reinterpret_cast<const uint4*>(
-                    p.q_ws + ((static_cast<size_t>(b) * L + j) * HQ + g * GRP + hh) * HD);
+                    p.q_ws + (((req * L + j) * ng + grp) * HQ + g * GRP + hh) * HD);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const uint4 v = src[c];
@@ -426,7 +431,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 m_run = -INFINITY;
                 l_run = 0.f;
                 if (j < L) {
-                    const int pos = static_cast<int>(p.positions[static_cast<size_t>(cb) * L + j]);
+                    const int pos = static_cast<int>(p.positions[static_cast<size_t>(item_req(cb, ng)) * L + j]);
                     hi_j = pos;
                     lo_j = p.window > 0 ? max(0, pos - p.window + 1) : 0;
                 } else {

@@ -8,14 +8,15 @@ with torch's own normalisation and float8 cast, which are distribution
 recipes, not steps of the method.  Both the CUDA path and the oracle consume
 what it returns.
 
-Layouts (all torch CPU tensors):
-  qkv        bf16  [T, 2304]  q 16x64 | k 2x64 | v 2x64 | gate 16x64, T = B*L
+Layouts (all torch CPU tensors), for hq query and hkv KV heads (16 and 2 on
+the page's "heads tp8" shapes, 128 and 16 on its "heads dp" ones):
+  qkv        bf16  [T, 64 (2 hq + 2 hkv)]  q | k | v | gate, T = B*L
   positions  int64 [T]        seq_lens[b] + j for token t = b*L + j
   seq_lens   int32 [B]        tokens cached before this step
   page_table int32 [B, max_pages]
   cache_loc  int64 [T]        cache row (page*page_size + slot) of token t
-  k_cache    uint8 [num_pages, page_size, 2, 64]   E4M3 codes
-  v_cache    uint8 [num_pages, page_size, 2, 64]
+  k_cache    uint8 [num_pages, page_size, hkv, 64]   E4M3 codes
+  v_cache    uint8 [num_pages, page_size, hkv, 64]
 """
 from __future__ import annotations
 
@@ -24,10 +25,15 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-HQ, HKV, D = 16, 2, 64
+HQ, HKV, D = 16, 2, 64                    # "heads tp8": per GPU of eight
+DP_HQ, DP_HKV = 8 * HQ, 8 * HKV           # "heads dp": all heads on one GPU
 QKV_COLS = HQ * D + 2 * HKV * D + HQ * D  # 2304
 GATE_OFF = HQ * D + 2 * HKV * D           # 1280
 ROW_BYTES = HKV * D                       # 128
+
+
+def qkv_cols(hq: int, hkv: int) -> int:
+    return (2 * hq + 2 * hkv) * D
 
 
 @dataclass
@@ -49,6 +55,8 @@ class Spec:
     seed: int = 0
     spare_pages: int = 0       # unused pages in the pool
     dist: str = "normal"       # "normal", "coherent" or "edges" (see make_inputs)
+    hq: int = HQ               # query heads
+    hkv: int = HKV             # key/value heads
     extra: dict = field(default_factory=dict)
 
 
@@ -76,6 +84,7 @@ def make_inputs(spec: Spec) -> dict:
     """Draw one step's inputs.  Deterministic in ``spec`` (including its seed)."""
     gen = torch.Generator().manual_seed(int(spec.seed))
     B, L, ps = spec.B, spec.L, spec.page_size
+    hq, hkv = spec.hq, spec.hkv
     T = B * L
     seq = resolve_seq_lens(spec, gen)
     total = seq + L                                   # keys per request after the append
@@ -99,34 +108,34 @@ def make_inputs(spec: Spec) -> dict:
     b_of_t = np.repeat(np.arange(B), L)
     cache_loc = (page_table[b_of_t, positions // ps].astype(np.int64) * ps + positions % ps)
 
-    qkv = torch.randn(T, QKV_COLS, generator=gen)
+    qkv = torch.randn(T, qkv_cols(hq, hkv), generator=gen)
     if spec.gate_std != 1.0:
-        qkv[:, GATE_OFF:] *= spec.gate_std
+        qkv[:, (hq + 2 * hkv) * D:] *= spec.gate_std
     qkv = qkv.to(torch.bfloat16)
 
     # Pre-existing cache: K = E4M3(unit-RMS N(0,1) / scale), V = E4M3(N(0,1) / scale),
     # drawn for every slot of the pool (including the rows this step overwrites).
     rows = n_pages * ps
-    k_cache = torch.empty(rows, HKV, D, dtype=torch.uint8)
-    v_cache = torch.empty(rows, HKV, D, dtype=torch.uint8)
+    k_cache = torch.empty(rows, hkv, D, dtype=torch.uint8)
+    v_cache = torch.empty(rows, hkv, D, dtype=torch.uint8)
     chunk = 1 << 20
     inv = 1.0 / float(spec.kv_scale)
     for r0 in range(0, rows, chunk):
         r1 = min(rows, r0 + chunk)
-        kx = _unit_rms(torch.randn(r1 - r0, HKV, D, generator=gen))
-        vx = torch.randn(r1 - r0, HKV, D, generator=gen)
+        kx = _unit_rms(torch.randn(r1 - r0, hkv, D, generator=gen))
+        vx = torch.randn(r1 - r0, hkv, D, generator=gen)
         k_cache[r0:r1] = _to_e4m3_codes(kx * inv)
         v_cache[r0:r1] = _to_e4m3_codes(vx * inv)
 
     if spec.dist == "coherent":
         # Keys of each KV head share a direction (so attention spreads over many
         # keys) and values share one too: the page's "dist coherent" loads.
-        u = _unit_rms(torch.randn(1, HKV, D, generator=gen))
-        vdir = torch.randn(1, HKV, D, generator=gen)
+        u = _unit_rms(torch.randn(1, hkv, D, generator=gen))
+        vdir = torch.randn(1, hkv, D, generator=gen)
         for r0 in range(0, rows, chunk):
             r1 = min(rows, r0 + chunk)
-            kx = _unit_rms(u + 0.35 * torch.randn(r1 - r0, HKV, D, generator=gen))
-            vx = vdir + 0.5 * torch.randn(r1 - r0, HKV, D, generator=gen)
+            kx = _unit_rms(u + 0.35 * torch.randn(r1 - r0, hkv, D, generator=gen))
+            vx = vdir + 0.5 * torch.randn(r1 - r0, hkv, D, generator=gen)
             k_cache[r0:r1] = _to_e4m3_codes(kx * inv)
             v_cache[r0:r1] = _to_e4m3_codes(vx * inv)
     elif spec.dist == "edges":
@@ -136,7 +145,7 @@ def make_inputs(spec: Spec) -> dict:
         # Meant for layers without RoPE, where that raw direction is the one the
         # scores see; a window off by one key changes the output completely.
         assert spec.window > 0, "edges needs a sliding window"
-        qraw = qkv.float()[:, :HQ * D].view(T, HKV, HQ // HKV, D).mean(2)  # [T, 2, 64]
+        qraw = qkv.float()[:, :hq * D].view(T, hkv, hq // hkv, D).mean(2)  # [T, hkv, 64]
         for t in range(T):
             b = t // L
             for key in (int(positions[t]) - spec.window + 1, int(positions[t]) - spec.window):
@@ -149,15 +158,16 @@ def make_inputs(spec: Spec) -> dict:
 
     return dict(
         name=spec.name,
-        B=B, L=L, page_size=ps, window=int(spec.window), use_rope=bool(spec.use_rope),
+        B=B, L=L, hq=hq, hkv=hkv, page_size=ps, window=int(spec.window),
+        use_rope=bool(spec.use_rope),
         k_scale=float(spec.kv_scale), v_scale=float(spec.kv_scale),
         qkv=qkv,
         positions=torch.from_numpy(positions),
         seq_lens=torch.from_numpy(seq.astype(np.int32)),
         page_table=torch.from_numpy(page_table),
         cache_loc=torch.from_numpy(cache_loc),
-        k_cache=k_cache.view(n_pages, ps, HKV, D),
-        v_cache=v_cache.view(n_pages, ps, HKV, D),
+        k_cache=k_cache.view(n_pages, ps, hkv, D),
+        v_cache=v_cache.view(n_pages, ps, hkv, D),
     )
 
 
@@ -216,6 +226,15 @@ def named(name: str, seed: int = 0) -> Spec:
                            gate_std=2.0, seed=seed + 41),
         "paged_sliding": Spec("paged_sliding", B=4, L=8, ctx=65536, page_size=64, window=2048,
                               use_rope=True, kv_scale=1 / 64, gate_std=2.0, seed=seed + 42),
+        # the page's three "heads dp" gating shapes (128 query, 16 KV heads); their
+        # page size is not given, so they take the default pool of 64-token pages
+        # ("spread mixed": contexts uniform in [1, ctx])
+        "dp8_full_mixed": Spec("dp8_full_mixed", B=8, ctx_range=(1, 8192), page_size=64,
+                               hq=DP_HQ, hkv=DP_HKV, seed=seed + 61),
+        "dp2_full_v8_soft": Spec("dp2_full_v8_soft", B=2, L=8, ctx=20000, page_size=64,
+                                 hq=DP_HQ, hkv=DP_HKV, seed=seed + 62),
+        "dp2_full_v8_coherent": Spec("dp2_full_v8_coherent", B=2, L=8, ctx=20000, page_size=64,
+                                     dist="coherent", hq=DP_HQ, hkv=DP_HKV, seed=seed + 63),
     }
     return specs[name]
 

@@ -25,29 +25,35 @@ def to_device(inp: dict, dev="cuda") -> dict:
     return d
 
 
+def heads(inp: dict) -> tuple[int, int]:
+    return inp.get("hq", 16), inp.get("hkv", 2)
+
+
 def run_gpu(inp: dict, dev="cuda", workspace=None):
     """One step through the C ABI on fresh device copies; returns host arrays
-    (out bf16 bits [T, 1024], k_cache, v_cache uint8 [rows, 128])."""
+    (out bf16 bits [T, 64 hq], k_cache, v_cache uint8 [rows, 64 hkv])."""
     from paged_fp8_gated_b200 import binding
+    hq, hkv = heads(inp)
     d = to_device(inp, dev)
     out = binding.attn_decode(d["qkv"], d["positions"], d["seq_lens"], d["page_table"],
                               d["cache_loc"], d["k_cache"], d["v_cache"], d["k_scale_t"],
                               d["v_scale_t"], inp["page_size"], inp["window"], inp["use_rope"],
-                              L=inp["L"], workspace=workspace)
+                              L=inp["L"], workspace=workspace, hq=hq, hkv=hkv)
     torch.cuda.synchronize()
     T = inp["B"] * inp["L"]
-    out_bits = out.view(torch.int16).reshape(T, 1024).cpu().numpy().astype(np.uint16)
-    kc = d["k_cache"].reshape(-1, 128).cpu().numpy()
-    vc = d["v_cache"].reshape(-1, 128).cpu().numpy()
+    out_bits = out.view(torch.int16).reshape(T, 64 * hq).cpu().numpy().astype(np.uint16)
+    kc = d["k_cache"].reshape(-1, 64 * hkv).cpu().numpy()
+    vc = d["v_cache"].reshape(-1, 64 * hkv).cpu().numpy()
     return out_bits, kc, vc
 
 
 def run_oracle(inp: dict, want=None) -> O.OracleResult:
+    hq, hkv = heads(inp)
     qkv = inp["qkv"].view(torch.int16).numpy().astype(np.uint16)
     return O.attn_decode(qkv, inp["positions"], inp["page_table"], inp["cache_loc"],
-                         inp["k_cache"].reshape(-1, 128), inp["v_cache"].reshape(-1, 128),
+                         inp["k_cache"].reshape(-1, 64 * hkv), inp["v_cache"].reshape(-1, 64 * hkv),
                          inp["k_scale"], inp["v_scale"], inp["page_size"], inp["window"],
-                         inp["use_rope"], want=want)
+                         inp["use_rope"], want=want, hq=hq, hkv=hkv)
 
 
 def new_rows(inp: dict) -> np.ndarray:
@@ -58,11 +64,11 @@ def compare(gpu_out_bits: np.ndarray, ref: O.OracleResult, want=None) -> dict:
     """Element-wise check on the selected (token, head) outputs; returns stats."""
     got = O.bf16_bits_to_float(gpu_out_bits)
     exact = ref.out_exact
-    T = got.shape[0]
+    T, cols = got.shape
     if want is None:
-        mask = np.ones((T, 1024), bool)
+        mask = np.ones((T, cols), bool)
     else:
-        mask = np.repeat(np.asarray(want, bool).reshape(T, 16), 64, axis=1)
+        mask = np.repeat(np.asarray(want, bool).reshape(T, cols // 64), 64, axis=1)
     g, e = got[mask], exact[mask]
     err = np.abs(g - e)
     bound = ATOL + RTOL * np.abs(e)
@@ -72,12 +78,12 @@ def compare(gpu_out_bits: np.ndarray, ref: O.OracleResult, want=None) -> dict:
                 ok=bool(np.isfinite(g).all() and (err <= bound).all()))
 
 
-def sample_want(T: int, n: int, seed: int = 0) -> np.ndarray:
+def sample_want(T: int, n: int, seed: int = 0, hq: int = 16) -> np.ndarray:
     """n (token, head) pairs, always including the first and last token."""
     rng = np.random.default_rng(seed)
-    want = np.zeros((T, 16), bool)
-    want[0, rng.integers(16)] = True
-    want[T - 1, rng.integers(16)] = True
+    want = np.zeros((T, hq), bool)
+    want[0, rng.integers(hq)] = True
+    want[T - 1, rng.integers(hq)] = True
     for _ in range(max(0, n - 2)):
-        want[rng.integers(T), rng.integers(16)] = True
+        want[rng.integers(T), rng.integers(hq)] = True
     return want

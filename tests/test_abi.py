@@ -82,6 +82,27 @@ def test_argument_checks_fail_before_launch(lib, over, status):
     assert lib.last_error()
 
 
+@pytest.mark.parametrize("over,status", [
+    (dict(hq=16, hkv=4), -4),             # 4 query heads per KV head
+    (dict(hq=24, hkv=3), -4),             # odd KV-head count
+    (dict(hq=0, hkv=0), -4),
+    (dict(hq=8, hkv=1), -4),
+    (dict(hq=128, hkv=16, B=513), -2),    # 513 requests x 8 head groups > 4096 list items
+    (dict(hq=128, hkv=16, qkv=FAKE + 8), -3),   # valid heads reach the later checks
+    (dict(hq=128, hkv=16, qkv=None), -1),
+])
+def test_heads_argument_checks(lib, over, status):
+    assert lib.raw_call(**_ok_args(**over)) == status
+    assert lib.last_error()
+
+
+def test_heads_workspace_query_rejects_bad_heads(lib):
+    so = lib.lib()
+    assert so.gad_attn_workspace_bytes_heads(4, 1, 16, 4) == 0
+    assert "hq=16" in lib.last_error()
+    assert so.gad_attn_workspace_bytes_heads(600, 8, 128, 16) == 0
+
+
 def test_binding_rejects_cpu_tensors(lib):
     import torch
     x = torch.zeros(1, 2304, dtype=torch.bfloat16)

@@ -57,6 +57,23 @@ SMALL = [
 ]
 
 
+# "heads dp" (128 query heads over 16 KV heads on one GPU): the page's three
+# gating shapes, then edge cases of the head-group split.
+DP = dict(hq=W.DP_HQ, hkv=W.DP_HKV)
+SMALL_DP = [
+    W.named("dp8_full_mixed"),
+    W.named("dp2_full_v8_soft"),
+    W.named("dp2_full_v8_coherent"),
+    S("dp_sliding_p1", B=3, ctx_range=(0, 4000), window=2048, use_rope=True, seed=140, **DP),
+    S("dp_sliding_v8_s64", B=2, L=8, seq_lens=[37, 3000], window=2048, use_rope=True,
+      page_size=64, kv_scale=1 / 64, gate_std=2.0, seed=141, **DP),
+    S("dp_ctx0_and_ragged_v3", B=3, L=3, seq_lens=[0, 63, 130], page_size=64, seed=142, **DP),
+    S("dp_edges_sliding", B=2, L=8, ctx=3000, window=2048, dist="edges", seed=143, **DP),
+    # 512 requests x 8 groups = 4096 list items, the most one call takes
+    S("dp_b512_most_items", B=512, ctx_range=(0, 40), seed=144, **DP),
+]
+
+
 def _check(inp, want=None, label=""):
     gpu_out, gpu_k, gpu_v = H.run_gpu(inp)
     ref = H.run_oracle(inp, want=want)
@@ -70,6 +87,42 @@ def _check(inp, want=None, label=""):
 @pytest.mark.parametrize("spec", SMALL, ids=lambda s: s.name)
 def test_small_full_compare(spec, cuda_dev):
     _check(W.make_inputs(spec), label=spec.name)
+
+
+@pytest.mark.parametrize("spec", SMALL_DP, ids=lambda s: s.name)
+def test_heads_dp_compare(spec, cuda_dev):
+    _check(W.make_inputs(spec), label=spec.name)
+
+
+def test_heads_dp_equals_eight_tp8_steps(cuda_dev):
+    """The library's 128/16-head step against eight of its own 16/2-head steps
+    on the column slices.  Cache bytes must match bit for bit; outputs to about
+    one bf16 rounding step (4e-3 absolute, for elements near zero after the
+    output norm), since the tile list (and with it where the key ranges are
+    split between CTAs, i.e. the fp32 summation order) differs."""
+    inp = W.make_inputs(S("dp_vs_tp8", B=3, L=8, seq_lens=[5, 700, 2100], window=2048,
+                          use_rope=True, seed=145, **DP))
+    out_dp, k_dp, v_dp = H.run_gpu(inp)
+    hq, hkv = W.DP_HQ, W.DP_HKV
+    qkv = inp["qkv"]
+    ks, vs, gs = 64 * hq, 64 * (hq + hkv), 64 * (hq + 2 * hkv)
+    kc = inp["k_cache"].reshape(-1, hkv, 64)
+    vc = inp["v_cache"].reshape(-1, hkv, 64)
+    for c in range(hkv // 2):
+        sub = dict(inp)
+        sub["hq"], sub["hkv"] = 16, 2
+        sub["qkv"] = torch.cat([qkv[:, 1024 * c:1024 * (c + 1)], qkv[:, ks + 128 * c:ks + 128 * (c + 1)],
+                                qkv[:, vs + 128 * c:vs + 128 * (c + 1)],
+                                qkv[:, gs + 1024 * c:gs + 1024 * (c + 1)]], dim=1).contiguous()
+        sub["k_cache"] = kc[:, 2 * c:2 * c + 2].contiguous()
+        sub["v_cache"] = vc[:, 2 * c:2 * c + 2].contiguous()
+        out_tp, k_tp, v_tp = H.run_gpu(sub)
+        a = H.O.bf16_bits_to_float(out_dp[:, 1024 * c:1024 * (c + 1)])
+        b = H.O.bf16_bits_to_float(out_tp)
+        err = np.abs(a - b)
+        assert (err <= 4e-3 + 2.0 ** -7 * np.abs(b)).all(), (c, float(err.max()))
+        assert np.array_equal(k_dp[:, 128 * c:128 * (c + 1)], k_tp), c
+        assert np.array_equal(v_dp[:, 128 * c:128 * (c + 1)], v_tp), c
 
 
 def test_verify_full_ctx100k(cuda_dev):
