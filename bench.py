@@ -42,6 +42,7 @@ METRIC = "µs/step and KV-cache GB/s (% of HBM roofline), decode-32 full-attn ct
 BYTES_PER_KEY = 256          # K and V rows: 2 KV heads x 64 E4M3 codes each
 PT_BYTES_PER_KEY = {1: 4, 64: 4 / 64}   # page-table bytes read per key
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_TC_TFLOPS = 1590.0  # dense bf16/fp16 burst
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the step's main
 # kernel on a workload, from the ncu captures summarised in profiles/, keyed by
@@ -76,8 +77,9 @@ def measured_peaks() -> dict:
     if os.path.exists(p):
         with open(p) as fh:
             d = json.load(fh)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
-    return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+        return {"hbm_gbs": float(d["hbm_gbs"]),
+                "tc_tflops": float(d.get("bf16_tflops", FALLBACK_TC_TFLOPS)), "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "tc_tflops": FALLBACK_TC_TFLOPS, "source": "fallback"}
 
 
 class ClockSampler:
@@ -130,33 +132,57 @@ class ClockSampler:
 
 
 def oracle_cpu_rate(inp: dict, max_key_heads: float = 40e6) -> dict:
-    """Time the CPU oracle on a bounded prefix of the step's requests (all heads
-    and tokens of each); returns KV-cache GB/s over that sample."""
+    """Time the CPU oracle on a bounded sample of the step and return the rate
+    it implies in the bench line's unit (KV-cache GB/s of the whole step).
+    Decode and verify steps: a prefix of the requests (all heads and tokens of
+    each).  Prefill blocks: the first tokens of request 0 (all heads), scaled
+    to the whole step by the (token, key) pairs attended."""
     import numpy as np
     import torch
     from oracle import oracle as O
-    from paged_fp8_gated_b200 import workloads as W
 
     B, L = inp["B"], inp["L"]
+    hq, hkv = inp.get("hq", 16), inp.get("hkv", 2)
     pos = inp["positions"].numpy().reshape(B, L)
     W_ = inp["window"]
+    lo_t = np.maximum(0, pos - W_ + 1) if W_ > 0 else np.zeros_like(pos)
+    tok_keys = (pos - lo_t + 1).astype(np.int64)          # keys per token
     keys = []
     for b in range(B):
-        lo = max(0, int(pos[b, 0]) - W_ + 1) if W_ > 0 else 0
-        keys.append(int(pos[b, -1]) - lo + 1)
+        keys.append(int(pos[b, -1]) - int(lo_t[b, 0]) + 1)
+    threads = os.cpu_count() or 1
+    cache = dict(k_cache=inp["k_cache"].reshape(-1, 64 * hkv),
+                 v_cache=inp["v_cache"].reshape(-1, 64 * hkv))
+    if L > 8:
+        n = 1
+        while n < L and tok_keys[0, :n + 1].sum() * hq <= max_key_heads:
+            n += 1
+        want = np.zeros((L, hq), bool)
+        want[:n] = True
+        qkv = inp["qkv"][:L].view(torch.int16).numpy().astype(np.uint16)
+        t = time.perf_counter()
+        O.attn_decode(qkv, inp["positions"][:L], inp["page_table"][:1], inp["cache_loc"][:L],
+                      cache["k_cache"], cache["v_cache"], inp["k_scale"], inp["v_scale"],
+                      inp["page_size"], inp["window"], inp["use_rope"], want=want,
+                      nthreads=threads, hq=hq, hkv=hkv)
+        dt = time.perf_counter() - t
+        full_dt = dt * float(tok_keys.sum()) / float(tok_keys[0, :n].sum())
+        kv = sum(keys) * 2 * 64 * hkv
+        return {"value": kv / full_dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                "seconds": dt,
+                "sample": f"tokens 0..{n - 1} of request 0 (all {hq} heads; {int(tok_keys[0, :n].sum())} "
+                          f"token-keys of {int(tok_keys.sum())}), scaled by token-keys; FP64 C oracle"}
     nb, kh = 0, 0.0
-    hq, hkv = inp.get("hq", 16), inp.get("hkv", 2)
     while nb < B and (nb == 0 or kh + keys[nb] * hq * L <= max_key_heads):
         kh += keys[nb] * hq * L
         nb += 1
     T = nb * L
     qkv = inp["qkv"][:T].view(torch.int16).numpy().astype(np.uint16)
-    threads = os.cpu_count() or 1
     t = time.perf_counter()
     O.attn_decode(qkv, inp["positions"][:T], inp["page_table"][:nb], inp["cache_loc"][:T],
-                  inp["k_cache"].reshape(-1, 64 * hkv), inp["v_cache"].reshape(-1, 64 * hkv),
-                  inp["k_scale"], inp["v_scale"], inp["page_size"], inp["window"],
-                  inp["use_rope"], nthreads=threads, hq=hq, hkv=hkv)
+                  cache["k_cache"], cache["v_cache"], inp["k_scale"], inp["v_scale"],
+                  inp["page_size"], inp["window"], inp["use_rope"], nthreads=threads, hq=hq,
+                  hkv=hkv)
     dt = time.perf_counter() - t
     kv = sum(keys[:nb]) * 2 * 64 * hkv
     return {"value": kv / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
@@ -453,10 +479,25 @@ def main():
         return
 
     peaks = measured_peaks()
-    achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
     kname = main_kernel(L)
     ksrc = kernel_source_hash(kname)
     traffic = TRAFFIC.get((args.workload, ksrc))
+    # algorithmic flops: q.K^T and P.V, 2 x 64 multiply-adds per (token, head, key)
+    flops = 256 * hq * token_keys(inp)
+    if L > 8:   # prefill blocks: compute-bound (dense fp16 MMA, fp32 accumulate)
+        roof = {"kernel": kname, "bound": "tensor",
+                "achieved": round(flops / (dec_ms * 1e-3) / 1e12, 1),
+                "peak": peaks["tc_tflops"], "peak_source": peaks["source"] + " bf16 burst",
+                "unit": "TFLOP/s", "frac": round(flops / (dec_ms * 1e-3) / 1e12 / peaks["tc_tflops"], 4),
+                "traffic": traffic, "algorithmic_flops_per_launch": int(flops)}
+    else:
+        achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
+        roof = {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "algorithmic_bytes_per_launch": int(alg_bytes)}
+    roof.update({"kernel_us": round(dec_ms * 1e3, 2), "prep_us": round(prep_ms * 1e3, 2),
+                 "combine_us": round(comb_ms * 1e3, 2)})
     line = {
         "metric": METRIC,
         "value": round(replicas.job_rate(kv_bytes, world, mean_ms * 1e-3) / 1e9, 2),
@@ -483,15 +524,8 @@ def main():
             "e2e_inputs": "qkv, positions, seq_lens, cache_loc copied H2D each step; cache and "
                           "page table device-resident",
         },
-        "roofline": {
-            "kernel": kname, "bound": "hbm", "achieved": round(achieved, 1),
-            "peak": peaks["hbm_gbs"], "peak_source": peaks["source"], "unit": "GB/s",
-            "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": traffic,
-            "algorithmic_bytes_per_launch": int(alg_bytes),
-            "kernel_us": round(dec_ms * 1e3, 2),
-            "prep_us": round(prep_ms * 1e3, 2), "combine_us": round(comb_ms * 1e3, 2),
-        },
+        "roofline": roof,
+        "tflops_step": round(flops / (mean_ms * 1e-3) / 1e12, 1),
         "e2e": {"value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "us_per_step": round(e2e_ms * 1e3, 2),
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},

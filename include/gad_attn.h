@@ -48,7 +48,9 @@ extern "C" {
 #define GAD_OUT_COLS 1024  /* 16 heads x 64                  */
 #define GAD_ROW_BYTES 128  /* one cache row: 2 KV heads x 64 E4M3 codes */
 #define GAD_MAX_L 8        /* longest verify block           */
-#define GAD_MAX_B 4096     /* most requests in one call      */
+#define GAD_MAX_B 4096     /* most requests in one call; also the most
+                              (request, 8-token chunk, head group) items  */
+#define GAD_MAX_PREFILL_L 65536 /* longest block of gad_attn_prefill */
 #define GAD_NOALLOC_SCRATCH_BYTES (16u << 20) /* built-in scratch of gad_attn_decode_noalloc */
 
 /* Return codes (0 = success). */
@@ -181,6 +183,37 @@ int gad_attn_decode_heads_timed(const void* qkv, const int64_t* positions,
                                 int hkv, int max_pages, int64_t num_rows, int page_size,
                                 int window, int use_rope, void* out, void* workspace,
                                 size_t workspace_bytes, void* stream, void* const* events);
+
+/*
+ * Prefill: the same step for a block of L new tokens per request, causal
+ * within the block, 1 <= L <= GAD_MAX_PREFILL_L.  The page "Prefill layer
+ * (muse_prefill_layer)" runs this attention (its "What to compute": QK-norm,
+ * RoPE, write fp8(k), fp8(v), rmsnorm(attention(q)) * sigmoid(g)) at q_len
+ * 753 on an 80,000-token context and at q_len 16,384.  Arguments, layouts
+ * and error behaviour are those of gad_attn_decode with L tokens per request
+ * (token t = b * L + j at position positions[t], contract positions[t] =
+ * seq_lens[b] + j); the workspace comes from gad_attn_prefill_workspace_bytes.
+ * Each request's tokens are split into chunks of 8 and B * ceil(L / 8) may
+ * not exceed GAD_MAX_B (GAD_ERR_SHAPE), e.g. L = 16,384 admits B <= 2.
+ */
+int gad_attn_prefill(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                     const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,
+                     uint8_t* v_cache, const float* k_scale, const float* v_scale, int B, int L,
+                     int max_pages, int64_t num_rows, int page_size, int window, int use_rope,
+                     void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of gad_attn_prefill on the CURRENT device (0 on bad
+ * arguments, with gad_last_error() set).  Host-only. */
+size_t gad_attn_prefill_workspace_bytes(int B, int L);
+
+/* Profiling variant of gad_attn_prefill, with the four events of
+ * gad_attn_decode_timed. */
+int gad_attn_prefill_timed(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                           const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,
+                           uint8_t* v_cache, const float* k_scale, const float* v_scale, int B,
+                           int L, int max_pages, int64_t num_rows, int page_size, int window,
+                           int use_rope, void* out, void* workspace, size_t workspace_bytes,
+                           void* stream, void* const* events);
 
 /*
  * Allocation-free variant of gad_attn_decode.  The page has no counterpart:

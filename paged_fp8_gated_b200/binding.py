@@ -40,6 +40,12 @@ _lib.gad_attn_decode_heads.argtypes = (list(_lib.gad_attn_decode.argtypes[:11])
                                        + list(_lib.gad_attn_decode.argtypes[11:]))
 _lib.gad_attn_decode_heads_timed.restype = ctypes.c_int
 _lib.gad_attn_decode_heads_timed.argtypes = list(_lib.gad_attn_decode_heads.argtypes) + [_vp]
+_lib.gad_attn_prefill.restype = ctypes.c_int
+_lib.gad_attn_prefill.argtypes = list(_lib.gad_attn_decode.argtypes)
+_lib.gad_attn_prefill_workspace_bytes.restype = ctypes.c_size_t
+_lib.gad_attn_prefill_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
+_lib.gad_attn_prefill_timed.restype = ctypes.c_int
+_lib.gad_attn_prefill_timed.argtypes = list(_lib.gad_attn_decode.argtypes) + [_vp]
 _lib.gad_attn_decode_timed.restype = ctypes.c_int
 _lib.gad_attn_decode_timed.argtypes = list(_lib.gad_attn_decode.argtypes) + [_vp]
 _lib.gad_attn_decode_noalloc.restype = ctypes.c_int
@@ -51,9 +57,11 @@ _lib.gad_status_string.argtypes = [ctypes.c_int]
 
 HQ, HKV, D = 16, 2, 64
 QKV_COLS, OUT_COLS, ROW_BYTES = 2304, 1024, 128
+MAX_L, MAX_PREFILL_L = 8, 65536
 
 EXPORTED = ("gad_attn_decode", "gad_attn_decode_heads", "gad_attn_decode_timed",
-            "gad_attn_decode_heads_timed",
+            "gad_attn_decode_heads_timed", "gad_attn_prefill", "gad_attn_prefill_timed",
+            "gad_attn_prefill_workspace_bytes",
             "gad_attn_decode_noalloc", "gad_attn_workspace_bytes",
             "gad_attn_workspace_bytes_heads", "gad_last_error", "gad_status_string")
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -72,7 +80,11 @@ def lib() -> ctypes.CDLL:
 
 
 def workspace_bytes(B: int, L: int, hq: int = HQ, hkv: int = HKV) -> int:
-    if (hq, hkv) == (HQ, HKV):
+    """Workspace of one step; blocks longer than MAX_L tokens go to the prefill
+    entry point (16 and 2 heads)."""
+    if L > MAX_L and (hq, hkv) == (HQ, HKV):
+        n = _lib.gad_attn_prefill_workspace_bytes(int(B), int(L))
+    elif (hq, hkv) == (HQ, HKV):
         n = _lib.gad_attn_workspace_bytes(int(B), int(L))
     else:
         n = _lib.gad_attn_workspace_bytes_heads(int(B), int(L), int(hq), int(hkv))
@@ -111,7 +123,9 @@ def attn_decode(qkv: torch.Tensor, positions: torch.Tensor, seq_lens: torch.Tens
                 out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                 stream: torch.cuda.Stream | None = None,
                 events: list | None = None, hq: int = HQ, hkv: int = HKV) -> torch.Tensor:
-    """One decode step (L = 1) or verify block (L <= 8); returns out bf16 [B, L, 64 hq].
+    """One decode step (L = 1), verify block (L <= 8) or prefill block (L up to
+    MAX_PREFILL_L, through gad_attn_prefill, 16 and 2 heads); returns out bf16
+    [B, L, 64 hq].
 
     Shapes: qkv bf16 [B*L, 64 (2 hq + 2 hkv)]; positions, cache_loc int64 [B*L];
     seq_lens int32 [B] (optional); page_table int32 [B, max_pages]; k_cache / v_cache
@@ -157,9 +171,15 @@ def attn_decode(qkv: torch.Tensor, positions: torch.Tensor, seq_lens: torch.Tens
             _ptr(out), _ptr(workspace), int(workspace.numel()), ctypes.c_void_p(s))
     args = head + tail
     tp8 = (hq, hkv) == (HQ, HKV)
+    prefill = L > MAX_L
+    if prefill and not tp8:
+        raise ValueError(f"blocks longer than {MAX_L} tokens take 16 query and 2 KV heads")
     if events is None:
-        st = _lib.gad_attn_decode(*args) if tp8 else \
-            _lib.gad_attn_decode_heads(*head, int(hq), int(hkv), *tail)
+        if prefill:
+            st = _lib.gad_attn_prefill(*args)
+        else:
+            st = _lib.gad_attn_decode(*args) if tp8 else \
+                _lib.gad_attn_decode_heads(*head, int(hq), int(hkv), *tail)
     else:
         if len(events) != 4:
             raise ValueError("events must hold four torch.cuda.Event")
@@ -167,10 +187,13 @@ def attn_decode(qkv: torch.Tensor, positions: torch.Tensor, seq_lens: torch.Tens
             if ev.cuda_event == 0:
                 ev.record()
         arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(ev.cuda_event) for ev in events])
-        st = _lib.gad_attn_decode_timed(*args, arr) if tp8 else \
-            _lib.gad_attn_decode_heads_timed(*head, int(hq), int(hkv), *tail, arr)
+        if prefill:
+            st = _lib.gad_attn_prefill_timed(*args, arr)
+        else:
+            st = _lib.gad_attn_decode_timed(*args, arr) if tp8 else \
+                _lib.gad_attn_decode_heads_timed(*head, int(hq), int(hkv), *tail, arr)
     if st != 0:
-        raise GadError(st, "gad_attn_decode")
+        raise GadError(st, "gad_attn_prefill" if prefill else "gad_attn_decode")
     return out
 
 
@@ -215,6 +238,8 @@ def raw_call(**kw) -> int:
     rest = [kw.get("max_pages", 1), kw.get("num_rows", 1), kw.get("page_size", 1),
             kw.get("window", 0), kw.get("use_rope", 0), kw.get("out"), kw.get("workspace"),
             kw.get("workspace_bytes", 0), kw.get("stream")]
+    if kw.get("prefill"):           # through gad_attn_prefill
+        return _lib.gad_attn_prefill(*args, *rest)
     if "hq" in kw or "hkv" in kw:   # through gad_attn_decode_heads
         return _lib.gad_attn_decode_heads(*args, kw.get("hq", HQ), kw.get("hkv", HKV), *rest)
     return _lib.gad_attn_decode(*args, *rest)

@@ -51,13 +51,15 @@ struct WsLayout {
     int lt;
 };
 
+int chunks_of(int L) { return (L + gad::CHUNK - 1) / gad::CHUNK; }
+
 // Partial slots: (CTAs + NB) * partials per (CTA, list item), each holding lt
-// tokens x 16 heads x (64 values + max + sum); NB = B * ngrp list items
-// (request, group of 16 query and 2 KV heads).
+// tokens x 16 heads x (64 values + max + sum); NB = B * chunks * ngrp list
+// items (request, chunk of up to 8 tokens, group of 16 query and 2 KV heads).
 WsLayout ws_layout(int B, int L, int ngrp, int sms) {
     WsLayout w{};
-    w.lt = L == 1 ? 1 : GAD_MAX_L;
-    const size_t NB = static_cast<size_t>(B) * ngrp;
+    w.lt = L == 1 ? 1 : gad::CHUNK;
+    const size_t NB = static_cast<size_t>(B) * chunks_of(L) * ngrp;
     const size_t units =
         (static_cast<size_t>(sms) * kMaxCtasPerSm + NB) * (L == 1 ? kV1SingleKG : 1);
     const size_t T = static_cast<size_t>(B) * L;
@@ -96,11 +98,11 @@ cudaLaunchAttribute pdl_attr() {
     return a;
 }
 
-template <int LT, int PS, int KG, int NS, int MINB, int TK, bool MERGE, bool GROUPS>
+template <int LT, int PS, int KG, int NS, int MINB, int TK, bool MERGE, bool MULTI>
 int launch_decode(const gad::StepParams& prm, int sms, int tiles_upper, cudaStream_t stream,
                   bool pdl) {
     using C = gad::DecodeCfg<LT, KG, NS, TK, MERGE>;
-    auto kern = gad::decode_kernel<LT, PS, KG, NS, MINB, TK, MERGE, GROUPS>;
+    auto kern = gad::decode_kernel<LT, PS, KG, NS, MINB, TK, MERGE, MULTI>;
     const size_t smem = C::smem_bytes(prm.NB);
     // Raise the kernel's dynamic shared-memory limit once per device, to the
     // largest size any item count needs, so no attribute call happens during capture.
@@ -141,11 +143,11 @@ int launch_decode(const gad::StepParams& prm, int sms, int tiles_upper, cudaStre
 
 // Verify blocks (L > 1) on the tcgen05 kernel: one CTA per SM; as many raw
 // stages as the shared memory leaves room for next to the per-request tables.
-template <int PS, int NS, bool GROUPS>
+template <int PS, int NS, bool MULTI>
 int launch_verify_tc(const gad::StepParams& prm, int sms, int tiles_upper, cudaStream_t stream,
                      bool pdl) {
     using C = gad::vtc::Cfg<NS>;
-    auto kern = gad::verify_tc_kernel<PS, NS, GROUPS>;
+    auto kern = gad::verify_tc_kernel<PS, NS, MULTI>;
     const size_t smem = C::smem_bytes(prm.NB);
     static std::atomic<bool> attr_done[kMaxDevices];
     int dev = 0;
@@ -186,39 +188,52 @@ bool verify_deep_fits(int NB, int optin) {
     return gad::vtc::Cfg<kVtcDeepStages>::smem_bytes(NB) <= static_cast<size_t>(optin);
 }
 
-// Head counts the kernels take: groups of 16 query heads over 2 KV heads.
-// Sets *ngrp to the group count, or returns an error status.
-int head_groups(int hq, int hkv, int B, int* ngrp) {
+// Shape checks shared by the entry points: B, L (at most max_L), the head
+// counts the kernels take (groups of 16 query heads over 2 KV heads) and the
+// number of tile-list items.  Sets *ngrp, or returns an error status.
+int check_shape(int B, int L, int max_L, int hq, int hkv, int* ngrp) {
+    if (B < 1 || B > GAD_MAX_B) return fail(GAD_ERR_SHAPE, "B=%d not in [1,%d]", B, GAD_MAX_B);
+    if (L < 1 || L > max_L) return fail(GAD_ERR_SHAPE, "L=%d not in [1,%d]", L, max_L);
     if (hkv < GAD_HKV || hkv % GAD_HKV != 0 || hq != hkv * (GAD_HQ / GAD_HKV))
         return fail(GAD_ERR_UNSUPPORTED,
                     "hq=%d, hkv=%d: supported head counts are hkv a positive multiple of %d and "
                     "hq = %d hkv", hq, hkv, GAD_HKV, GAD_HQ / GAD_HKV);
     *ngrp = hkv / GAD_HKV;
-    if (static_cast<long long>(B) * *ngrp > GAD_MAX_B)
-        return fail(GAD_ERR_SHAPE, "B=%d requests x %d head groups exceeds %d", B, *ngrp,
-                    GAD_MAX_B);
+    const long long items = static_cast<long long>(B) * chunks_of(L) * *ngrp;
+    if (items > GAD_MAX_B)
+        return fail(GAD_ERR_SHAPE,
+                    "B=%d requests x %d chunks of 8 tokens x %d head groups = %lld items exceeds %d",
+                    B, chunks_of(L), *ngrp, items, GAD_MAX_B);
     return GAD_OK;
 }
 
+size_t workspace_bytes(int B, int L, int max_L, int hq, int hkv) {
+    int ngrp = 0;
+    if (check_shape(B, L, max_L, hq, hkv, &ngrp) != GAD_OK) return 0;
+    int sms = 0, major = 0;
+    if (current_device_sms(&sms, &major) != GAD_OK) return 0;
+    return ws_layout(B, L, ngrp, sms).total;
+}
+
 // Single-token steps and verify blocks, by page size (and stage count).
-template <bool GROUPS>
+template <bool MULTI>
 int launch_single(const gad::StepParams& prm, int page_size, int sms, int tiles_upper,
                   cudaStream_t s, bool pdl) {
     return page_size == 1
-               ? launch_decode<1, 1, kV1SingleKG, kV1SingleNS, 2, kV1SingleTK, false, GROUPS>(
+               ? launch_decode<1, 1, kV1SingleKG, kV1SingleNS, 2, kV1SingleTK, false, MULTI>(
                      prm, sms, tiles_upper, s, pdl)
-               : launch_decode<1, 64, kV1SingleKG, kV1SingleNS, 2, kV1SingleTK, false, GROUPS>(
+               : launch_decode<1, 64, kV1SingleKG, kV1SingleNS, 2, kV1SingleTK, false, MULTI>(
                      prm, sms, tiles_upper, s, pdl);
 }
 
-template <bool GROUPS>
+template <bool MULTI>
 int launch_block(const gad::StepParams& prm, int page_size, bool deep, int sms, int tiles_upper,
                  cudaStream_t s, bool pdl) {
     if (page_size == 1)
-        return deep ? launch_verify_tc<1, kVtcDeepStages, GROUPS>(prm, sms, tiles_upper, s, pdl)
-                    : launch_verify_tc<1, kVtcShallowStages, GROUPS>(prm, sms, tiles_upper, s, pdl);
-    return deep ? launch_verify_tc<64, kVtcDeepStages, GROUPS>(prm, sms, tiles_upper, s, pdl)
-                : launch_verify_tc<64, kVtcShallowStages, GROUPS>(prm, sms, tiles_upper, s, pdl);
+        return deep ? launch_verify_tc<1, kVtcDeepStages, MULTI>(prm, sms, tiles_upper, s, pdl)
+                    : launch_verify_tc<1, kVtcShallowStages, MULTI>(prm, sms, tiles_upper, s, pdl);
+    return deep ? launch_verify_tc<64, kVtcDeepStages, MULTI>(prm, sms, tiles_upper, s, pdl)
+                : launch_verify_tc<64, kVtcShallowStages, MULTI>(prm, sms, tiles_upper, s, pdl);
 }
 
 }  // namespace
@@ -242,15 +257,11 @@ const char* gad_status_string(int status) {
 }
 
 size_t gad_attn_workspace_bytes_heads(int B, int L, int hq, int hkv) {
-    if (B < 1 || B > GAD_MAX_B || L < 1 || L > GAD_MAX_L) {
-        fail(GAD_ERR_SHAPE, "B=%d must be in [1,%d] and L=%d in [1,%d]", B, GAD_MAX_B, L, GAD_MAX_L);
-        return 0;
-    }
-    int ngrp = 0;
-    if (head_groups(hq, hkv, B, &ngrp) != GAD_OK) return 0;
-    int sms = 0, major = 0;
-    if (current_device_sms(&sms, &major) != GAD_OK) return 0;
-    return ws_layout(B, L, ngrp, sms).total;
+    return workspace_bytes(B, L, GAD_MAX_L, hq, hkv);
+}
+
+size_t gad_attn_prefill_workspace_bytes(int B, int L) {
+    return workspace_bytes(B, L, GAD_MAX_PREFILL_L, GAD_HQ, GAD_HKV);
 }
 
 size_t gad_attn_workspace_bytes(int B, int L) {
@@ -259,21 +270,20 @@ size_t gad_attn_workspace_bytes(int B, int L) {
 
 static int run_step(const void* qkv, const int64_t* positions, const int32_t* page_table,
                     const int64_t* cache_loc, uint8_t* k_cache, uint8_t* v_cache,
-                    const float* k_scale, const float* v_scale, int B, int L, int hq, int hkv,
-                    int max_pages, int64_t num_rows, int page_size, int window, int use_rope,
-                    void* out, void* workspace, size_t workspace_bytes, void* stream,
-                    void* const* events) {
+                    const float* k_scale, const float* v_scale, int B, int L, int max_L, int hq,
+                    int hkv, int max_pages, int64_t num_rows, int page_size, int window,
+                    int use_rope, void* out, void* workspace, size_t workspace_bytes,
+                    void* stream, void* const* events) {
     if (!qkv || !positions || !page_table || !cache_loc || !k_cache || !v_cache || !k_scale ||
         !v_scale || !out)
         return fail(GAD_ERR_NULL, "a required pointer is NULL");
     if (!workspace) return fail(GAD_ERR_WORKSPACE, "workspace is NULL");
-    if (B < 1 || B > GAD_MAX_B) return fail(GAD_ERR_SHAPE, "B=%d not in [1,%d]", B, GAD_MAX_B);
-    if (L < 1 || L > GAD_MAX_L) return fail(GAD_ERR_SHAPE, "L=%d not in [1,%d]", L, GAD_MAX_L);
     int ngrp = 0;
     {
-        const int hs = head_groups(hq, hkv, B, &ngrp);
+        const int hs = check_shape(B, L, max_L, hq, hkv, &ngrp);
         if (hs != GAD_OK) return hs;
     }
+    const int nchunk = chunks_of(L);
     if (max_pages < 1) return fail(GAD_ERR_SHAPE, "max_pages=%d < 1", max_pages);
     if (page_size != 1 && page_size != 64)
         return fail(GAD_ERR_UNSUPPORTED, "page_size=%d (supported: 1, 64)", page_size);
@@ -312,7 +322,8 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     prm.B = B;
     prm.L = L;
     prm.ngrp = ngrp;
-    prm.NB = B * ngrp;
+    prm.nchunk = nchunk;
+    prm.NB = B * nchunk * ngrp;
     prm.max_pages = max_pages;
     prm.window = window;
     prm.use_rope = use_rope ? 1 : 0;
@@ -332,7 +343,7 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     long long per_req;
     if (window > 0) per_req = (static_cast<long long>(window) + L - 1 + gad::TILE - 1) / gad::TILE + 1;
     else per_req = (static_cast<long long>(max_pages) * page_size + gad::TILE - 1) / gad::TILE + 1;
-    long long tiles_upper_ll = per_req * B * ngrp;
+    long long tiles_upper_ll = per_req * prm.NB;
     const int tiles_upper = tiles_upper_ll > INT32_MAX ? INT32_MAX : static_cast<int>(tiles_upper_ll);
 
     const bool timed = events != nullptr;
@@ -347,16 +358,16 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     if (timed) cudaEventRecord(static_cast<cudaEvent_t>(events[1]), s);
 
     if (L == 1) {
-        st = ngrp > 1 ? launch_single<true>(prm, page_size, sms, tiles_upper, s, !timed)
-                      : launch_single<false>(prm, page_size, sms, tiles_upper, s, !timed);
+        st = prm.NB != B ? launch_single<true>(prm, page_size, sms, tiles_upper, s, !timed)
+                         : launch_single<false>(prm, page_size, sms, tiles_upper, s, !timed);
     } else {
         int optin = 0, dev = 0;
         if (cudaGetDevice(&dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
             return fail(GAD_ERR_CUDA, "shared-memory opt-in query failed");
         const bool deep = verify_deep_fits(prm.NB, optin);
-        st = ngrp > 1 ? launch_block<true>(prm, page_size, deep, sms, tiles_upper, s, !timed)
-                      : launch_block<false>(prm, page_size, deep, sms, tiles_upper, s, !timed);
+        st = prm.NB != B ? launch_block<true>(prm, page_size, deep, sms, tiles_upper, s, !timed)
+                         : launch_block<false>(prm, page_size, deep, sms, tiles_upper, s, !timed);
     }
     if (st != GAD_OK) return st;
     if (timed) cudaEventRecord(static_cast<cudaEvent_t>(events[2]), s);
@@ -390,7 +401,8 @@ int gad_attn_decode(const void* qkv, const int64_t* positions, const int32_t* se
                     void* out, void* workspace, size_t workspace_bytes, void* stream) {
     (void)seq_lens;
     return run_step(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale, B,
-                    L, GAD_HQ, GAD_HKV, max_pages, num_rows, page_size, window, use_rope, out,
+                    L, GAD_MAX_L, GAD_HQ, GAD_HKV, max_pages, num_rows, page_size, window,
+                    use_rope, out,
                     workspace, workspace_bytes, stream, nullptr);
 }
 
@@ -402,7 +414,8 @@ int gad_attn_decode_heads(const void* qkv, const int64_t* positions, const int32
                           size_t workspace_bytes, void* stream) {
     (void)seq_lens;
     return run_step(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale, B,
-                    L, hq, hkv, max_pages, num_rows, page_size, window, use_rope, out, workspace,
+                    L, GAD_MAX_L, hq, hkv, max_pages, num_rows, page_size, window, use_rope, out,
+                    workspace,
                     workspace_bytes, stream, nullptr);
 }
 
@@ -416,7 +429,8 @@ int gad_attn_decode_timed(const void* qkv, const int64_t* positions, const int32
     if (!events || !events[0] || !events[1] || !events[2] || !events[3])
         return fail(GAD_ERR_NULL, "events must hold four cudaEvent_t");
     return run_step(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale, B,
-                    L, GAD_HQ, GAD_HKV, max_pages, num_rows, page_size, window, use_rope, out,
+                    L, GAD_MAX_L, GAD_HQ, GAD_HKV, max_pages, num_rows, page_size, window,
+                    use_rope, out,
                     workspace, workspace_bytes, stream, events);
 }
 
@@ -431,8 +445,34 @@ int gad_attn_decode_heads_timed(const void* qkv, const int64_t* positions,
     if (!events || !events[0] || !events[1] || !events[2] || !events[3])
         return fail(GAD_ERR_NULL, "events must hold four cudaEvent_t");
     return run_step(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale, B,
-                    L, hq, hkv, max_pages, num_rows, page_size, window, use_rope, out, workspace,
+                    L, GAD_MAX_L, hq, hkv, max_pages, num_rows, page_size, window, use_rope, out,
+                    workspace,
                     workspace_bytes, stream, events);
+}
+
+int gad_attn_prefill(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                     const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,
+                     uint8_t* v_cache, const float* k_scale, const float* v_scale, int B, int L,
+                     int max_pages, int64_t num_rows, int page_size, int window, int use_rope,
+                     void* out, void* workspace, size_t workspace_bytes, void* stream) {
+    (void)seq_lens;
+    return run_step(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale, B,
+                    L, GAD_MAX_PREFILL_L, GAD_HQ, GAD_HKV, max_pages, num_rows, page_size,
+                    window, use_rope, out, workspace, workspace_bytes, stream, nullptr);
+}
+
+int gad_attn_prefill_timed(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                           const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,
+                           uint8_t* v_cache, const float* k_scale, const float* v_scale, int B,
+                           int L, int max_pages, int64_t num_rows, int page_size, int window,
+                           int use_rope, void* out, void* workspace, size_t workspace_bytes,
+                           void* stream, void* const* events) {
+    (void)seq_lens;
+    if (!events || !events[0] || !events[1] || !events[2] || !events[3])
+        return fail(GAD_ERR_NULL, "events must hold four cudaEvent_t");
+    return run_step(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale, B,
+                    L, GAD_MAX_PREFILL_L, GAD_HQ, GAD_HKV, max_pages, num_rows, page_size,
+                    window, use_rope, out, workspace, workspace_bytes, stream, events);
 }
 
 }  // extern "C"
@@ -491,6 +531,7 @@ extern "C" int gad_attn_decode_noalloc(const void* qkv, const int64_t* positions
     const int st = noalloc_scratch_address(&scratch);
     if (st != GAD_OK) return st;
     return run_step(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale, B,
-                    L, GAD_HQ, GAD_HKV, max_pages, num_rows, page_size, window, use_rope, out,
+                    L, GAD_MAX_L, GAD_HQ, GAD_HKV, max_pages, num_rows, page_size, window,
+                    use_rope, out,
                     scratch, static_cast<size_t>(GAD_NOALLOC_SCRATCH_BYTES), stream, nullptr);
 }

@@ -61,7 +61,8 @@ struct StepParams {
     __nv_bfloat16* out;
     int B, L, max_pages, window, use_rope;
     int ngrp;        // head groups (16 query + 2 KV heads each)
-    int NB;          // items of the tile list: B * ngrp; item i = (request i / ngrp, group i % ngrp)
+    int nchunk;      // token chunks per request: ceil(L / CHUNK)
+    int NB;          // items of the tile list: B * nchunk * ngrp (see ItemRef)
     int64_t num_rows;
     // workspace views
     __half* q_ws;    // [T][ngrp][16][64]  normalised (rotated) queries
@@ -72,10 +73,27 @@ struct StepParams {
     int tl;          // partials per (CTA, request) and KV-head group
 };
 
-// List item -> (request, head group).  One group is the common case, kept
-// free of integer divisions.
-__device__ __forceinline__ int item_req(int b, int ng) { return ng == 1 ? b : b / ng; }
-__device__ __forceinline__ int item_grp(int b, int ng) { return ng == 1 ? 0 : b % ng; }
+// Items of the tile list.  Item i = (request, token chunk, head group) with
+// i = (request * nchunk + chunk) * ngrp + group: a chunk is up to CHUNK
+// consecutive tokens of one request (a whole decode token or verify block,
+// or a slice of a longer prefill block), and its key range is the union of
+// its tokens' ranges.  The MULTI = false instantiations of the kernels serve
+// steps with one chunk and one group per request, where item = request.
+constexpr int CHUNK = 8;
+struct ItemRef {
+    int req;   // request
+    int grp;   // head group
+    int t0;    // first token (global index b * L + j)
+    int len;   // tokens in the chunk
+};
+template <bool MULTI>
+__device__ __forceinline__ ItemRef item_ref(const StepParams& p, int i) {
+    if (!MULTI) return ItemRef{i, 0, i * p.L, p.L};
+    const int grp = i % p.ngrp, rc = i / p.ngrp;
+    const int chunk = rc % p.nchunk, req = rc / p.nchunk;
+    const int j0 = chunk * CHUNK;
+    return ItemRef{req, grp, req * p.L + j0, min(CHUNK, p.L - j0)};
+}
 
 // Layout of StepParams::meta (ints).
 constexpr int META_TOTAL = 0;    // tiles in the step
@@ -187,17 +205,17 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) 
 // i % ngrp, so a request's groups are adjacent in the list and the CTAs that
 // share its pages run at about the same time.  Every thread of the block must
 // call it.  CTA 0 also writes the list to the workspace for the combine kernel.
-template <int TK, bool GROUPS>
+template <int TK, bool MULTI>
 __device__ __forceinline__ void build_tile_list(const StepParams& p, int* tpre, int* rlo, int* rhi,
                                                 int* rnew, int nthreads, int& total, int& per,
                                                 int& t0, int& t1) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int B = GROUPS ? p.NB : p.B, L = p.L, ng = GROUPS ? p.ngrp : 1;
+    const int B = MULTI ? p.NB : p.B;
     for (int b = tid; b < B; b += nthreads) {
-        const int req = item_req(b, ng);
+        const ItemRef it = item_ref<MULTI>(p, b);
         int lo = INT_MAX, hi = -1, first = INT_MAX;
-        for (int j = 0; j < L; ++j) {
-            const int pos = static_cast<int>(p.positions[static_cast<size_t>(req) * L + j]);
+        for (int j = 0; j < it.len; ++j) {
+            const int pos = static_cast<int>(p.positions[static_cast<size_t>(it.t0) + j]);
             const int l = p.window > 0 ? max(0, pos - p.window + 1) : 0;
             lo = min(lo, l);
             hi = max(hi, pos);
@@ -269,9 +287,9 @@ __device__ __forceinline__ int kappa(int l) {
     return (l & 8) | s;
 }
 
-// GROUPS: more than one head group (the one-group instantiation keeps the
+// MULTI: more than one head group (the one-group instantiation keeps the
 // list item equal to the request, with no index arithmetic for groups).
-template <int LT, int PS, int KG, int NS, int MINB, int TK, bool MERGE, bool GROUPS>
+template <int LT, int PS, int KG, int NS, int MINB, int TK, bool MERGE, bool MULTI>
 __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepParams p) {
     using C = DecodeCfg<LT, KG, NS, TK, MERGE>;
     constexpr int NT = C::NT, MT = C::MT, RG = C::RG;
@@ -290,12 +308,12 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
     const int rg = (warp / HKV) % RG;
     const int kg = warp / (HKV * RG);
     // B counts list items (request, head group); b below is an item index.
-    const int B = GROUPS ? p.NB : p.B, L = p.L, ng = GROUPS ? p.ngrp : 1;
+    const int B = MULTI ? p.NB : p.B, ng = MULTI ? p.ngrp : 1;
     const size_t row_pitch = static_cast<size_t>(ROWB) * ng;  // cache bytes per row
 
     // ---- request key ranges and the tile list (reads inputs only) ----
     int total, per, t0, t1;
-    build_tile_list<TK, GROUPS>(p, tpre, rlo, rhi, rnew, DEC_THREADS, total, per, t0, t1);
+    build_tile_list<TK, MULTI>(p, tpre, rlo, rhi, rnew, DEC_THREADS, total, per, t0, t1);
     if (t0 >= t1) return;
     // The normalised q and this step's new cache rows come from the prep kernel,
     // which may still be running (programmatic dependent launch): wait for it
@@ -333,7 +351,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
         if (tau >= t1) return;
         const int k0 = tile_k0(tau, b);
         int* dst = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
-        const int32_t* pt = p.page_table + static_cast<size_t>(item_req(b, ng)) * p.max_pages;
+        const int32_t* pt = p.page_table + static_cast<size_t>(item_ref<MULTI>(p, b).req) * p.max_pages;
         if (PS == 1) {
             if (tid < TK) {
                 const int k = k0 + tid;
@@ -355,7 +373,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
         const int* ix = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
         const uint32_t base = smem_addr(kv_smem + ((tau - t0) % NS) * C::STAGE);
         const int lo = rlo[b], hi = rhi[b];
-        const size_t gofs = static_cast<size_t>(item_grp(b, ng)) * ROWB;
+        const size_t gofs = static_cast<size_t>(item_ref<MULTI>(p, b).grp) * ROWB;
 #pragma unroll
         for (int i = 0; i < TK / 32; ++i) {
             const int r = (tid >> 3) + 32 * i;  // tile row
@@ -382,17 +400,19 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
     uint32_t qf[NT][8];
     int tok_lo[NT], tok_hi[NT];
     int req_lo_max = 0, req_hi_min = -1;
+    int cur_len = 0;  // tokens of the current item
 
     const int krow = kappa(gid);             // QK^T: rows krow, krow + 8 of each group
     const int vrow0 = kappa(2 * tig), vrow1 = kappa(2 * tig + 1);  // PV: + 0 and + 8
 
     auto begin_request = [&](int b) {
         ensure_prep();
-        const int req = item_req(b, ng), grp = item_grp(b, ng);
+        const ItemRef it = item_ref<MULTI>(p, b);
+        cur_len = it.len;
         req_lo_max = 0;
         req_hi_min = INT_MAX;
-        for (int j = 0; j < L; ++j) {
-            const int pos = static_cast<int>(p.positions[static_cast<size_t>(req) * L + j]);
+        for (int j = 0; j < it.len; ++j) {
+            const int pos = static_cast<int>(p.positions[static_cast<size_t>(it.t0) + j]);
             const int l = p.window > 0 ? max(0, pos - p.window + 1) : 0;
             req_lo_max = max(req_lo_max, l);
             req_hi_min = min(req_hi_min, pos);
@@ -400,13 +420,13 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int j = rg * NT + nt;
-            if (j < L) {
-                const size_t t = static_cast<size_t>(req) * L + j;
+            if (j < it.len) {
+                const size_t t = static_cast<size_t>(it.t0) + j;
                 const int pos = static_cast<int>(p.positions[t]);
                 tok_hi[nt] = pos;
                 tok_lo[nt] = p.window > 0 ? max(0, pos - p.window + 1) : 0;
                 const uint4* q = reinterpret_cast<const uint4*>(
-                    p.q_ws + ((t * ng + grp) * HQ + g * GRP + gid) * HD + 16 * tig);
+                    p.q_ws + ((t * ng + it.grp) * HQ + g * GRP + gid) * HD + 16 * tig);
                 const uint4 a = q[0], c = q[1];
                 qf[nt][0] = a.x; qf[nt][1] = a.y; qf[nt][2] = a.z; qf[nt][3] = a.w;
                 qf[nt][4] = c.x; qf[nt][5] = c.y; qf[nt][6] = c.z; qf[nt][7] = c.w;
@@ -598,7 +618,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int j = rg * NT + nt;
-                if (j >= L) continue;
+                if (j >= cur_len) continue;
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int h = g * GRP + 2 * tig + e;
@@ -678,7 +698,9 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams 
     const int t = blockIdx.x / hq_all, hh = blockIdx.x % hq_all;  // hh = 16 * group + h
     const int h = hh % HQ;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = (t / p.L) * ng + hh / HQ, j = t % p.L;        // list item (request, group)
+    // list item (request, chunk, group) and the token's place in the chunk
+    const int jr = t % p.L;
+    const int b = ((t / p.L) * p.nchunk + jr / CHUNK) * ng + hh / HQ, j = jr % CHUNK;
     const int tp = p.meta[META_PREFIX + b];
     const int n = p.meta[META_PREFIX + b + 1] - tp;
     const int per = p.meta[META_PER];

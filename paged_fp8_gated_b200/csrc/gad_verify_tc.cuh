@@ -108,8 +108,8 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
 
 }  // namespace vtc
 
-// GROUPS: more than one head group (see decode_kernel).
-template <int PS, int NS, bool GROUPS>
+// MULTI: more than one head group (see decode_kernel).
+template <int PS, int NS, bool MULTI>
 __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepParams p) {
     using namespace vtc;
     using C = Cfg<NS>;
@@ -129,10 +129,10 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
 
     const int tid = threadIdx.x, warp = tid >> 5;
     // B counts list items (request, head group); b below is an item index.
-    const int B = GROUPS ? p.NB : p.B, L = p.L, ng = GROUPS ? p.ngrp : 1;
+    const int B = MULTI ? p.NB : p.B, ng = MULTI ? p.ngrp : 1;
 
     int total, per, t0, t1;
-    build_tile_list<TK, GROUPS>(p, tpre, rlo, rhi, rnew, THREADS, total, per, t0, t1);
+    build_tile_list<TK, MULTI>(p, tpre, rlo, rhi, rnew, THREADS, total, per, t0, t1);
     if (t0 >= t1) return;
 
     const uint32_t bar0 = smem_addr(ctrl);
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
             if (tau >= t1) return;
             const int k0 = tile_k0(tau, b);
             int* dst = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
-            const int32_t* pt = p.page_table + static_cast<size_t>(item_req(b, ng)) * p.max_pages;
+            const int32_t* pt = p.page_table + static_cast<size_t>(item_ref<MULTI>(p, b).req) * p.max_pages;
             if (PS == 1) {
                 if (ltid < TK) {
                     const int k = k0 + ltid;
@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
             const uint32_t base = smem_addr(raw + ((tau - t0) % NS) * RAW_STAGE);
             const int lo = rlo[b], hi = rhi[b];
             const size_t row_pitch = static_cast<size_t>(ROWB) * ng;
-            const size_t gofs = static_cast<size_t>(item_grp(b, ng)) * ROWB;
+            const size_t gofs = static_cast<size_t>(item_ref<MULTI>(p, b).grp) * ROWB;
             constexpr int ROWS = TK * 8 / LOADERS;  // rows per thread
             const int j = ltid & 7;                 // 16-byte chunk
             // all page-table reads first, then the copies (the copies are ordered
@@ -250,13 +250,13 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
         auto write_q = [&](int b) {
             ensure_prep();
             const int g = ltid >> 6, j = (ltid >> 3) & 7, hh = ltid & 7;
-            const size_t req = static_cast<size_t>(item_req(b, ng)), grp = static_cast<size_t>(item_grp(b, ng));
+            const ItemRef it = item_ref<MULTI>(p, b);
             uint32_t q[32], z[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) z[c] = 0u;
-            if (j < L) {
+            if (j < it.len) {
                 const uint4* src = reinterpret_cast<const uint4*>(
-                    p.q_ws + (((req * L + j) * ng + grp) * HQ + g * GRP + hh) * HD);
+                    p.q_ws + (((static_cast<size_t>(it.t0) + j) * ng + it.grp) * HQ + g * GRP + hh) * HD);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const uint4 v = src[c];
@@ -422,6 +422,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
         int seg_b = -1, seg_t1 = 0, k0 = 0;  // current request, end of its tiles here, tile key
         float m_run = -INFINITY, l_run = 0.f;
         int lo_j = INT_MAX, hi_j = -1;
+        int seg_len = 0;  // tokens of the current item
         for (int i = 0; ct < t1; ++i) {
             const bool seg_start = cb != seg_b;
             if (seg_start) {
@@ -430,8 +431,10 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 k0 = tile_k0(ct, cb);
                 m_run = -INFINITY;
                 l_run = 0.f;
-                if (j < L) {
-                    const int pos = static_cast<int>(p.positions[static_cast<size_t>(item_req(cb, ng)) * L + j]);
+                const ItemRef it = item_ref<MULTI>(p, cb);
+                seg_len = it.len;
+                if (j < it.len) {
+                    const int pos = static_cast<int>(p.positions[static_cast<size_t>(it.t0) + j]);
                     hi_j = pos;
                     lo_j = p.window > 0 ? max(0, pos - p.window + 1) : 0;
                 } else {
@@ -523,7 +526,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 tc_ld32(oa, o);
                 tc_ld32(oa + 32u, o + 32);
                 tc_wait_ld();
-                if (j < L) {
+                if (j < seg_len) {
                     const size_t slot = static_cast<size_t>(blockIdx.x) + cb;
                     const size_t base = (slot * p.lt + j) * HQ + qh;
                     float4* dst = reinterpret_cast<float4*>(p.part_o + base * HD);

@@ -54,7 +54,7 @@ class Spec:
     gate_std: float = 1.0
     seed: int = 0
     spare_pages: int = 0       # unused pages in the pool
-    dist: str = "normal"       # "normal", "coherent" or "edges" (see make_inputs)
+    dist: str = "normal"       # "normal", "coherent", "edges" or "outliers" (see make_inputs)
     hq: int = HQ               # query heads
     hkv: int = HKV             # key/value heads
     extra: dict = field(default_factory=dict)
@@ -111,6 +111,17 @@ def make_inputs(spec: Spec) -> dict:
     qkv = torch.randn(T, qkv_cols(hq, hkv), generator=gen)
     if spec.gate_std != 1.0:
         qkv[:, (hq + 2 * hkv) * D:] *= spec.gate_std
+    outlier_dims = None
+    if spec.dist == "outliers":
+        # Two channels per KV head carry 16x the scale in q and k (and in the
+        # cached keys below), so after the QK-norm those channels dominate the
+        # directions and the scores reach several tens: sharp attention.
+        outlier_dims = torch.stack([torch.randperm(D, generator=gen)[:2] for _ in range(hkv)])
+        grp = hq // hkv
+        for g in range(hkv):
+            for c in outlier_dims[g].tolist():
+                qkv[:, [(g * grp + h) * D + c for h in range(grp)]] *= 16.0
+                qkv[:, hq * D + g * D + c] *= 16.0
     qkv = qkv.to(torch.bfloat16)
 
     # Pre-existing cache: K = E4M3(unit-RMS N(0,1) / scale), V = E4M3(N(0,1) / scale),
@@ -122,7 +133,11 @@ def make_inputs(spec: Spec) -> dict:
     inv = 1.0 / float(spec.kv_scale)
     for r0 in range(0, rows, chunk):
         r1 = min(rows, r0 + chunk)
-        kx = _unit_rms(torch.randn(r1 - r0, hkv, D, generator=gen))
+        kx = torch.randn(r1 - r0, hkv, D, generator=gen)
+        if outlier_dims is not None:
+            for g in range(hkv):
+                kx[:, g, outlier_dims[g]] *= 16.0
+        kx = _unit_rms(kx)
         vx = torch.randn(r1 - r0, hkv, D, generator=gen)
         k_cache[r0:r1] = _to_e4m3_codes(kx * inv)
         v_cache[r0:r1] = _to_e4m3_codes(vx * inv)
@@ -153,7 +168,7 @@ def make_inputs(spec: Spec) -> dict:
                     row = int(page_table[b, key // ps]) * ps + key % ps
                     kdir = _unit_rms(qraw[t])
                     k_cache[row] = _to_e4m3_codes(kdir * (3.0 * inv))
-    elif spec.dist != "normal":
+    elif spec.dist not in ("normal", "outliers"):
         raise ValueError(f"unknown dist {spec.dist!r}")
 
     return dict(
@@ -235,6 +250,22 @@ def named(name: str, seed: int = 0) -> Spec:
                                  hq=DP_HQ, hkv=DP_HKV, seed=seed + 62),
         "dp2_full_v8_coherent": Spec("dp2_full_v8_coherent", B=2, L=8, ctx=20000, page_size=64,
                                      dist="coherent", hq=DP_HQ, hkv=DP_HKV, seed=seed + 63),
+        # prefill blocks (the page "Prefill layer (muse_prefill_layer)", its load
+        # table): 753 new tokens on an 80,000-token context, one or four
+        # conversations; a first turn of 16,384 tokens after 0, 32,768 or 65,536
+        "prefill1_sliding": Spec("prefill1_sliding", B=1, L=753, ctx=80000, window=2048,
+                                 use_rope=True, seed=seed + 71),
+        "prefill1_full": Spec("prefill1_full", B=1, L=753, ctx=80000, seed=seed + 72),
+        "prefill4_sliding": Spec("prefill4_sliding", B=4, L=753, ctx=80000, window=2048,
+                                 use_rope=True, seed=seed + 73),
+        "prefill4_full": Spec("prefill4_full", B=4, L=753, ctx=80000, seed=seed + 74),
+        "prefill16k_ctx0_full": Spec("prefill16k_ctx0_full", B=1, L=16384, ctx=0, seed=seed + 75),
+        "prefill16k_ctx32k_sliding": Spec("prefill16k_ctx32k_sliding", B=1, L=16384, ctx=32768,
+                                          window=2048, use_rope=True, seed=seed + 76),
+        "prefill16k_ctx32k_full": Spec("prefill16k_ctx32k_full", B=1, L=16384, ctx=32768,
+                                       seed=seed + 77),
+        "prefill16k_ctx64k_full": Spec("prefill16k_ctx64k_full", B=1, L=16384, ctx=65536,
+                                       seed=seed + 78),
     }
     return specs[name]
 
@@ -253,3 +284,14 @@ LOAD_SET = [
     ("verify 32", "sliding", "verify32_sliding"), ("verify 32", "full", "verify32_full"),
 ]
 LAYER_WEIGHT = {"sliding": 46.0, "full": 16.0}
+
+# The prefill page's eight scored shapes (load, layer, q_len, ctx) -> workload,
+# with the weight it gives each shape inside its load.
+PREFILL_SET = [
+    ("turn 1", "sliding", "prefill1_sliding", 46.0), ("turn 1", "full", "prefill1_full", 16.0),
+    ("turn 4", "sliding", "prefill4_sliding", 46.0), ("turn 4", "full", "prefill4_full", 16.0),
+    ("first turn", "full ctx 0", "prefill16k_ctx0_full", 16.0),
+    ("first turn", "sliding ctx 32768", "prefill16k_ctx32k_sliding", 138.0),
+    ("first turn", "full ctx 32768", "prefill16k_ctx32k_full", 16.0),
+    ("first turn", "full ctx 65536", "prefill16k_ctx64k_full", 16.0),
+]

@@ -96,6 +96,25 @@ def test_heads_argument_checks(lib, over, status):
     assert lib.last_error()
 
 
+@pytest.mark.parametrize("over,status", [
+    (dict(L=9), -2),                           # the decode entry point stops at 8 tokens
+    (dict(L=9, prefill=True, qkv=FAKE + 8), -3),   # the prefill one takes them
+    (dict(L=65537, prefill=True), -2),
+    (dict(B=3, L=16384, prefill=True), -2),    # 3 x 2048 chunks > 4096 items
+    (dict(B=2, L=16384, prefill=True, qkv=None), -1),
+])
+def test_prefill_argument_checks(lib, over, status):
+    assert lib.raw_call(**_ok_args(**over)) == status
+    assert lib.last_error()
+
+
+def test_prefill_workspace_query_limits(lib):
+    so = lib.lib()
+    assert so.gad_attn_prefill_workspace_bytes(3, 16384) == 0
+    assert "items" in lib.last_error()
+    assert so.gad_attn_prefill_workspace_bytes(1, 0) == 0
+
+
 def test_heads_workspace_query_rejects_bad_heads(lib):
     so = lib.lib()
     assert so.gad_attn_workspace_bytes_heads(4, 1, 16, 4) == 0

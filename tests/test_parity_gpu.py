@@ -125,6 +125,47 @@ def test_heads_dp_equals_eight_tp8_steps(cuda_dev):
         assert np.array_equal(v_dp[:, 128 * c:128 * (c + 1)], v_tp), c
 
 
+# Prefill blocks (gad_attn_prefill): the prefill page's five gating tests,
+# ragged chunk edges, then its scored shapes on sampled heads.
+SMALL_PREFILL = [
+    S("pf_b1_ctx0_sliding_q300", B=1, L=300, ctx=0, window=2048, use_rope=True, seed=150),
+    S("pf_b1_ctx3000_full_q753", B=1, L=753, ctx=3000, seed=151),
+    S("pf_b2_ctx2500_sliding_q753", B=2, L=753, ctx=2500, window=2048, use_rope=True, seed=152),
+    # "dist outliers", the one test on 64-token pages
+    S("pf_b3_ctx5000_full_q200_outliers_p64", B=3, L=200, ctx=5000, page_size=64,
+      dist="outliers", seed=153),
+    S("pf_L9_ragged", B=3, L=9, seq_lens=[0, 70, 1000], page_size=64, seed=155),
+    S("pf_L13_window_edge", B=2, L=13, seq_lens=[2040, 5000], window=2048, use_rope=True,
+      seed=156),
+    S("pf_L100_window_small", B=2, L=100, seq_lens=[10, 300], window=64, use_rope=True,
+      seed=157),
+]
+
+
+@pytest.mark.parametrize("spec", SMALL_PREFILL, ids=lambda s: s.name)
+def test_prefill_compare(spec, cuda_dev):
+    _check(W.make_inputs(spec), label=spec.name)
+
+
+def test_prefill_q4096_sliding_sampled(cuda_dev):
+    # "batch 1, ctx 4096, layer sliding, q_len 4096, page 1"
+    inp = W.make_inputs(S("pf_b1_ctx4096_sliding_q4096", B=1, L=4096, ctx=4096, window=2048,
+                          use_rope=True, seed=154))
+    _check(inp, want=H.sample_want(4096, 512, seed=5), label="q4096")
+
+
+PREFILL_FULL = {"prefill1_full": 96, "prefill4_sliding": 96, "prefill16k_ctx0_full": 64,
+                "prefill16k_ctx64k_full": 48}
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", sorted(PREFILL_FULL))
+def test_prefill_named_sampled(name, cuda_dev):
+    inp = W.make_inputs(W.named(name))
+    T = inp["B"] * inp["L"]
+    _check(inp, want=H.sample_want(T, PREFILL_FULL[name], seed=6), label=name)
+
+
 def test_verify_full_ctx100k(cuda_dev):
     # "batch 2, ctx 100000, heads tp8, layer full, q_len 8, page 1"
     _check(W.make_inputs(S("b2_ctx100k_full_v8", B=2, L=8, ctx=100000, seed=121)))
