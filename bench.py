@@ -52,16 +52,18 @@ TRAFFIC = {("decode32_full", "64c5ab721f0a7f48"): 474521600,
            ("verify16_full", "9c1a1c537fa1f9f0"): 337947136}
 
 # Sources of the step's main kernel: decode_kernel for single-token steps,
-# verify_tc_kernel for verify blocks (the launch code is in gad_attn.cu).
+# verify_tc_kernel for verify blocks, prefill_tc_kernel for longer blocks (the
+# launch code is in gad_attn.cu).
 _CSRC = os.path.join(ROOT, "paged_fp8_gated_b200", "csrc")
 KERNEL_SOURCES = {
     "decode_kernel": ["gad_kernels.cuh", "gad_ptx.cuh"],
     "verify_tc_kernel": ["gad_kernels.cuh", "gad_ptx.cuh", "gad_tc.cuh", "gad_verify_tc.cuh"],
+    "prefill_tc_kernel": ["gad_kernels.cuh", "gad_ptx.cuh", "gad_tc.cuh", "gad_prefill_tc.cuh"],
 }
 
 
 def main_kernel(L: int) -> str:
-    return "decode_kernel" if L == 1 else "verify_tc_kernel"
+    return "decode_kernel" if L == 1 else "verify_tc_kernel" if L <= 8 else "prefill_tc_kernel"
 
 
 def kernel_source_hash(kernel: str = "decode_kernel") -> str:

@@ -49,7 +49,7 @@ extern "C" {
 #define GAD_ROW_BYTES 128  /* one cache row: 2 KV heads x 64 E4M3 codes */
 #define GAD_MAX_L 8        /* longest verify block           */
 #define GAD_MAX_B 4096     /* most requests in one call; also the most
-                              (request, 8-token chunk, head group) items  */
+                              work items (request, token chunk, heads)    */
 #define GAD_MAX_PREFILL_L 65536 /* longest block of gad_attn_prefill */
 #define GAD_NOALLOC_SCRATCH_BYTES (16u << 20) /* built-in scratch of gad_attn_decode_noalloc */
 
@@ -193,8 +193,10 @@ int gad_attn_decode_heads_timed(const void* qkv, const int64_t* positions,
  * and error behaviour are those of gad_attn_decode with L tokens per request
  * (token t = b * L + j at position positions[t], contract positions[t] =
  * seq_lens[b] + j); the workspace comes from gad_attn_prefill_workspace_bytes.
- * Each request's tokens are split into chunks of 8 and B * ceil(L / 8) may
- * not exceed GAD_MAX_B (GAD_ERR_SHAPE), e.g. L = 16,384 admits B <= 2.
+ * For L > GAD_MAX_L each request's tokens are split into chunks of 32, one
+ * work item per (chunk, KV head), and 2 B ceil(L / 32) may not exceed
+ * GAD_MAX_B (GAD_ERR_SHAPE), e.g. L = 16,384 admits B <= 4; L <= GAD_MAX_L
+ * runs as gad_attn_decode.
  */
 int gad_attn_prefill(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
                      const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,

@@ -18,6 +18,7 @@
 
 #include "gad_attn.h"
 #include "gad_kernels.cuh"
+#include "gad_prefill_tc.cuh"
 #include "gad_verify_tc.cuh"
 
 namespace {
@@ -48,22 +49,40 @@ constexpr int kV1SingleKG = 4, kV1SingleNS = 3, kV1SingleTK = 128;
 
 struct WsLayout {
     size_t q_off, po_off, pml_off, meta_off, total;
-    int lt;
 };
 
-int chunks_of(int L) { return (L + gad::CHUNK - 1) / gad::CHUNK; }
+// How a step's tokens and heads become tile-list items.  Blocks longer than
+// GAD_MAX_L (prefill) run prefill_tc_kernel on items (request, 32-token
+// chunk, KV head) whose partial rows hold 32 tokens x 8 heads; other steps
+// run decode_kernel or verify_tc_kernel on items (request, head group) with
+// partial rows of up to 8 tokens x 16 heads.
+struct StepShape {
+    bool prefill;
+    int chunk, nchunk, nsub, hp, lt;
+    long long NB;
+};
+StepShape shape_of(int B, int L, int ngrp) {
+    StepShape sh{};
+    sh.prefill = L > GAD_MAX_L;
+    sh.chunk = sh.prefill ? gad::PF_CHUNK : gad::CHUNK;
+    sh.nchunk = (L + sh.chunk - 1) / sh.chunk;
+    sh.nsub = sh.prefill ? GAD_HKV : ngrp;
+    sh.hp = sh.prefill ? gad::GRP : gad::HQ;
+    sh.lt = sh.prefill ? gad::PF_CHUNK : (L == 1 ? 1 : gad::CHUNK);
+    sh.NB = static_cast<long long>(B) * sh.nchunk * sh.nsub;
+    return sh;
+}
 
 // Partial slots: (CTAs + NB) * partials per (CTA, list item), each holding lt
-// tokens x 16 heads x (64 values + max + sum); NB = B * chunks * ngrp list
-// items (request, chunk of up to 8 tokens, group of 16 query and 2 KV heads).
+// tokens x hp heads x (64 values + max + sum).
 WsLayout ws_layout(int B, int L, int ngrp, int sms) {
     WsLayout w{};
-    w.lt = L == 1 ? 1 : gad::CHUNK;
-    const size_t NB = static_cast<size_t>(B) * chunks_of(L) * ngrp;
+    const StepShape sh = shape_of(B, L, ngrp);
+    const size_t NB = static_cast<size_t>(sh.NB);
     const size_t units =
         (static_cast<size_t>(sms) * kMaxCtasPerSm + NB) * (L == 1 ? kV1SingleKG : 1);
     const size_t T = static_cast<size_t>(B) * L;
-    const size_t parts = units * w.lt * GAD_HQ;
+    const size_t parts = units * sh.lt * sh.hp;
     size_t off = 0;
     w.q_off = off;
     off = align_up(off + T * ngrp * GAD_HQ * GAD_HEAD_DIM * 2);
@@ -199,11 +218,14 @@ int check_shape(int B, int L, int max_L, int hq, int hkv, int* ngrp) {
                     "hq=%d, hkv=%d: supported head counts are hkv a positive multiple of %d and "
                     "hq = %d hkv", hq, hkv, GAD_HKV, GAD_HQ / GAD_HKV);
     *ngrp = hkv / GAD_HKV;
-    const long long items = static_cast<long long>(B) * chunks_of(L) * *ngrp;
-    if (items > GAD_MAX_B)
+    if (L > GAD_MAX_L && *ngrp != 1)
+        return fail(GAD_ERR_UNSUPPORTED, "blocks longer than %d tokens take %d query and %d KV heads",
+                    GAD_MAX_L, GAD_HQ, GAD_HKV);
+    const StepShape sh = shape_of(B, L, *ngrp);
+    if (sh.NB > GAD_MAX_B)
         return fail(GAD_ERR_SHAPE,
-                    "B=%d requests x %d chunks of 8 tokens x %d head groups = %lld items exceeds %d",
-                    B, chunks_of(L), *ngrp, items, GAD_MAX_B);
+                    "B=%d requests x %d chunks of %d tokens x %d = %lld tile-list items exceeds %d",
+                    B, sh.nchunk, sh.chunk, sh.nsub, sh.NB, GAD_MAX_B);
     return GAD_OK;
 }
 
@@ -213,6 +235,43 @@ size_t workspace_bytes(int B, int L, int max_L, int hq, int hkv) {
     int sms = 0, major = 0;
     if (current_device_sms(&sms, &major) != GAD_OK) return 0;
     return ws_layout(B, L, ngrp, sms).total;
+}
+
+// Prefill blocks on the tcgen05 prefill kernel: one CTA per SM.
+constexpr int kPtcStages = 6;
+template <int PS>
+int launch_prefill_tc(const gad::StepParams& prm, int sms, int tiles_upper, cudaStream_t stream,
+                      bool pdl) {
+    using C = gad::ptc::Cfg<kPtcStages>;
+    auto kern = gad::prefill_tc_kernel<PS, kPtcStages>;
+    const size_t smem = C::smem_bytes(prm.NB);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", dev);
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(C::smem_bytes(GAD_MAX_B)));
+        if (e != cudaSuccess)
+            return fail(GAD_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    long long grid = sms;
+    if (grid > tiles_upper) grid = tiles_upper;
+    if (grid < 1) grid = 1;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(gad::ptc::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr = pdl_attr();
+    cfg.attrs = &attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, prm);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
+    return GAD_OK;
 }
 
 // Single-token steps and verify blocks, by page size (and stage count).
@@ -283,7 +342,7 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
         const int hs = check_shape(B, L, max_L, hq, hkv, &ngrp);
         if (hs != GAD_OK) return hs;
     }
-    const int nchunk = chunks_of(L);
+    const StepShape sh = shape_of(B, L, ngrp);
     if (max_pages < 1) return fail(GAD_ERR_SHAPE, "max_pages=%d < 1", max_pages);
     if (page_size != 1 && page_size != 64)
         return fail(GAD_ERR_UNSUPPORTED, "page_size=%d (supported: 1, 64)", page_size);
@@ -322,8 +381,11 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     prm.B = B;
     prm.L = L;
     prm.ngrp = ngrp;
-    prm.nchunk = nchunk;
-    prm.NB = B * nchunk * ngrp;
+    prm.chunk = sh.chunk;
+    prm.nchunk = sh.nchunk;
+    prm.nsub = sh.nsub;
+    prm.hp = sh.hp;
+    prm.NB = static_cast<int>(sh.NB);
     prm.max_pages = max_pages;
     prm.window = window;
     prm.use_rope = use_rope ? 1 : 0;
@@ -333,7 +395,7 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     prm.part_o = reinterpret_cast<float*>(ws + w.po_off);
     prm.part_ml = reinterpret_cast<float*>(ws + w.pml_off);
     prm.meta = reinterpret_cast<int*>(ws + w.meta_off);
-    prm.lt = w.lt;
+    prm.lt = sh.lt;
     prm.tl = L == 1 ? kV1SingleKG : 1;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -357,7 +419,10 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "prep launch: %s", cudaGetErrorString(e));
     if (timed) cudaEventRecord(static_cast<cudaEvent_t>(events[1]), s);
 
-    if (L == 1) {
+    if (sh.prefill) {
+        st = page_size == 1 ? launch_prefill_tc<1>(prm, sms, tiles_upper, s, !timed)
+                            : launch_prefill_tc<64>(prm, sms, tiles_upper, s, !timed);
+    } else if (L == 1) {
         st = prm.NB != B ? launch_single<true>(prm, page_size, sms, tiles_upper, s, !timed)
                          : launch_single<false>(prm, page_size, sms, tiles_upper, s, !timed);
     } else {
@@ -379,7 +444,13 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     cudaLaunchAttribute attr = pdl_attr();
     cfg.attrs = &attr;
     cfg.numAttrs = timed ? 0 : 1;
-    if (T * ngrp <= 16) {
+    if (sh.prefill) {  // one warp per (token, head)
+        constexpr int per_block = gad::COMBW_THREADS / 32;
+        cfg.gridDim = dim3(static_cast<unsigned>((static_cast<long long>(T) * gad::HQ * ngrp +
+                                                  per_block - 1) / per_block));
+        cfg.blockDim = dim3(gad::COMBW_THREADS);
+        e = cudaLaunchKernelEx(&cfg, gad::combine_warp_kernel, prm);
+    } else if (T * ngrp <= 16) {
         cfg.blockDim = dim3(1024);
         e = cudaLaunchKernelEx(&cfg, gad::combine_kernel<1024>, prm);
     } else {

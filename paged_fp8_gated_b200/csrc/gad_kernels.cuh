@@ -61,8 +61,11 @@ struct StepParams {
     __nv_bfloat16* out;
     int B, L, max_pages, window, use_rope;
     int ngrp;        // head groups (16 query + 2 KV heads each)
-    int nchunk;      // token chunks per request: ceil(L / CHUNK)
-    int NB;          // items of the tile list: B * nchunk * ngrp (see ItemRef)
+    int chunk;       // tokens per item chunk (CHUNK, or PF_CHUNK for prefill_tc_kernel)
+    int nchunk;      // token chunks per request: ceil(L / chunk)
+    int nsub;        // items per chunk: head groups, or KV heads for prefill_tc_kernel
+    int hp;          // query heads per partial row block (16, or 8 for prefill_tc_kernel)
+    int NB;          // items of the tile list: B * nchunk * nsub (see ItemRef)
     int64_t num_rows;
     // workspace views
     __half* q_ws;    // [T][ngrp][16][64]  normalised (rotated) queries
@@ -73,26 +76,28 @@ struct StepParams {
     int tl;          // partials per (CTA, request) and KV-head group
 };
 
-// Items of the tile list.  Item i = (request, token chunk, head group) with
-// i = (request * nchunk + chunk) * ngrp + group: a chunk is up to CHUNK
+// Items of the tile list.  Item i = (request, token chunk, sub) with
+// i = (request * nchunk + chunk) * nsub + sub: a chunk is up to p.chunk
 // consecutive tokens of one request (a whole decode token or verify block,
 // or a slice of a longer prefill block), and its key range is the union of
-// its tokens' ranges.  The MULTI = false instantiations of the kernels serve
-// steps with one chunk and one group per request, where item = request.
-constexpr int CHUNK = 8;
+// its tokens' ranges.  sub is the head group for decode_kernel and
+// verify_tc_kernel, the KV head for prefill_tc_kernel.  The MULTI = false
+// instantiations serve steps with one item per request, where item = request.
+constexpr int CHUNK = 8;      // tokens per item: decode and verify kernels
+constexpr int PF_CHUNK = 32;  // tokens per item: prefill_tc_kernel
 struct ItemRef {
     int req;   // request
-    int grp;   // head group
+    int grp;   // sub: head group, or KV head (prefill_tc_kernel)
     int t0;    // first token (global index b * L + j)
     int len;   // tokens in the chunk
 };
 template <bool MULTI>
 __device__ __forceinline__ ItemRef item_ref(const StepParams& p, int i) {
     if (!MULTI) return ItemRef{i, 0, i * p.L, p.L};
-    const int grp = i % p.ngrp, rc = i / p.ngrp;
+    const int sub = i % p.nsub, rc = i / p.nsub;
     const int chunk = rc % p.nchunk, req = rc / p.nchunk;
-    const int j0 = chunk * CHUNK;
-    return ItemRef{req, grp, req * p.L + j0, min(CHUNK, p.L - j0)};
+    const int j0 = chunk * p.chunk;
+    return ItemRef{req, sub, req * p.L + j0, min(p.chunk, p.L - j0)};
 }
 
 // Layout of StepParams::meta (ints).
@@ -221,9 +226,13 @@ __device__ __forceinline__ void build_tile_list(const StepParams& p, int* tpre, 
             hi = max(hi, pos);
             first = min(first, pos);
         }
+        // Keys at or above the request's first position are written by this
+        // step (by the prep kernel, which may still be running), including the
+        // keys of the request's earlier chunks.
+        if (MULTI) first = min(first, static_cast<int>(p.positions[static_cast<size_t>(it.req) * p.L]));
         rlo[b] = lo;
         rhi[b] = hi;
-        rnew[b] = first;  // keys at or above this one are written by this step
+        rnew[b] = first;
         tpre[b + 1] = (hi >= lo && hi >= 0) ? (hi / TK - lo / TK + 1) : 0;
     }
     if (tid == 0) tpre[0] = 0;
@@ -696,11 +705,12 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams 
     __shared__ float red_ss[4];
     const int ng = p.ngrp, hq_all = HQ * ng;
     const int t = blockIdx.x / hq_all, hh = blockIdx.x % hq_all;  // hh = 16 * group + h
-    const int h = hh % HQ;
+    const int h = hh % p.hp;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // list item (request, chunk, group) and the token's place in the chunk
+    // list item (request, chunk, sub) and the token's place in the chunk; the
+    // partial rows of an item hold p.hp query heads (sub = hh / hp)
     const int jr = t % p.L;
-    const int b = ((t / p.L) * p.nchunk + jr / CHUNK) * ng + hh / HQ, j = jr % CHUNK;
+    const int b = ((t / p.L) * p.nchunk + jr / p.chunk) * p.nsub + hh / p.hp, j = jr % p.chunk;
     const int tp = p.meta[META_PREFIX + b];
     const int n = p.meta[META_PREFIX + b + 1] - tp;
     const int per = p.meta[META_PER];
@@ -717,7 +727,7 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams 
     // request has max -inf and is skipped).
     auto slot_base = [&](int s) {
         const int c = c_lo + s / TL, tl = s % TL;
-        return ((static_cast<size_t>(c + b) * TL + tl) * p.lt + j) * HQ + h;
+        return ((static_cast<size_t>(c + b) * TL + tl) * p.lt + j) * p.hp + h;
     };
     // 1. global max over the slots
     float mx = -INFINITY;
@@ -769,6 +779,65 @@ __global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams 
             p.qkv[static_cast<size_t>(t) * QKV_COLS * ng + G_OFF * ng + hh * HD + tid]);
         outp[tid] = __float2bfloat16(a * rinv / (1.0f + expf(-g)));
     }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 3b: the same merge and gated output norm with one warp per (token,
+// query head), lane l holding dims 2l and 2l + 1.  For prefill blocks, whose
+// items each span few CTAs, so a (token, head) has few partials and the
+// block-per-(token, head) form above would spend its time on launch overhead.
+// ---------------------------------------------------------------------------
+constexpr int COMBW_THREADS = 256;
+__global__ void __launch_bounds__(COMBW_THREADS) combine_warp_kernel(const StepParams p) {
+    pdl_wait_primary();
+    const int ng = p.ngrp, hq_all = HQ * ng;
+    const int lane = threadIdx.x & 31;
+    const long long gw = static_cast<long long>(blockIdx.x) * (COMBW_THREADS / 32) + (threadIdx.x >> 5);
+    if (gw >= static_cast<long long>(p.B) * p.L * hq_all) return;
+    const int t = static_cast<int>(gw / hq_all), hh = static_cast<int>(gw % hq_all);
+    const int h = hh % p.hp;
+    const int jr = t % p.L;
+    const int b = ((t / p.L) * p.nchunk + jr / p.chunk) * p.nsub + hh / p.hp, j = jr % p.chunk;
+    const int tp = p.meta[META_PREFIX + b];
+    const int n = p.meta[META_PREFIX + b + 1] - tp;
+    const int per = p.meta[META_PER];
+    __nv_bfloat16* outp = p.out + static_cast<size_t>(t) * OUT_COLS * ng + hh * HD + 2 * lane;
+    if (n <= 0 || per <= 0) {  // no key in range (positions outside the contract)
+        outp[0] = outp[1] = __float2bfloat16(NAN);
+        return;
+    }
+    const int c_lo = tp / per, c_hi = (tp + n - 1) / per;
+    const int TL = p.tl;
+    const int ns = (c_hi - c_lo + 1) * TL;
+    auto slot_base = [&](int s) {
+        const int c = c_lo + s / TL, tl = s % TL;
+        return ((static_cast<size_t>(c + b) * TL + tl) * p.lt + j) * p.hp + h;
+    };
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, p.part_ml[slot_base(s) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float o0 = 0.f, o1 = 0.f, l = 0.f;
+    for (int s = 0; s < ns; ++s) {
+        const size_t base = slot_base(s);
+        const float ms = p.part_ml[base * 2];
+        if (ms == -INFINITY) continue;
+        const float w = exp2f(ms - M);
+        const float2 o = *reinterpret_cast<const float2*>(p.part_o + base * HD + 2 * lane);
+        o0 += w * o.x;
+        o1 += w * o.y;
+        l += w * p.part_ml[base * 2 + 1];
+    }
+    const float vs = __ldg(p.v_scale);
+    const float a0 = o0 / l * vs, a1 = o1 / l * vs;
+    float ss = a0 * a0 + a1 * a1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rinv = 1.0f / sqrtf(ss * (1.0f / 64.0f) + 1e-6f);
+    const __nv_bfloat16* gp = p.qkv + static_cast<size_t>(t) * QKV_COLS * ng + G_OFF * ng + hh * HD + 2 * lane;
+    const float g0 = __bfloat162float(gp[0]), g1 = __bfloat162float(gp[1]);
+    outp[0] = __float2bfloat16(a0 * rinv / (1.0f + expf(-g0)));
+    outp[1] = __float2bfloat16(a1 * rinv / (1.0f + expf(-g1)));
 }
 
 }  // namespace gad

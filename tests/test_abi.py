@@ -100,7 +100,7 @@ def test_heads_argument_checks(lib, over, status):
     (dict(L=9), -2),                           # the decode entry point stops at 8 tokens
     (dict(L=9, prefill=True, qkv=FAKE + 8), -3),   # the prefill one takes them
     (dict(L=65537, prefill=True), -2),
-    (dict(B=3, L=16384, prefill=True), -2),    # 3 x 2048 chunks > 4096 items
+    (dict(B=5, L=16384, prefill=True), -2),    # 5 x 512 chunks x 2 KV heads > 4096 items
     (dict(B=2, L=16384, prefill=True, qkv=None), -1),
 ])
 def test_prefill_argument_checks(lib, over, status):
@@ -110,7 +110,7 @@ def test_prefill_argument_checks(lib, over, status):
 
 def test_prefill_workspace_query_limits(lib):
     so = lib.lib()
-    assert so.gad_attn_prefill_workspace_bytes(3, 16384) == 0
+    assert so.gad_attn_prefill_workspace_bytes(5, 16384) == 0
     assert "items" in lib.last_error()
     assert so.gad_attn_prefill_workspace_bytes(1, 0) == 0
 
