@@ -29,7 +29,11 @@
 // thread per row; at an item's first tile it writes its row of Q_w into
 // tensor memory; per tile S from tensor memory, mask, online softmax with lazy
 // rescaling of O in tensor memory, P (fp16) written over the first half of
-// its S buffer.  Every
+// its S buffer.  The two warpgroups take turns on the exponentials (the MUFU
+// units they share bound the softmax): warpgroup 0 runs those of tile i,
+// then warpgroup 1 those of tile i, then warpgroup 0 those of tile i + 1, ...,
+// so each warpgroup's S load, mask and max overlap the other's exponentials.
+// Every
 // mbarrier wait is bounded; an expired wait sets the step's error word and
 // the CTA winds down, waits for its MMAs and frees its tensor memory.
 #pragma once
@@ -50,6 +54,8 @@ constexpr int RAW_ROW = 64;                  // bytes of one KV head in a cache 
 constexpr int RAW_STAGE = 2 * TK * RAW_ROW;  // 8 KB: 64 K halves then 64 V halves (E4M3)
 constexpr int F16_TILE = TK * 128;           // 64 keys x 64 fp16 = 8 KB (128-byte rows)
 constexpr int F16_BUF = 2 * F16_TILE;        // K tile then V tile: 16 KB
+constexpr int NKV = 3;                       // converted K/V buffers: the loader converts tile
+                                             // i + 1 while P.V of tile i - 1 still reads its own
 constexpr uint32_t TM_COLS = 512;            // tensor-memory columns allocated
 constexpr uint32_t TM_Q = 0;                 // Q_w at TM_Q + 32 w (fp16 pairs, 32 columns)
 constexpr uint32_t TM_S = 64;                // S_w buffer b at TM_S + 128 w + 64 b (P aliases its first 32)
@@ -58,18 +64,19 @@ constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr float RESCALE_LOG2 = 8.f;          // lazy rescale threshold (P stays <= 2^8)
 
 // mbarrier indices
-constexpr int BAR_KV_READY = 0;   // [2] converted K and V tile                      (64 loader arrivals)
-constexpr int BAR_KV_FREE = 2;    // [2] both P.V of the tile done: buffers free     (MMA commit)
-constexpr int BAR_S_FULL = 4;     // [w][2] S_w of the tile in tensor memory         (MMA commit)
-constexpr int BAR_P_FULL = 8;     // [w][2] P_w of the tile in tensor memory         (128 arrivals)
-constexpr int BAR_O_FREE = 12;    // [w] O_w read out at an item's last tile         (128 arrivals)
-constexpr int BAR_MMA_DONE = 14;  // teardown: all MMAs done                         (MMA commit)
-constexpr int BAR_Q_READY = 15;   // [w] Q_w of the item in tensor memory            (128 arrivals)
-constexpr int NBARS = 17;
+constexpr int BAR_KV_READY = 0;   // [NKV] converted K and V tile                    (64 loader arrivals)
+constexpr int BAR_KV_FREE = 3;    // [NKV] both P.V of the tile done: buffer free    (MMA commit)
+constexpr int BAR_S_FULL = 6;     // [w][2] S_w of the tile in tensor memory         (MMA commit)
+constexpr int BAR_P_FULL = 10;    // [w][2] P_w of the tile in tensor memory         (128 arrivals)
+constexpr int BAR_O_FREE = 14;    // [w] O_w read out at an item's last tile         (128 arrivals)
+constexpr int BAR_MMA_DONE = 16;  // teardown: all MMAs done                         (MMA commit)
+constexpr int BAR_Q_READY = 17;   // [w] Q_w of the item in tensor memory            (128 arrivals)
+constexpr int BAR_TURN = 19;      // [w] warpgroup w may run its exponentials        (128 arrivals)
+constexpr int NBARS = 21;
 
 template <int NS>
 struct Cfg {
-    static constexpr size_t F16_BYTES = 2 * F16_BUF;
+    static constexpr size_t F16_BYTES = NKV * F16_BUF;
     static constexpr size_t RAW_BYTES = static_cast<size_t>(NS) * RAW_STAGE;
     static constexpr int IDX_SLOTS = 2 * NS;
     static constexpr size_t IDX_BYTES = static_cast<size_t>(IDX_SLOTS) * TK * 4;
@@ -113,7 +120,7 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-    uint8_t* f16 = smem;                                     // [2][K, V][64 keys][128 B]
+    uint8_t* f16 = smem;                                     // [NKV][K, V][64 keys][128 B]
     uint8_t* raw = smem + C::F16_BYTES;                      // [NS][K halves, V halves]
     int* idx_smem = reinterpret_cast<int*>(raw + C::RAW_BYTES);
     uint8_t* ctrl = reinterpret_cast<uint8_t*>(idx_smem) + C::IDX_BYTES;
@@ -134,11 +141,14 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
     const uint32_t bar0 = smem_addr(ctrl);
     auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
     if (tid == 0) {
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NKV; ++b) {
             mbar_init(BAR(BAR_KV_READY + b), LOADERS);
             mbar_init(BAR(BAR_KV_FREE + b), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
             mbar_init(BAR(BAR_O_FREE + b), SM_THREADS);
             mbar_init(BAR(BAR_Q_READY + b), SM_THREADS);
+            mbar_init(BAR(BAR_TURN + b), SM_THREADS);
         }
         for (int i = 0; i < 4; ++i) {
             mbar_init(BAR(BAR_S_FULL + i), 1);
@@ -184,49 +194,89 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
                 prep_done = true;
             }
         };
-        auto issue_idx = [&](int tau, int b) {
-            if (tau >= t1) return;
-            const int k0 = tile_k0(tau, b);
-            int* dst = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
-            const int32_t* pt = p.page_table + static_cast<size_t>(item_ref<true>(p, b).req) * p.max_pages;
+        // A cursor over the tile list that keeps its item's data in registers:
+        // shared memory is read only when it enters a new item, and so is the
+        // item's request and KV head (integer division by a runtime value runs
+        // on the MUFU, which the softmax warps keep busy with exponentials).
+        struct Cur {
+            int tau, b, end, k0, lo, hi, rnew;
+            const int32_t* pt;  // page-table row of the item's request
+            size_t gofs;        // byte offset of KV head g in a cache row
+        };
+        auto cur_enter = [&](Cur& c) {  // c.tau and c.b set
+            c.end = tpre[c.b + 1];
+            c.lo = rlo[c.b];
+            c.hi = rhi[c.b];
+            c.rnew = rnew[c.b];
+            c.k0 = (c.lo / TK + (c.tau - tpre[c.b])) * TK;
+            const ItemRef it = item_ref<true>(p, c.b);
+            c.pt = p.page_table + static_cast<size_t>(it.req) * p.max_pages;
+            c.gofs = static_cast<size_t>(it.grp) * RAW_ROW;
+        };
+        auto cur_init = [&](Cur& c, int tau) {
+            c.tau = tau;
+            c.b = find_req(tau);
+            cur_enter(c);
+        };
+        auto cur_next = [&](Cur& c) {
+            ++c.tau;
+            c.k0 += TK;
+            if (c.tau >= c.end && c.tau < t1 && c.b < B - 1) {
+                do {
+                    ++c.b;
+                } while (c.b < B - 1 && c.tau >= tpre[c.b + 1]);
+                cur_enter(c);
+            }
+        };
+        auto issue_idx = [&](const Cur& c) {
+            if (c.tau >= t1) return;
+            int* dst = idx_smem + ((c.tau - t0) % C::IDX_SLOTS) * TK;
             if (PS == 1) {
                 if (ltid < TK) {
-                    const int k = k0 + ltid;
-                    if (k >= rlo[b] && k <= rhi[b] && k < p.max_pages) cp_async4(smem_addr(dst + ltid), pt + k);
+                    const int k = c.k0 + ltid;
+                    if (k >= c.lo && k <= c.hi && k < p.max_pages) cp_async4(smem_addr(dst + ltid), c.pt + k);
                     else dst[ltid] = -1;
                 }
             } else {
                 if (ltid < TK / PS) {
-                    const int pg = k0 / PS + ltid;
-                    if (pg < p.max_pages) cp_async4(smem_addr(dst + ltid), pt + pg);
+                    const int pg = c.k0 / PS + ltid;
+                    if (pg < p.max_pages) cp_async4(smem_addr(dst + ltid), c.pt + pg);
                     else dst[ltid] = -1;
                 }
             }
         };
-        // Tile rows: thread = row r = ltid, all 4 16-byte chunks of the 64-byte K
-        // and V halves of KV head g; raw rows are 64 bytes with chunk j stored
-        // at j ^ ((r / 2) & 3), so 8 consecutive rows cover all 32 banks.
-        auto issue_kv = [&](int tau, int b) {
-            if (tau >= t1) return;
-            const int k0 = tile_k0(tau, b);
-            if (k0 + TK - 1 >= rnew[b]) ensure_prep();
-            const int* ix = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
-            const uint32_t base = smem_addr(raw + ((tau - t0) % NS) * RAW_STAGE);
-            const int r = ltid;
-            const int k = k0 + r;
-            const int pix = PS == 1 ? ix[r] : ix[r / PS];
-            int64_t crow;
-            if (PS == 1) crow = pix;
-            else crow = pix >= 0 ? static_cast<int64_t>(pix) * PS + r % PS : -1;
-            const bool ok = k >= rlo[b] && k <= rhi[b] && crow >= 0 && crow < p.num_rows;
-            const size_t off =
-                ok ? static_cast<size_t>(crow) * ROWB + static_cast<size_t>(item_ref<true>(p, b).grp) * RAW_ROW : 0;
-            const int nbytes = ok ? 16 : 0;
+        // Tile rows: thread = (16-byte chunk j = ltid % 4, rows ltid / 4 + 16 i) of
+        // the 64-byte K and V halves of KV head g, so the 4 chunks of a half row
+        // come from consecutive lanes (8 rows per warp instruction).  Raw rows are
+        // 64 bytes with chunk j stored at j ^ ((r / 2) & 3): 8 consecutive rows
+        // cover all 32 banks for the conversion's reads.
+        auto issue_kv = [&](const Cur& c) {
+            if (c.tau >= t1) return;
+            if (c.k0 + TK - 1 >= c.rnew) ensure_prep();
+            const int* ix = idx_smem + ((c.tau - t0) % C::IDX_SLOTS) * TK;
+            const uint32_t base = smem_addr(raw + ((c.tau - t0) % NS) * RAW_STAGE);
+            const int j = ltid & 3;
+            const size_t gofs = c.gofs + j * 16;
+            constexpr int ROWS = TK * 4 / LOADERS;  // rows per thread
+            // all page-table reads first, then the copies
+            int pix[ROWS];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int i = 0; i < ROWS; ++i) {
+                const int r = (ltid >> 2) + (LOADERS / 4) * i;
+                pix[i] = PS == 1 ? ix[r] : ix[r / PS];
+            }
+#pragma unroll
+            for (int i = 0; i < ROWS; ++i) {
+                const int r = (ltid >> 2) + (LOADERS / 4) * i;
+                const int k = c.k0 + r;
+                int64_t crow;
+                if (PS == 1) crow = pix[i];
+                else crow = pix[i] >= 0 ? static_cast<int64_t>(pix[i]) * PS + r % PS : -1;
+                const bool ok = k >= c.lo && k <= c.hi && crow >= 0 && crow < p.num_rows;
+                const size_t off = ok ? static_cast<size_t>(crow) * ROWB + gofs : 0;
                 const uint32_t d = base + r * RAW_ROW + ((j ^ ((r >> 1) & 3)) << 4);
-                cp_async16(d, p.k_cache + off + j * 16, nbytes);
-                cp_async16(d + TK * RAW_ROW, p.v_cache + off + j * 16, nbytes);
+                cp_async16(d, p.k_cache + off, ok ? 16 : 0);
+                cp_async16(d + TK * RAW_ROW, p.v_cache + off, ok ? 16 : 0);
             }
         };
         // raw stage -> fp16 tiles: thread = row r of K and of V; 64 codes -> 8 fp16
@@ -257,40 +307,40 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
             }
         };
 
-        int xt = t0, xb = find_req(t0);
-        int kt = t0, kb = xb;
-        int ct = t0, cb = xb;
+        Cur xc, kc;  // page-table cursor (runs NS - 1 tiles ahead), gather cursor
+        cur_init(xc, t0);
+        kc = xc;
         for (int d = 0; d < NS - 1; ++d) {
-            issue_idx(xt, xb);
-            advance(xt, xb);
+            issue_idx(xc);
+            cur_next(xc);
         }
         cp_async_commit();
         cp_async_wait<0>();
         bar_red_or(1, LOADERS, false);
         for (int d = 0; d < NS - 1; ++d) {
-            issue_kv(kt, kb);
-            advance(kt, kb);
-            issue_idx(xt, xb);
-            advance(xt, xb);
+            issue_kv(kc);
+            cur_next(kc);
+            issue_idx(xc);
+            cur_next(xc);
             cp_async_commit();
         }
-        for (int i = 0; ct < t1; ++i) {
+        const int n_tiles = t1 - t0;
+        for (int i = 0; i < n_tiles; ++i) {
             cp_async_wait<NS - 2>();
             bool bad = false;
-            // buffers i & 1 are free once both P.V of tile i - 2 are done
-            if (i >= 2) bad = !wait_bounded(BAR(BAR_KV_FREE + (i & 1)), ((i - 2) >> 1) & 1, abort_flag);
+            // buffer i % NKV is free once both P.V of tile i - NKV are done
+            if (i >= NKV) bad = !wait_bounded(BAR(BAR_KV_FREE + i % NKV), (i / NKV - 1) & 1, abort_flag);
             // past this barrier: tile i landed for every loader, and every loader
             // has converted tile i - 1, so its raw stage may be refilled
             if (bar_red_or(1, LOADERS, bad)) break;
-            convert(i % NS, i & 1);
+            convert(i % NS, i % NKV);
             fence_proxy_async_smem();
-            mbar_arrive(BAR(BAR_KV_READY + (i & 1)));
-            issue_kv(kt, kb);
-            advance(kt, kb);
-            issue_idx(xt, xb);
-            advance(xt, xb);
+            mbar_arrive(BAR(BAR_KV_READY + i % NKV));
+            issue_kv(kc);
+            cur_next(kc);
+            issue_idx(xc);
+            cur_next(xc);
             cp_async_commit();
-            advance(ct, cb);
         }
         cp_async_wait<0>();
     }
@@ -301,7 +351,9 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
         const uint32_t f16_base = smem_addr(f16);
         // O_w += P_w(k) . V(k) for both tiles; the commit frees the tile's buffers.
         auto issue_pv = [&](int k, bool first, int seg) {
-            const uint32_t vbuf = f16_base + (k & 1) * F16_BUF + F16_TILE;
+            const uint32_t vbuf = f16_base + (k % NKV) * F16_BUF + F16_TILE;
+            const uint64_t vdesc[4] = {smem_desc_sw128(vbuf), smem_desc_sw128(vbuf + 2048),
+                                       smem_desc_sw128(vbuf + 4096), smem_desc_sw128(vbuf + 6144)};
 #pragma unroll
             for (int w = 0; w < 2; ++w) {
                 if (!wait_warp(BAR(BAR_P_FULL + 2 * w + (k & 1)), (k >> 1) & 1, abort_flag)) return false;
@@ -309,12 +361,10 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
                     return false;
                 tc_fence_after();
                 const uint32_t pa = tmem + TM_S + 128u * w + 64u * (k & 1);
-#pragma unroll
-                for (int ks = 0; ks < TK / 16; ++ks)
-                    tc_mma_ts(tmem + TM_O + 64u * w, pa + 8u * ks, smem_desc_sw128(vbuf + ks * 2048), ID_O,
-                              (ks > 0 || !first) ? 1u : 0u);
+                const uint32_t av[4] = {pa, pa + 8u, pa + 16u, pa + 24u};
+                tc_mma_ts4(tmem + TM_O + 64u * w, av, vdesc, ID_O, first ? 0u : 1u);
             }
-            tc_commit(BAR(BAR_KV_FREE + (k & 1)));
+            tc_commit(BAR(BAR_KV_FREE + k % NKV));
             return true;
         };
         int ct = t0, cb = find_req(t0);
@@ -336,12 +386,14 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
                 ok = false;
                 break;
             }
-            if (!wait_warp(BAR(BAR_KV_READY + (i & 1)), (i >> 1) & 1, abort_flag)) {
+            if (!wait_warp(BAR(BAR_KV_READY + i % NKV), (i / NKV) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t kbuf = f16_base + (i & 1) * F16_BUF;
+            const uint32_t kbuf = f16_base + (i % NKV) * F16_BUF;
+            const uint64_t kdesc[4] = {smem_desc_sw128(kbuf), smem_desc_sw128(kbuf + 32),
+                                       smem_desc_sw128(kbuf + 64), smem_desc_sw128(kbuf + 96)};
 #pragma unroll
             for (int w = 0; w < 2; ++w) {
                 if (first) {  // the item's Q_w, written by its softmax warpgroup
@@ -352,10 +404,9 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
                     tc_fence_after();
                 }
                 const uint32_t sd = tmem + TM_S + 128u * w + 64u * (i & 1);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    tc_mma_ts(sd, tmem + TM_Q + 32u * w + 8u * ks, smem_desc_sw128(kbuf + ks * 32), ID_S,
-                              ks > 0 ? 1u : 0u);
+                const uint32_t qa = tmem + TM_Q + 32u * w;
+                const uint32_t aq[4] = {qa, qa + 8u, qa + 16u, qa + 24u};
+                tc_mma_ts4(sd, aq, kdesc, ID_S, 0u);
                 tc_commit(BAR(BAR_S_FULL + 2 * w + (i & 1)));
             }
             if (!ok) break;
@@ -384,6 +435,8 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
         const uint32_t o_base = tmem + TM_O + 64u * w + lane_base;
         const uint32_t q_row = tmem + TM_Q + 32u * w + lane_base;
         bool prep_done = false;
+        // warpgroup 1 hands warpgroup 0 the first turn
+        if (w == 1) mbar_arrive(BAR(BAR_TURN + 0));
         int ct = t0, cb = find_req(t0);
         int seg_b = -1, seg_t1 = 0, k0 = 0;  // current item, end of its tiles here, tile key
         float m_run = -INFINITY, l_run = 0.f;
@@ -472,7 +525,7 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
             }
             if (__any_sync(0xffffffffu, corr)) {
                 // the P.V of tile i - 1 (same item) must be done before O is touched
-                if (!wait_warp(BAR(BAR_KV_FREE + ((i - 1) & 1)), ((i - 1) >> 1) & 1, abort_flag)) break;
+                if (!wait_warp(BAR(BAR_KV_FREE + (i - 1) % NKV), ((i - 1) / NKV) & 1, abort_flag)) break;
                 tc_fence_after();
                 const float alpha = corr ? fast_exp2((m_run - m_new) * C2) : 1.f;
                 uint32_t o[32];
@@ -493,6 +546,8 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
             const float mc = m_run == -INFINITY ? 0.f : m_run * C2;
             uint32_t pk[32];
             float l4[4] = {0.f, 0.f, 0.f, 0.f};
+            // this warpgroup's turn on the exponentials of tile i (phase i of TURN_w)
+            if (!wait_warp(BAR(BAR_TURN + w), i & 1, abort_flag)) break;
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
                 const float p0 = fast_exp2(fmaf(s[2 * c], C2, -mc));
@@ -500,6 +555,7 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
                 l4[c & 3] += p0 + p1;
                 pk[c] = pack_f16x2(p0, p1);
             }
+            mbar_arrive(BAR(BAR_TURN + (1 - w)));
             l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
             tc_st32(sbuf, pk);
             tc_wait_st();
@@ -507,7 +563,7 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
             mbar_arrive(BAR(BAR_P_FULL + 2 * w + (i & 1)));
 
             if (seg_end) {
-                if (!wait_warp(BAR(BAR_KV_FREE + (i & 1)), (i >> 1) & 1, abort_flag)) break;
+                if (!wait_warp(BAR(BAR_KV_FREE + i % NKV), (i / NKV) & 1, abort_flag)) break;
                 tc_fence_after();
                 const size_t slot = static_cast<size_t>(blockIdx.x) + cb;
                 const size_t base = (slot * p.lt + jt) * p.hp + hh;

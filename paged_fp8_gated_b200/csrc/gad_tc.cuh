@@ -99,6 +99,24 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a, uint64_t bdesc
         "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u)
         : "memory");
 }
+// Four MMAs of one K = 64 contraction (K16 steps) from one elected lane:
+// D (+)= A(a[k]) * B(b[k])^T for k = 0..3, the first accumulating into D only
+// if `accumulate` is nonzero, the other three always.  Whole warp, warp-uniform
+// operands.  One election for the four keeps the issuing warp off the
+// critical path (an election and predicate per MMA cost as much as the MMA).
+__device__ __forceinline__ void tc_mma_ts4(uint32_t d, const uint32_t (&a)[4], const uint64_t (&b)[4],
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p, e, t;\n .reg .b32 rx;\n elect.sync rx|e, 0xffffffff;\n"
+        " setp.ne.b32 p, %9, 0;\n setp.eq.b32 t, %10, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %4, {%10,%10,%10,%10}, p;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %4, {%10,%10,%10,%10}, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %4, {%10,%10,%10,%10}, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%11], %8, %4, {%10,%10,%10,%10}, t;\n}\n" ::"r"(d),
+        "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(idesc), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]),
+        "r"(accumulate), "r"(0u), "r"(a[3])
+        : "memory");
+}
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
