@@ -48,8 +48,9 @@ FALLBACK_TC_TFLOPS = 1590.0  # dense bf16/fp16 burst
 # kernel on a workload, from the ncu captures summarised in profiles/, keyed by
 # the hash of that kernel's sources when the counters were taken (null once the
 # sources change).
-TRAFFIC = {("decode32_full", "64c5ab721f0a7f48"): 474521600,
-           ("verify16_full", "9c1a1c537fa1f9f0"): 337947136}
+TRAFFIC = {("decode32_full", "ecccb345769b7cca"): 475291136,
+           ("verify16_full", "5f0d2aa17c4a40fd"): 338384640,
+           ("prefill1_full", "e507e97fc090faf7"): 22618624}
 
 # Sources of the step's main kernel: decode_kernel for single-token steps,
 # verify_tc_kernel for verify blocks, prefill_tc_kernel for longer blocks (the
