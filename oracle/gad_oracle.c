@@ -40,6 +40,9 @@
  *     (round to nearest even, saturating to +-448, NaN kept).
  *   - All of the step's cache writes happen before any attention read.
  *
+ * The file also holds the output projection that follows the step in the
+ * decoder layer (gado_oproj, at the end).
+ *
  * Parity pins: tests/test_oracle_pins.py checks every function here against
  * closed forms, library routines and invariants that do not come from this
  * file.
@@ -414,3 +417,79 @@ int gado_attn_decode(const uint16_t* qkv, const int64_t* positions, const int32_
                                   v_scale, B, L, GADO_HQ, GADO_HKV, max_pages, num_rows, page_size,
                                   window, use_rope, want, out, out_exact, attn_out, nthreads);
 }
+
+/* ------------------------------------------------------------------------- */
+/* Output projection                                                          */
+/* ------------------------------------------------------------------------- */
+
+typedef struct {
+    const uint16_t *out, *o;
+    int T, K, N;
+    uint16_t* a;
+    double* a_exact;
+    int tid, nthreads;
+} gado_oproj_job;
+
+static void* gado_oproj_worker(void* arg) {
+    gado_oproj_job* J = (gado_oproj_job*)arg;
+    for (int n = J->tid; n < J->N; n += J->nthreads) {
+        const uint16_t* orow = J->o + (int64_t)n * J->K;
+        for (int t = 0; t < J->T; ++t) {
+            const uint16_t* xrow = J->out + (int64_t)t * J->K;
+            double acc = 0.0;
+            for (int k = 0; k < J->K; ++k) acc += gado_bf16_decode(xrow[k]) * gado_bf16_decode(orow[k]);
+            const int64_t i = (int64_t)t * J->N + n;
+            J->a[i] = gado_bf16_encode(acc);
+            if (J->a_exact) J->a_exact[i] = acc;
+        }
+    }
+    return NULL;
+}
+
+/*
+ * The projection that follows the attention in the decoder layer (the pages
+ * "Decode layer (muse_decode_layer)" and "Prefill layer (muse_prefill_layer)",
+ * section "What to compute": a = (rmsnorm(attention(q)) * sigmoid(g)) @ o.T,
+ * the all-reduce after it being the identity on one GPU):
+ *   a[t][n] = sum_k out[t][k] * o[n][k]
+ * in double, k in index order, then one rounding to bf16.
+ *   out      bf16 bits [T, K]  the attention step's output
+ *   o        bf16 bits [N, K]  the projection weight (row n = hidden unit n)
+ *   a        bf16 bits [T, N]
+ *   a_exact  [T, N] or NULL: before the bf16 rounding
+ * Returns 0, or GADO_ERR_ARG / GADO_ERR_NOMEM.
+ */
+int gado_oproj(const uint16_t* out, const uint16_t* o, int T, int K, int N, uint16_t* a,
+               double* a_exact, int nthreads) {
+    if (T <= 0 || K <= 0 || N <= 0 || !out || !o || !a) return GADO_ERR_ARG;
+    if (nthreads < 1) nthreads = 1;
+    gado_oproj_job* jobs = (gado_oproj_job*)calloc((size_t)nthreads, sizeof(gado_oproj_job));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) {
+        free(jobs);
+        free(th);
+        return GADO_ERR_NOMEM;
+    }
+    for (int i = 0; i < nthreads; ++i) {
+        gado_oproj_job* J = &jobs[i];
+        J->out = out;
+        J->o = o;
+        J->T = T;
+        J->K = K;
+        J->N = N;
+        J->a = a;
+        J->a_exact = a_exact;
+        J->tid = i;
+        J->nthreads = nthreads;
+    }
+    if (nthreads == 1) {
+        gado_oproj_worker(&jobs[0]);
+    } else {
+        for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, gado_oproj_worker, &jobs[i]);
+        for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    }
+    free(jobs);
+    free(th);
+    return GADO_OK;
+}
+

@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
             vp, vp, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp,
             ctypes.c_int]
+        L.gado_oproj.restype = ctypes.c_int
+        L.gado_oproj.argtypes = [vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, ctypes.c_int]
         L.gado_attn_decode_heads.restype = ctypes.c_int
         L.gado_attn_decode_heads.argtypes = [
             vp, vp, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float, ctypes.c_int, ctypes.c_int,
@@ -170,6 +172,26 @@ def attn_decode(qkv_bits, positions, page_table, cache_loc, k_cache, v_cache, k_
     if st != 0:
         raise RuntimeError(f"oracle gado_attn_decode failed with status {st}")
     return OracleResult(out, out_exact, attn, kc, vc)
+
+
+def oproj(out_bits, o_bits, nthreads: int | None = None) -> tuple[np.ndarray, np.ndarray]:
+    """The output projection a = out @ o^T (bf16 in, double sum, one bf16
+    rounding).  out_bits: uint16 [T, K]; o_bits: uint16 [N, K].  Returns
+    (a bits uint16 [T, N], a before rounding float64 [T, N])."""
+    x = _np(out_bits, np.uint16)
+    w = _np(o_bits, np.uint16)
+    T, K = x.shape
+    N, K2 = w.shape
+    assert K == K2
+    a = np.zeros((T, N), np.uint16)
+    a_exact = np.zeros((T, N), np.float64)
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    vp = lambda arr: arr.ctypes.data_as(ctypes.c_void_p)
+    st = lib().gado_oproj(vp(x), vp(w), T, K, N, vp(a), vp(a_exact), int(nthreads))
+    if st != 0:
+        raise RuntimeError(f"oracle gado_oproj failed with status {st}")
+    return a, a_exact
 
 
 def bf16_bits_to_float(bits: np.ndarray) -> np.ndarray:

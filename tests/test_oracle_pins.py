@@ -468,6 +468,54 @@ def test_heads_dp_gate_columns():
 
 
 # ----------------------------------------------------------------------------
+# Output projection a = out @ o^T (decoder-layer pages, "What to compute")
+# ----------------------------------------------------------------------------
+
+def test_oproj_matches_numpy_matmul():
+    """Against numpy's float64 matmul of the decoded bf16 values (a library
+    routine, not the oracle's loop), and bf16 of that."""
+    rng = np.random.default_rng(31)
+    x = _bf16_bits(rng.normal(size=(5, 96)))
+    w = _bf16_bits(rng.normal(size=(40, 96)) / 10)
+    a, a_exact = O.oproj(x, w, nthreads=3)
+    ref = O.bf16_bits_to_float(x) @ O.bf16_bits_to_float(w).T
+    assert np.allclose(a_exact, ref, rtol=1e-12, atol=1e-13)
+    assert np.array_equal(a, np.array([[O.bf16_encode(v) for v in row] for row in a_exact], np.uint16))
+
+
+def test_oproj_selection_rows_copy_inputs():
+    """Row n of o selects input column n % K (scaled by 2^-j, exact in bf16):
+    a[t][n] = out[t][n % K] * 2^-(n % 3), bit for bit."""
+    rng = np.random.default_rng(32)
+    K, N = 64, 160
+    x = _bf16_bits(rng.normal(size=(3, K)))
+    wf = np.zeros((N, K), np.float32)
+    for n in range(N):
+        wf[n, n % K] = 2.0 ** -(n % 3)
+    a, _ = O.oproj(x, _bf16_bits(wf), nthreads=2)
+    xv = O.bf16_bits_to_float(x)
+    want = np.stack([xv[:, n % K] * 2.0 ** -(n % 3) for n in range(N)], axis=1)
+    assert np.array_equal(O.bf16_bits_to_float(a), want)
+
+
+def test_oproj_sign_and_transpose():
+    """Negating o negates a; swapping two rows of o swaps the two columns of a
+    (a wrong operand order or a transposed weight fails one of these)."""
+    rng = np.random.default_rng(33)
+    x = _bf16_bits(rng.normal(size=(4, 32)))
+    wf = rng.normal(size=(24, 32)).astype(np.float32)
+    _, e0 = O.oproj(x, _bf16_bits(wf))
+    _, e1 = O.oproj(x, _bf16_bits(-wf))
+    assert np.array_equal(e1, -e0)
+    ws = wf.copy()
+    ws[[3, 17]] = ws[[17, 3]]
+    _, e2 = O.oproj(x, _bf16_bits(ws))
+    assert np.array_equal(e2[:, [3, 17]], e0[:, [17, 3]])
+    # a non-square case where out @ o (no transpose) would not even be defined
+    assert e0.shape == (4, 24)
+
+
+# ----------------------------------------------------------------------------
 # The page's own numbers: the floor column of the load table
 # ----------------------------------------------------------------------------
 
