@@ -321,6 +321,105 @@ def run_suite(args):
     print(json.dumps(line), flush=True)
 
 
+def run_oproj(args):
+    """The output projection a = out @ o^T after the step (decoder-layer pages,
+    "What to compute"): the projection kernel alone (CUDA events, cold L2,
+    against its roofline: the weight stream or the tensor peak, whichever is
+    longer) and the step with the projection chained to it (graph replay)
+    against the step alone.  One JSON line."""
+    import torch
+    from paged_fp8_gated_b200 import binding
+    from paged_fp8_gated_b200 import workloads as W
+
+    dev = torch.device("cuda", 0)
+    peaks = measured_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sink = torch.empty((), dtype=torch.int64, device=dev)
+
+    def cold():
+        flush.fill_(1)
+        torch.sum(flush.view(torch.int64), dim=0, out=sink)
+
+    w = W.oproj_weight().to(dev)
+    N, K = w.shape
+    rows = []
+    for name in ("decode32_full", "verify16_full", "prefill1_full"):
+        inp = W.make_inputs(W.named(name))
+        B, L = inp["B"], inp["L"]
+        T = B * L
+        d = {k: inp[k].to(dev) for k in ("qkv", "positions", "seq_lens", "page_table", "cache_loc",
+                                           "k_cache", "v_cache")}
+        ks = torch.tensor([inp["k_scale"]], dtype=torch.float32, device=dev)
+        vs = torch.tensor([inp["v_scale"]], dtype=torch.float32, device=dev)
+        out = torch.empty(B, L, 1024, dtype=torch.bfloat16, device=dev)
+        a = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
+        ws = binding.alloc_workspace(B, L, dev)
+
+        def step():
+            binding.attn_decode(d["qkv"], d["positions"], d["seq_lens"], d["page_table"], d["cache_loc"],
+                                d["k_cache"], d["v_cache"], ks, vs, inp["page_size"], inp["window"],
+                                inp["use_rope"], L=L, out=out, workspace=ws)
+
+        def fused():
+            binding.attn_decode_oproj(d["qkv"], d["positions"], d["seq_lens"], d["page_table"],
+                                      d["cache_loc"], d["k_cache"], d["v_cache"], ks, vs, inp["page_size"],
+                                      inp["window"], inp["use_rope"], w, L=L, out=out, a=a, workspace=ws)
+
+        def proj():
+            binding.oproj(out.view(T, 1024), w, a)
+
+        def timed(fn, graph: bool):
+            if graph:
+                side = torch.cuda.Stream(dev)
+                side.wait_stream(torch.cuda.current_stream(dev))
+                with torch.cuda.stream(side):
+                    fn()
+                side.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    fn()
+                torch.cuda.synchronize(dev)
+                run = g.replay
+            else:
+                run = fn
+            for _ in range(args.warmup):
+                cold()
+                run()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for e0, e1 in evs:
+                cold()
+                e0.record()
+                run()
+                e1.record()
+            torch.cuda.synchronize(dev)
+            return statistics.median(e0.elapsed_time(e1) * 1e3 for e0, e1 in evs)
+
+        step_us = timed(step, True)
+        fused_us = timed(fused, True)
+        proj_us = timed(proj, True)
+        bytes_ = N * K * 2 + T * K * 2 + T * N * 2
+        flops = 2.0 * T * N * K
+        t_mem = bytes_ / (peaks["hbm_gbs"] * 1e9) * 1e6
+        t_tc = flops / (peaks["tc_tflops"] * 1e12) * 1e6
+        bound = "hbm" if t_mem >= t_tc else "tensor"
+        rows.append({"workload": name, "T": T, "proj_us": round(proj_us, 2), "bound": bound,
+                     "roofline_us": round(max(t_mem, t_tc), 2),
+                     "frac": round(max(t_mem, t_tc) / proj_us, 4),
+                     "achieved_gbs": round(bytes_ / (proj_us * 1e-6) / 1e9, 1),
+                     "achieved_tflops": round(flops / (proj_us * 1e-6) / 1e12, 1),
+                     "step_us": round(step_us, 2), "step_plus_proj_us": round(fused_us, 2),
+                     "added_us": round(fused_us - step_us, 2)})
+        del d, out, a, ws
+        torch.cuda.empty_cache()
+    line = {"metric": "output projection a = out @ o^T after the step: kernel time vs roofline, and the "
+                      "step with the projection chained (PDL) vs the step alone",
+            "unit": "us", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "data": "synthetic",
+            "weights": f"bf16 [{N}, {K}] N(0, 1/{K})", "peak_hbm_gbs": peaks["hbm_gbs"],
+            "peak_tc_tflops": peaks["tc_tflops"], "peak_source": peaks["source"], "loads": rows}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -331,11 +430,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--suite", action="store_true",
                     help="time the page's twelve scored loads instead (one GPU, one JSON line)")
+    ap.add_argument("--oproj", action="store_true",
+                    help="time the output projection after the step instead (one GPU, one JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.suite:
         run_suite(args)
+        return
+    if args.oproj:
+        run_oproj(args)
         return
 
     from paged_fp8_gated_b200 import replicas

@@ -51,6 +51,8 @@ extern "C" {
 #define GAD_MAX_B 4096     /* most requests in one call; also the most
                               work items (request, token chunk, heads)    */
 #define GAD_MAX_PREFILL_L 65536 /* longest block of gad_attn_prefill */
+#define GAD_HIDDEN 8192    /* decoder hidden size: rows of the o-projection weight */
+#define GAD_MAX_OPROJ_T 262144 /* most tokens in one projection call */
 #define GAD_NOALLOC_SCRATCH_BYTES (16u << 20) /* built-in scratch of gad_attn_decode_noalloc */
 
 /* Return codes (0 = success). */
@@ -216,6 +218,44 @@ int gad_attn_prefill_timed(const void* qkv, const int64_t* positions, const int3
                            int L, int max_pages, int64_t num_rows, int page_size, int window,
                            int use_rope, void* out, void* workspace, size_t workspace_bytes,
                            void* stream, void* const* events);
+
+/*
+ * Output projection that follows the attention in the decoder layer (the
+ * pages "Decode layer (muse_decode_layer)" and "Prefill layer
+ * (muse_prefill_layer)", section "What to compute":
+ * a = (rmsnorm(attention(q)) * sigmoid(g)) @ o.T, its all-reduce being the
+ * identity on one GPU):
+ *
+ *   a[t][n] = sum_k out[t][k] * o_weight[n][k]     fp32 accumulation, bf16 a
+ *
+ *   out       bf16 [T, K] row-major (the attention step's output: K = 1024)
+ *   o_weight  bf16 [N, K] row-major (N = GAD_HIDDEN for the decoder layer)
+ *   a         bf16 [T, N] row-major, written
+ *   K a positive multiple of 64, N a positive multiple of 128, 1 <= T <=
+ *   GAD_MAX_OPROJ_T; all three pointers 16-byte aligned (GAD_ERR_SHAPE,
+ *   GAD_ERR_ALIGN, GAD_ERR_NULL otherwise, checked before any launch).
+ * One hand-written tcgen05 kernel (TMA-staged operands, accumulator in tensor
+ * memory); asynchronous on `stream`, allocates nothing, graph-capturable.
+ */
+int gad_oproj(const void* out, const void* o_weight, void* a, int T, int K, int N, void* stream);
+
+/*
+ * The attention step followed by its output projection in one call:
+ * gad_attn_decode's step (or gad_attn_prefill's for L > GAD_MAX_L; any
+ * 1 <= L <= GAD_MAX_PREFILL_L), writing `out` as they do, then
+ * a = out @ o_weight^T as in gad_oproj with K = 1024 and N = hidden.  The
+ * projection kernel is chained to the step's last kernel by programmatic
+ * dependent launch: its first weight tiles load while the step finishes.
+ * workspace: gad_attn_prefill_workspace_bytes(B, L) bytes (which equals
+ * gad_attn_workspace_bytes(B, L) for L <= GAD_MAX_L).  Arguments and errors
+ * as gad_attn_decode and gad_oproj.
+ */
+int gad_attn_decode_oproj(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                          const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,
+                          uint8_t* v_cache, const float* k_scale, const float* v_scale, int B, int L,
+                          int max_pages, int64_t num_rows, int page_size, int window, int use_rope,
+                          void* out, void* workspace, size_t workspace_bytes, const void* o_weight,
+                          int hidden, void* a, void* stream);
 
 /*
  * Allocation-free variant of gad_attn_decode.  The page has no counterpart:

@@ -46,6 +46,11 @@ _lib.gad_attn_prefill_workspace_bytes.restype = ctypes.c_size_t
 _lib.gad_attn_prefill_workspace_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
 _lib.gad_attn_prefill_timed.restype = ctypes.c_int
 _lib.gad_attn_prefill_timed.argtypes = list(_lib.gad_attn_decode.argtypes) + [_vp]
+_lib.gad_oproj.restype = ctypes.c_int
+_lib.gad_oproj.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp]
+_lib.gad_attn_decode_oproj.restype = ctypes.c_int
+_lib.gad_attn_decode_oproj.argtypes = (list(_lib.gad_attn_decode.argtypes[:19])
+                                       + [_vp, ctypes.c_int, _vp, _vp])  # o_weight, hidden, a, stream
 _lib.gad_attn_decode_timed.restype = ctypes.c_int
 _lib.gad_attn_decode_timed.argtypes = list(_lib.gad_attn_decode.argtypes) + [_vp]
 _lib.gad_attn_decode_noalloc.restype = ctypes.c_int
@@ -58,10 +63,11 @@ _lib.gad_status_string.argtypes = [ctypes.c_int]
 HQ, HKV, D = 16, 2, 64
 QKV_COLS, OUT_COLS, ROW_BYTES = 2304, 1024, 128
 MAX_L, MAX_PREFILL_L = 8, 65536
+HIDDEN = 8192
 
 EXPORTED = ("gad_attn_decode", "gad_attn_decode_heads", "gad_attn_decode_timed",
             "gad_attn_decode_heads_timed", "gad_attn_prefill", "gad_attn_prefill_timed",
-            "gad_attn_prefill_workspace_bytes",
+            "gad_attn_prefill_workspace_bytes", "gad_oproj", "gad_attn_decode_oproj",
             "gad_attn_decode_noalloc", "gad_attn_workspace_bytes",
             "gad_attn_workspace_bytes_heads", "gad_last_error", "gad_status_string")
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -227,6 +233,69 @@ def attn_decode_noalloc(qkv: torch.Tensor, positions: torch.Tensor,
     if st != 0:
         raise GadError(st, "gad_attn_decode_noalloc")
     return out
+
+
+def oproj(out: torch.Tensor, o_weight: torch.Tensor, a: torch.Tensor | None = None,
+          stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """a = out @ o_weight^T through gad_oproj: out bf16 [T, K], o_weight bf16 [N, K]
+    (both CUDA, contiguous); returns a bf16 [T, N]."""
+    _need(out, "out", torch.bfloat16)
+    _need(o_weight, "o_weight", torch.bfloat16, 2)
+    K = out.shape[-1]
+    T = out.numel() // K
+    N = o_weight.shape[0]
+    if o_weight.shape[1] != K:
+        raise ValueError(f"o_weight must be [N, {K}], got {tuple(o_weight.shape)}")
+    if a is None:
+        a = torch.empty(T, N, dtype=torch.bfloat16, device=out.device)
+    else:
+        _need(a, "a", torch.bfloat16)
+        if a.numel() != T * N:
+            raise ValueError(f"a must hold {T}x{N} values")
+    s = (stream or torch.cuda.current_stream(out.device)).cuda_stream
+    st = _lib.gad_oproj(_ptr(out), _ptr(o_weight), _ptr(a), int(T), int(K), int(N), ctypes.c_void_p(s))
+    if st != 0:
+        raise GadError(st, "gad_oproj")
+    return a
+
+
+def attn_decode_oproj(qkv, positions, seq_lens, page_table, cache_loc, k_cache, v_cache, k_scale,
+                      v_scale, page_size: int, window: int, use_rope: bool, o_weight: torch.Tensor,
+                      L: int = 1, out: torch.Tensor | None = None, a: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None,
+                      stream: torch.cuda.Stream | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """The step and its output projection in one call (gad_attn_decode_oproj);
+    returns (out bf16 [B, L, 1024], a bf16 [B * L, hidden])."""
+    for t, n, dt in ((qkv, "qkv", torch.bfloat16), (positions, "positions", torch.int64),
+                     (page_table, "page_table", torch.int32), (cache_loc, "cache_loc", torch.int64),
+                     (k_cache, "k_cache", torch.uint8), (v_cache, "v_cache", torch.uint8),
+                     (k_scale, "k_scale", torch.float32), (v_scale, "v_scale", torch.float32)):
+        _need(t, n, dt)
+    _need(o_weight, "o_weight", torch.bfloat16, 2)
+    B, max_pages = page_table.shape
+    T = qkv.shape[0]
+    if qkv.shape[1] != QKV_COLS or T != B * L:
+        raise ValueError(f"qkv must be [B*L={B * L}, {QKV_COLS}], got {tuple(qkv.shape)}")
+    hidden = o_weight.shape[0]
+    num_rows = k_cache.numel() // ROW_BYTES
+    if out is None:
+        out = torch.empty(B, L, OUT_COLS, dtype=torch.bfloat16, device=qkv.device)
+    if a is None:
+        a = torch.empty(T, hidden, dtype=torch.bfloat16, device=qkv.device)
+    if workspace is None:
+        n = _lib.gad_attn_prefill_workspace_bytes(int(B), int(L))
+        if n == 0:
+            raise GadError(-2, "gad_attn_prefill_workspace_bytes")
+        workspace = torch.empty(int(n), dtype=torch.uint8, device=qkv.device)
+    s = (stream or torch.cuda.current_stream(qkv.device)).cuda_stream
+    st = _lib.gad_attn_decode_oproj(
+        _ptr(qkv), _ptr(positions), _ptr(seq_lens), _ptr(page_table), _ptr(cache_loc), _ptr(k_cache),
+        _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), int(B), int(L), int(max_pages), int(num_rows),
+        int(page_size), int(window), int(bool(use_rope)), _ptr(out), _ptr(workspace),
+        int(workspace.numel()), _ptr(o_weight), int(hidden), _ptr(a), ctypes.c_void_p(s))
+    if st != 0:
+        raise GadError(st, "gad_attn_decode_oproj")
+    return out, a
 
 
 def raw_call(**kw) -> int:

@@ -8,6 +8,8 @@
 // at 76.6% (page size 1) / 78.8% (page size 64) of the measured HBM copy rate;
 // a warp-specialised variant with one producer warp issuing 2D TMA page loads
 // reached 64%, and producer-warp cp.async gathers about 55%.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -17,7 +19,9 @@
 #include <string>
 
 #include "gad_attn.h"
+#include "gad_combine.cuh"
 #include "gad_kernels.cuh"
+#include "gad_oproj.cuh"
 #include "gad_prefill_tc.cuh"
 #include "gad_verify_tc.cuh"
 
@@ -295,6 +299,100 @@ int launch_block(const gad::StepParams& prm, int page_size, bool deep, int sms, 
                 : launch_verify_tc<64, kVtcShallowStages, MULTI>(prm, sms, tiles_upper, s, pdl);
 }
 
+// ---------------------------------------------------------------------------
+// Output projection a = out @ o^T (oproj_kernel)
+// ---------------------------------------------------------------------------
+// Error word of the projection kernel (a bounded wait timed out); the
+// standalone entry point has no workspace to hold it.
+__device__ int g_oproj_err;
+
+int encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                   uint32_t box_outer) {
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> encode{nullptr};
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode.load(std::memory_order_acquire);
+    if (fn == nullptr) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || f == nullptr)
+            return fail(GAD_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+        encode.store(fn, std::memory_order_release);
+    }
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(GAD_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return GAD_OK;
+}
+
+int check_oproj(const void* out, const void* w, const void* a, int T, int K, int N) {
+    if (!out || !w || !a) return fail(GAD_ERR_NULL, "out, o_weight and a must be non-NULL");
+    if (T < 1 || T > GAD_MAX_OPROJ_T) return fail(GAD_ERR_SHAPE, "T=%d not in [1,%d]", T, GAD_MAX_OPROJ_T);
+    if (K < gad::opj::BK || K % gad::opj::BK != 0 || K > 65536)
+        return fail(GAD_ERR_SHAPE, "K=%d must be a positive multiple of %d (at most 65536)", K, gad::opj::BK);
+    if (N < gad::opj::BM || N % gad::opj::BM != 0 || N > 65536 * gad::opj::BM)
+        return fail(GAD_ERR_SHAPE, "N=%d must be a positive multiple of %d", N, gad::opj::BM);
+    if (!aligned(out, 16) || !aligned(w, 16) || !aligned(a, 16))
+        return fail(GAD_ERR_ALIGN, "out, o_weight and a must be 16-byte aligned");
+    return GAD_OK;
+}
+
+int launch_oproj(const void* out, const void* w, void* a, int T, int K, int N, cudaStream_t s, bool pdl) {
+    const int tt = T >= gad::opj::TT_MAX ? gad::opj::TT_MAX : (T + 15) / 16 * 16;
+    const int nstg = gad::opj::stages(tt, K / gad::opj::BK);
+    const size_t smem = gad::opj::smem_bytes(tt, nstg);
+    static std::atomic<bool> attr_done[kMaxDevices];
+    static std::atomic<void*> err_addr[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", dev);
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(gad::oproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(1024 + gad::opj::SMEM_BUDGET + gad::opj::ctrl_bytes()));
+        if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        void* ea = nullptr;
+        e = cudaGetSymbolAddress(&ea, g_oproj_err);
+        if (e != cudaSuccess || ea == nullptr)
+            return fail(GAD_ERR_CUDA, "cudaGetSymbolAddress(error word): %s", cudaGetErrorString(e));
+        err_addr[dev].store(ea, std::memory_order_release);
+        attr_done[dev].store(true, std::memory_order_release);
+    }
+    CUtensorMap wmap, xmap;
+    int st = encode_bf16_2d(&wmap, w, static_cast<uint64_t>(K), static_cast<uint64_t>(N), gad::opj::BK,
+                            gad::opj::BM);
+    if (st != GAD_OK) return st;
+    st = encode_bf16_2d(&xmap, out, static_cast<uint64_t>(K), static_cast<uint64_t>(T), gad::opj::BK,
+                        static_cast<uint32_t>(tt));
+    if (st != GAD_OK) return st;
+    gad::OprojParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.a = static_cast<__nv_bfloat16*>(a);
+    prm.T = T;
+    prm.K = K;
+    prm.N = N;
+    prm.tt = tt;
+    prm.nstg = nstg;
+    prm.err = static_cast<int*>(err_addr[dev].load(std::memory_order_acquire));
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(N / gad::opj::BM), static_cast<unsigned>((T + tt - 1) / tt));
+    cfg.blockDim = dim3(gad::opj::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr = pdl_attr();
+    cfg.attrs = &attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, gad::oproj_kernel, wmap, xmap, prm);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "projection launch: %s", cudaGetErrorString(e));
+    return GAD_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -519,6 +617,31 @@ int gad_attn_decode_heads_timed(const void* qkv, const int64_t* positions,
                     L, GAD_MAX_L, hq, hkv, max_pages, num_rows, page_size, window, use_rope, out,
                     workspace,
                     workspace_bytes, stream, events);
+}
+
+int gad_oproj(const void* out, const void* o_weight, void* a, int T, int K, int N, void* stream) {
+    const int st = check_oproj(out, o_weight, a, T, K, N);
+    if (st != GAD_OK) return st;
+    return launch_oproj(out, o_weight, a, T, K, N, static_cast<cudaStream_t>(stream), false);
+}
+
+int gad_attn_decode_oproj(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
+                          const int32_t* page_table, const int64_t* cache_loc, uint8_t* k_cache,
+                          uint8_t* v_cache, const float* k_scale, const float* v_scale, int B, int L,
+                          int max_pages, int64_t num_rows, int page_size, int window, int use_rope,
+                          void* out, void* workspace, size_t workspace_bytes, const void* o_weight,
+                          int hidden, void* a, void* stream) {
+    (void)seq_lens;
+    if (L < 1 || L > GAD_MAX_PREFILL_L) return fail(GAD_ERR_SHAPE, "L=%d not in [1,%d]", L, GAD_MAX_PREFILL_L);
+    if (B < 1 || B > GAD_MAX_B) return fail(GAD_ERR_SHAPE, "B=%d not in [1,%d]", B, GAD_MAX_B);
+    int st = check_oproj(out, o_weight, a, B * L, GAD_OUT_COLS, hidden);
+    if (st != GAD_OK) return st;
+    st = run_step(qkv, positions, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale, B, L,
+                  GAD_MAX_PREFILL_L, GAD_HQ, GAD_HKV, max_pages, num_rows, page_size, window, use_rope,
+                  out, workspace, workspace_bytes, stream, nullptr);
+    if (st != GAD_OK) return st;
+    return launch_oproj(out, o_weight, a, B * L, GAD_OUT_COLS, hidden, static_cast<cudaStream_t>(stream),
+                        true);
 }
 
 int gad_attn_prefill(const void* qkv, const int64_t* positions, const int32_t* seq_lens,

@@ -158,11 +158,48 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
     return d;
 }
 
+// mbarrier arrive that also expects `bytes` of asynchronous (TMA) transactions.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+// 2D TMA tile load global -> shared (this CTA only, no multicast), completion
+// counted in bytes on `bar`.  x is the inner coordinate in elements.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Four MMAs of a K = 64 contraction with both operands in shared memory:
+// D (+)= A(a[k]) * B(b[k])^T for k = 0..3, the first accumulating only if
+// `accumulate` is nonzero.  Whole warp, one elected lane issues.
+__device__ __forceinline__ void tc_mma_ss4(uint32_t d, const uint64_t (&a)[4], const uint64_t (&b)[4],
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p, e, t;\n .reg .b32 rx;\n elect.sync rx|e, 0xffffffff;\n"
+        " setp.ne.b32 p, %10, 0;\n setp.eq.b32 t, %11, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %9, {%11,%11,%11,%11}, p;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %9, {%11,%11,%11,%11}, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %9, {%11,%11,%11,%11}, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %9, {%11,%11,%11,%11}, t;\n}\n" ::"r"(d),
+        "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]),
+        "r"(idesc), "r"(accumulate), "r"(0u)
+        : "memory");
+}
+
 // Instruction descriptor, kind::f16: fp16 A and B, fp32 D, A K-major,
 // B K-major (b_mn = 0) or MN-major (b_mn = 1), shape M x N.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int b_mn) {
     return (1u << 4) | (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);
+}
+// The same with bf16 A and B (A and B format fields = 1).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn) {
+    return idesc_f16_f32(M, N, b_mn) | (1u << 7) | (1u << 10);
 }
 
 }  // namespace gad

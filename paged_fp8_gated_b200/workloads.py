@@ -186,6 +186,23 @@ def make_inputs(spec: Spec) -> dict:
     )
 
 
+def oproj_weight(seed: int = 7, hidden: int = 8192, k: int = HQ * D) -> torch.Tensor:
+    """The decoder layer's output-projection weight o [hidden, k] as seeded
+    synthetic bf16 values N(0, 1/k) (the usual fan-in scale; no trained weights
+    are available)."""
+    gen = torch.Generator().manual_seed(int(seed))
+    return (torch.randn(hidden, k, generator=gen) / k ** 0.5).to(torch.bfloat16)
+
+
+def oproj_input(T: int, seed: int = 8, k: int = HQ * D) -> torch.Tensor:
+    """A stand-in for the attention step's output [T, k]: bf16 rows shaped
+    like rmsnorm(a) * sigmoid(gate) (unit-RMS rows times sigmoids of N(0,1))."""
+    gen = torch.Generator().manual_seed(int(seed))
+    x = _unit_rms(torch.randn(T, k // D, D, generator=gen))
+    g = torch.sigmoid(torch.randn(T, k // D, D, generator=gen))
+    return (x * g).reshape(T, k).to(torch.bfloat16)
+
+
 def keys_attended(inp: dict) -> int:
     """Distinct cache rows the step reads: sum over requests of the union of
     its tokens' key ranges (full: p_last + 1; sliding: at most W + L - 1)."""

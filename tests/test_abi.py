@@ -122,6 +122,21 @@ def test_heads_workspace_query_rejects_bad_heads(lib):
     assert so.gad_attn_workspace_bytes_heads(600, 8, 128, 16) == 0
 
 
+@pytest.mark.parametrize("T,K,N,out,status", [
+    (0, 1024, 8192, FAKE, -2),
+    (4, 1000, 8192, FAKE, -2),     # K not a multiple of 64
+    (4, 1024, 8000, FAKE, -2),     # N not a multiple of 128
+    (4, 1024, 8192, None, -1),
+    (4, 1024, 8192, FAKE + 8, -3),
+])
+def test_oproj_argument_checks(lib, T, K, N, out, status):
+    so = lib.lib()
+    args = [None if out is None else ctypes.c_void_p(out), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE),
+            T, K, N, None]
+    assert so.gad_oproj(*args) == status
+    assert lib.last_error()
+
+
 def test_binding_rejects_cpu_tensors(lib):
     import torch
     x = torch.zeros(1, 2304, dtype=torch.bfloat16)
