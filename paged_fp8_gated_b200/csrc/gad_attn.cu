@@ -13,6 +13,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -487,6 +488,16 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     prm.max_pages = max_pages;
     prm.window = window;
     prm.use_rope = use_rope ? 1 : 0;
+    {
+        // RoPE frequencies theta^(-2i/64), theta = 10000, once per process
+        static const struct Freqs {
+            double v[gad::HD / 2];
+            Freqs() {
+                for (int i = 0; i < gad::HD / 2; ++i) v[i] = std::pow(10000.0, -2.0 * i / 64.0);
+            }
+        } freqs;
+        std::memcpy(prm.inv_freq, freqs.v, sizeof(prm.inv_freq));
+    }
     prm.num_rows = num_rows;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     prm.q_ws = reinterpret_cast<__half*>(ws + w.q_off);

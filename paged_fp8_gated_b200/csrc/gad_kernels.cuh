@@ -72,6 +72,7 @@ struct StepParams {
     float* part_o;   // [slots][lt][16][64]  un-normalised partial outputs (slot = CTA + item)
     float* part_ml;  // [slots][lt][16][2]   (running max in log2 units, sum)
     int* meta;       // see META_*: tile count, tiles per CTA, error word, tile prefix over items
+    double inv_freq[HD / 2];  // RoPE: 10000^(-2i/64) for pair i, computed on the host
     int lt;          // token capacity of one partial slot (1 or 8)
     int tl;          // partials per (CTA, request) and KV-head group
 };
@@ -145,9 +146,9 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) 
     }
     if (p.use_rope) {
         const double pos = static_cast<double>(p.positions[t]);
-        const double inv_freq = pow(10000.0, -2.0 * lane / 64.0);
-        const double phi = __dmul_rn(pos, inv_freq);
-        const double c = cos(phi), s = sin(phi);
+        const double phi = __dmul_rn(pos, p.inv_freq[lane]);
+        double s, c;
+        sincos(phi, &s, &c);
         const double r0 = __dsub_rn(__dmul_rn(u0, c), __dmul_rn(u1, s));
         const double r1 = __dadd_rn(__dmul_rn(u1, c), __dmul_rn(u0, s));
         u0 = r0;
