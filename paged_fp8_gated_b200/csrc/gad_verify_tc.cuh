@@ -187,34 +187,65 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 prep_done = true;
             }
         };
-        auto issue_idx = [&](int tau, int b) {
-            if (tau >= t1) return;
-            const int k0 = tile_k0(tau, b);
-            int* dst = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
-            const int32_t* pt = p.page_table + static_cast<size_t>(item_ref<MULTI>(p, b).req) * p.max_pages;
+        // A cursor over the tile list that keeps its item's data in registers:
+        // shared memory is read only when it enters a new item (a chain of
+        // dependent shared-memory reads per tile slowed the loaders).
+        struct Cur {
+            int tau, b, end, k0, lo, hi, rnew;
+            const int32_t* pt;  // page-table row of the item's request
+            size_t gofs;        // byte offset of the item's head group in a cache row
+        };
+        auto cur_enter = [&](Cur& c) {  // c.tau and c.b set
+            c.end = tpre[c.b + 1];
+            c.lo = rlo[c.b];
+            c.hi = rhi[c.b];
+            c.rnew = rnew[c.b];
+            c.k0 = (c.lo / TK + (c.tau - tpre[c.b])) * TK;
+            const ItemRef it = item_ref<MULTI>(p, c.b);
+            c.pt = p.page_table + static_cast<size_t>(it.req) * p.max_pages;
+            c.gofs = static_cast<size_t>(it.grp) * ROWB;
+        };
+        auto cur_init = [&](Cur& c, int tau) {
+            c.tau = tau;
+            c.b = find_req(tau);
+            cur_enter(c);
+        };
+        auto cur_next = [&](Cur& c) {
+            ++c.tau;
+            c.k0 += TK;
+            if (c.tau >= c.end && c.tau < t1 && c.b < B - 1) {
+                do {
+                    ++c.b;
+                } while (c.b < B - 1 && c.tau >= tpre[c.b + 1]);
+                cur_enter(c);
+            }
+        };
+        auto issue_idx = [&](const Cur& c) {
+            if (c.tau >= t1) return;
+            int* dst = idx_smem + ((c.tau - t0) % C::IDX_SLOTS) * TK;
             if (PS == 1) {
                 if (ltid < TK) {
-                    const int k = k0 + ltid;
-                    if (k >= rlo[b] && k <= rhi[b] && k < p.max_pages) cp_async4(smem_addr(dst + ltid), pt + k);
+                    const int k = c.k0 + ltid;
+                    if (k >= c.lo && k <= c.hi && k < p.max_pages) cp_async4(smem_addr(dst + ltid), c.pt + k);
                     else dst[ltid] = -1;
                 }
             } else {
                 if (ltid < TK / PS) {
-                    const int pg = k0 / PS + ltid;
-                    if (pg < p.max_pages) cp_async4(smem_addr(dst + ltid), pt + pg);
+                    const int pg = c.k0 / PS + ltid;
+                    if (pg < p.max_pages) cp_async4(smem_addr(dst + ltid), c.pt + pg);
                     else dst[ltid] = -1;
                 }
             }
         };
-        auto issue_kv = [&](int tau, int b) {
-            if (tau >= t1) return;
-            const int k0 = tile_k0(tau, b);
-            if (k0 + TK - 1 >= rnew[b]) ensure_prep();
-            const int* ix = idx_smem + ((tau - t0) % C::IDX_SLOTS) * TK;
-            const uint32_t base = smem_addr(raw + ((tau - t0) % NS) * RAW_STAGE);
-            const int lo = rlo[b], hi = rhi[b];
+        auto issue_kv = [&](const Cur& c) {
+            if (c.tau >= t1) return;
+            const int k0 = c.k0;
+            if (k0 + TK - 1 >= c.rnew) ensure_prep();
+            const int* ix = idx_smem + ((c.tau - t0) % C::IDX_SLOTS) * TK;
+            const uint32_t base = smem_addr(raw + ((c.tau - t0) % NS) * RAW_STAGE);
+            const int lo = c.lo, hi = c.hi;
             const size_t row_pitch = static_cast<size_t>(ROWB) * ng;
-            const size_t gofs = static_cast<size_t>(item_ref<MULTI>(p, b).grp) * ROWB;
+            const size_t gofs = c.gofs;
             constexpr int ROWS = TK * 8 / LOADERS;  // rows per thread
             const int j = ltid & 7;                 // 16-byte chunk
             // all page-table reads first, then the copies (the copies are ordered
@@ -299,26 +330,29 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
             }
         };
 
-        int xt = t0, xb = find_req(t0);
-        int kt = t0, kb = xb;
-        int ct = t0, cb = xb;
+        Cur xc, kc, cc;  // page-table cursor (NS - 1 tiles ahead), gather cursor, current tile
+        cur_init(xc, t0);
+        kc = xc;
+        cc = xc;
         for (int d = 0; d < NS - 1; ++d) {
-            issue_idx(xt, xb);
-            advance(xt, xb);
+            issue_idx(xc);
+            cur_next(xc);
         }
         cp_async_commit();
         cp_async_wait<0>();
         bar_red_or(1, LOADERS, false);
         for (int d = 0; d < NS - 1; ++d) {
-            issue_kv(kt, kb);
-            advance(kt, kb);
-            issue_idx(xt, xb);
-            advance(xt, xb);
+            issue_kv(kc);
+            cur_next(kc);
+            issue_idx(xc);
+            cur_next(xc);
             cp_async_commit();
         }
         int seg_b = -1;
-        for (int i = 0; ct < t1; ++i) {
+        const int n_tiles = t1 - t0;
+        for (int i = 0; i < n_tiles; ++i) {
             cp_async_wait<NS - 2>();
+            const int cb = cc.b;
             const bool seg_start = cb != seg_b;
             bool bad = false;
             // buffers i & 1 are free once PV(i - 2) is done (which also means every
@@ -341,12 +375,12 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
             mbar_arrive(BAR(BAR_KV_READY + (i & 1)));
             // gathers for tile i + NS - 1 (into the stage of tile i - 1), off the
             // path from "buffer free" to "tile ready"
-            issue_kv(kt, kb);
-            advance(kt, kb);
-            issue_idx(xt, xb);
-            advance(xt, xb);
+            issue_kv(kc);
+            cur_next(kc);
+            issue_idx(xc);
+            cur_next(xc);
             cp_async_commit();
-            advance(ct, cb);
+            cur_next(cc);
         }
         cp_async_wait<0>();
     }
