@@ -48,9 +48,9 @@ FALLBACK_TC_TFLOPS = 1590.0  # dense bf16/fp16 burst
 # kernel on a workload, from the ncu captures summarised in profiles/, keyed by
 # the hash of that kernel's sources when the counters were taken (null once the
 # sources change).
-TRAFFIC = {("decode32_full", "ecccb345769b7cca"): 475291136,
-           ("verify16_full", "5f0d2aa17c4a40fd"): 338384640,
-           ("prefill1_full", "e507e97fc090faf7"): 22618624}
+TRAFFIC = {("decode32_full", "dce70aae8d336778"): 474898688,
+           ("verify16_full", "5108fbb7729675b7"): 337329152,
+           ("prefill1_full", "90bafec800f8719d"): 22619136}
 
 # Sources of the step's main kernel: decode_kernel for single-token steps,
 # verify_tc_kernel for verify blocks, prefill_tc_kernel for longer blocks (the
