@@ -18,8 +18,11 @@ namespace gad {
 // ---------------------------------------------------------------------------
 // Block width: 1024 threads (64 slot lanes) for steps with few tokens, whose
 // requests are spread over many CTAs; 256 (16 slot lanes) otherwise.
+// The 1024-thread form must keep two blocks per SM (at most 32 registers a
+// thread): a 16-token step launches 256 of them, one wave on 148 SMs only if
+// two fit.
 template <int COMB_THREADS>
-__global__ void __launch_bounds__(COMB_THREADS) combine_kernel(const StepParams p) {
+__global__ void __launch_bounds__(COMB_THREADS, COMB_THREADS >= 1024 ? 2 : 1) combine_kernel(const StepParams p) {
     constexpr int COMB_SLOT_LANES = COMB_THREADS / 16;
     pdl_wait_primary();
     pdl_launch_dependents();  // a following projection may start its weight loads
