@@ -562,6 +562,12 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     } else if (T * ngrp <= 16) {
         cfg.blockDim = dim3(1024);
         e = cudaLaunchKernelEx(&cfg, gad::combine_kernel<1024>, prm);
+    } else if (L > 1) {  // verify blocks: one warp per (token, head), four slots at a time
+        constexpr int per_block = gad::COMBW4_THREADS / 32;
+        cfg.gridDim = dim3(static_cast<unsigned>((static_cast<long long>(T) * gad::HQ * ngrp +
+                                                  per_block - 1) / per_block));
+        cfg.blockDim = dim3(gad::COMBW4_THREADS);
+        e = cudaLaunchKernelEx(&cfg, gad::combine_warp4_kernel, prm);
     } else {
         cfg.blockDim = dim3(256);
         e = cudaLaunchKernelEx(&cfg, gad::combine_kernel<256>, prm);

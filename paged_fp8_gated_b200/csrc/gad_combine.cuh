@@ -18,11 +18,11 @@ namespace gad {
 // ---------------------------------------------------------------------------
 // Block width: 1024 threads (64 slot lanes) for steps with few tokens, whose
 // requests are spread over many CTAs; 256 (16 slot lanes) otherwise.
-// The 1024-thread form must keep two blocks per SM (at most 32 registers a
-// thread): a 16-token step launches 256 of them, one wave on 148 SMs only if
-// two fit.
+// Both forms keep 2,048 threads per SM (at most 32 registers a thread): a
+// 16-token step launches 256 blocks of 1024 threads, one wave on 148 SMs only
+// if two fit, and verify steps launch thousands of 256-thread blocks.
 template <int COMB_THREADS>
-__global__ void __launch_bounds__(COMB_THREADS, COMB_THREADS >= 1024 ? 2 : 1) combine_kernel(const StepParams p) {
+__global__ void __launch_bounds__(COMB_THREADS, 2048 / COMB_THREADS) combine_kernel(const StepParams p) {
     constexpr int COMB_SLOT_LANES = COMB_THREADS / 16;
     pdl_wait_primary();
     pdl_launch_dependents();  // a following projection may start its weight loads
@@ -41,21 +41,24 @@ __global__ void __launch_bounds__(COMB_THREADS, COMB_THREADS >= 1024 ? 2 : 1) co
     const int tp = p.meta[META_PREFIX + b];
     const int n = p.meta[META_PREFIX + b + 1] - tp;
     const int per = p.meta[META_PER];
-    __nv_bfloat16* outp = p.out + static_cast<size_t>(t) * OUT_COLS * ng + hh * HD;
+    // the output row is addressed only at the end (a 64-bit pointer held across
+    // the loops would not fit the 32-register budget)
+    auto outp = [&]() { return p.out + static_cast<size_t>(t) * OUT_COLS * ng + hh * HD; };
     if (n <= 0 || per <= 0) {  // no key in range (positions outside the contract)
-        if (tid < HD) outp[tid] = __float2bfloat16(NAN);
+        if (tid < HD) outp()[tid] = __float2bfloat16(NAN);
         return;
     }
     const int c_lo = tp / per, c_hi = (tp + n - 1) / per;
     const int TL = p.tl;
     const int ns = (c_hi - c_lo + 1) * TL;
-    // Partial s = (CTA c_lo + s / TL, lane s % TL); every CTA that covered some
-    // of the request's tiles wrote all its lanes (a lane that saw no key of the
-    // request has max -inf and is skipped).
-    auto slot_base = [&](int s) {
-        const int c = c_lo + s / TL, tl = s % TL;
-        return ((static_cast<size_t>(c + b) * TL + tl) * p.lt + j) * p.hp + h;
-    };
+    // Partial s = (CTA c_lo + s / TL, lane s % TL) sits in slot (c + b) * TL + lane
+    // = (c_lo + b) * TL + s; every CTA that covered some of the request's tiles
+    // wrote all its lanes (a lane that saw no key of the request has max -inf and
+    // is skipped).  Row (token j, head h) of a slot: slot * lt * hp + j * hp + h.
+    // 32-bit row indices: the workspace holds fewer than 2^25 partial rows
+    const int slot0 = (c_lo + b) * TL;
+    const int stride = p.lt * p.hp, row0 = j * p.hp + h;
+    auto slot_base = [&](int s) { return (slot0 + s) * stride + row0; };
     // 1. global max over the slots
     float mx = -INFINITY;
     for (int s = tid; s < ns; s += COMB_THREADS) mx = fmaxf(mx, p.part_ml[slot_base(s) * 2]);
@@ -72,7 +75,7 @@ __global__ void __launch_bounds__(COMB_THREADS, COMB_THREADS >= 1024 ? 2 : 1) co
     float lsum = 0.f;
 #pragma unroll 2
     for (int s = sl; s < ns; s += COMB_SLOT_LANES) {
-        const size_t base = slot_base(s);
+        const int base = slot_base(s);
         const float ms = p.part_ml[base * 2];
         if (ms == -INFINITY) continue;
         const float w = exp2f(ms - M);
@@ -104,7 +107,7 @@ __global__ void __launch_bounds__(COMB_THREADS, COMB_THREADS >= 1024 ? 2 : 1) co
         const float rinv = 1.0f / sqrtf(tot * (1.0f / 64.0f) + 1e-6f);
         const float g = __bfloat162float(
             p.qkv[static_cast<size_t>(t) * QKV_COLS * ng + G_OFF * ng + hh * HD + tid]);
-        outp[tid] = __float2bfloat16(a * rinv / (1.0f + expf(-g)));
+        outp()[tid] = __float2bfloat16(a * rinv / (1.0f + expf(-g)));
     }
 }
 
@@ -137,17 +140,16 @@ __global__ void __launch_bounds__(COMBW_THREADS) combine_warp_kernel(const StepP
     const int c_lo = tp / per, c_hi = (tp + n - 1) / per;
     const int TL = p.tl;
     const int ns = (c_hi - c_lo + 1) * TL;
-    auto slot_base = [&](int s) {
-        const int c = c_lo + s / TL, tl = s % TL;
-        return ((static_cast<size_t>(c + b) * TL + tl) * p.lt + j) * p.hp + h;
-    };
+    const int slot0 = (c_lo + b) * TL;  // slot of partial s: slot0 + s (32-bit row indices)
+    const int stride = p.lt * p.hp, row0 = j * p.hp + h;
+    auto slot_base = [&](int s) { return (slot0 + s) * stride + row0; };
     float M = -INFINITY;
     for (int s = lane; s < ns; s += 32) M = fmaxf(M, p.part_ml[slot_base(s) * 2]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float o0 = 0.f, o1 = 0.f, l = 0.f;
     for (int s = 0; s < ns; ++s) {
-        const size_t base = slot_base(s);
+        const int base = slot_base(s);
         const float ms = p.part_ml[base * 2];
         if (ms == -INFINITY) continue;
         const float w = exp2f(ms - M);
@@ -166,6 +168,90 @@ __global__ void __launch_bounds__(COMBW_THREADS) combine_warp_kernel(const StepP
     const float g0 = __bfloat162float(gp[0]), g1 = __bfloat162float(gp[1]);
     outp[0] = __float2bfloat16(a0 * rinv / (1.0f + expf(-g0)));
     outp[1] = __float2bfloat16(a1 * rinv / (1.0f + expf(-g1)));
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 3c: one warp per (token, query head) in four slot groups of eight
+// lanes, lane (g, dl) holding dims 8dl..8dl+7 of slots g, g + 4, ...; the
+// groups are summed with shuffles.  For verify blocks: thousands of (token,
+// head) pairs with tens of partials each, where the block form above leaves
+// most of its threads idle behind barriers and the single-slot warp form
+// walks the partials one by one.
+// ---------------------------------------------------------------------------
+constexpr int COMBW4_THREADS = 256;
+__global__ void __launch_bounds__(COMBW4_THREADS) combine_warp4_kernel(const StepParams p) {
+    pdl_wait_primary();
+    pdl_launch_dependents();  // a following projection may start its weight loads
+    const int ng = p.ngrp, hq_all = HQ * ng;
+    const int lane = threadIdx.x & 31, g = lane >> 3, dl = lane & 7;
+    const long long gw = static_cast<long long>(blockIdx.x) * (COMBW4_THREADS / 32) + (threadIdx.x >> 5);
+    if (gw >= static_cast<long long>(p.B) * p.L * hq_all) return;
+    const int t = static_cast<int>(gw / hq_all), hh = static_cast<int>(gw % hq_all);
+    const int h = hh % p.hp;
+    const int jr = t % p.L;
+    const int b = ((t / p.L) * p.nchunk + jr / p.chunk) * p.nsub + hh / p.hp, j = jr % p.chunk;
+    const int tp = p.meta[META_PREFIX + b];
+    const int n = p.meta[META_PREFIX + b + 1] - tp;
+    const int per = p.meta[META_PER];
+    const int d0 = 8 * dl + 2 * g;  // the two output dims this lane writes
+    __nv_bfloat162* outp = reinterpret_cast<__nv_bfloat162*>(p.out + static_cast<size_t>(t) * OUT_COLS * ng +
+                                                             hh * HD + d0);
+    if (n <= 0 || per <= 0) {  // no key in range (positions outside the contract)
+        *outp = __floats2bfloat162_rn(NAN, NAN);
+        return;
+    }
+    const int c_lo = tp / per, c_hi = (tp + n - 1) / per;
+    const int TL = p.tl;
+    const int ns = (c_hi - c_lo + 1) * TL;
+    const int slot0 = (c_lo + b) * TL;  // slot of partial s: slot0 + s (32-bit row indices)
+    const int stride = p.lt * p.hp, row0 = j * p.hp + h;
+    auto slot_base = [&](int s) { return (slot0 + s) * stride + row0; };
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, p.part_ml[slot_base(s) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float l = 0.f;
+#pragma unroll 2
+    for (int s = g; s < ns; s += 4) {
+        const int base = slot_base(s);
+        const float ms = p.part_ml[base * 2];
+        if (ms == -INFINITY) continue;
+        const float w = exp2f(ms - M);
+        const float4* src = reinterpret_cast<const float4*>(p.part_o + base * HD + 8 * dl);
+        const float4 x = src[0], y = src[1];
+        acc[0] += w * x.x;
+        acc[1] += w * x.y;
+        acc[2] += w * x.z;
+        acc[3] += w * x.w;
+        acc[4] += w * y.x;
+        acc[5] += w * y.y;
+        acc[6] += w * y.z;
+        acc[7] += w * y.w;
+        l += w * p.part_ml[base * 2 + 1];
+    }
+#pragma unroll
+    for (int o = 8; o <= 16; o <<= 1) {  // sum the four slot groups
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+        l += __shfl_xor_sync(0xffffffffu, l, o);
+    }
+    const float vs = __ldg(p.v_scale);
+    float ss = 0.f, a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float a = acc[i] / l * vs;
+        ss += a * a;
+        if (i == 2 * g) a0 = a;  // unrolled selects: no local-memory indexing
+        if (i == 2 * g + 1) a1 = a;
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);  // over the 8 dim lanes
+    const float rinv = 1.0f / sqrtf(ss * (1.0f / 64.0f) + 1e-6f);
+    const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162*>(
+        p.qkv + static_cast<size_t>(t) * QKV_COLS * ng + G_OFF * ng + hh * HD + d0);
+    const float g0 = __low2float(gv), g1 = __high2float(gv);
+    *outp = __floats2bfloat162_rn(a0 * rinv / (1.0f + expf(-g0)), a1 * rinv / (1.0f + expf(-g1)));
 }
 
 }  // namespace gad
