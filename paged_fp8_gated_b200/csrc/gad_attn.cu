@@ -24,6 +24,7 @@
 #include "gad_kernels.cuh"
 #include "gad_oproj.cuh"
 #include "gad_prefill_tc.cuh"
+#include "gad_prep.cuh"
 #include "gad_verify_tc.cuh"
 
 namespace {
@@ -346,6 +347,7 @@ int check_oproj(const void* out, const void* w, const void* a, int T, int K, int
 int launch_oproj(const void* out, const void* w, void* a, int T, int K, int N, cudaStream_t s, bool pdl) {
     const int tt = T >= gad::opj::TT_MAX ? gad::opj::TT_MAX : (T + 15) / 16 * 16;
     const int nstg = gad::opj::stages(tt, K / gad::opj::BK);
+    if (nstg < 1) return fail(GAD_ERR_SHAPE, "projection ring: %d stages", nstg);  // never launched empty
     const size_t smem = gad::opj::smem_bytes(tt, nstg);
     static std::atomic<bool> attr_done[kMaxDevices];
     static std::atomic<void*> err_addr[kMaxDevices];
@@ -561,7 +563,8 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
         e = cudaLaunchKernelEx(&cfg, gad::combine_warp_kernel, prm);
     } else if (T * ngrp <= 16) {
         cfg.blockDim = dim3(1024);
-        e = cudaLaunchKernelEx(&cfg, gad::combine_kernel<1024>, prm);
+        e = T * gad::HQ * ngrp <= sms ? cudaLaunchKernelEx(&cfg, gad::combine_kernel<1024, 1>, prm)
+                                      : cudaLaunchKernelEx(&cfg, gad::combine_kernel<1024, 2>, prm);
     } else if (L > 1) {  // verify blocks: one warp per (token, head), four slots at a time
         constexpr int per_block = gad::COMBW4_THREADS / 32;
         cfg.gridDim = dim3(static_cast<unsigned>((static_cast<long long>(T) * gad::HQ * ngrp +
@@ -570,7 +573,7 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
         e = cudaLaunchKernelEx(&cfg, gad::combine_warp4_kernel, prm);
     } else {
         cfg.blockDim = dim3(256);
-        e = cudaLaunchKernelEx(&cfg, gad::combine_kernel<256>, prm);
+        e = cudaLaunchKernelEx(&cfg, gad::combine_kernel<256, 8>, prm);
     }
     if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
     if (timed) {

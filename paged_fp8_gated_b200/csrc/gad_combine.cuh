@@ -18,22 +18,30 @@ namespace gad {
 // ---------------------------------------------------------------------------
 // Block width: 1024 threads (64 slot lanes) for steps with few tokens, whose
 // requests are spread over many CTAs; 256 (16 slot lanes) otherwise.
-// Both forms keep 2,048 threads per SM (at most 32 registers a thread): a
+// MINB blocks per SM: a grid of at most one block per SM (a 1-token step: 16
+// blocks) runs each block faster with registers to spare (56 a thread); a
 // 16-token step launches 256 blocks of 1024 threads, one wave on 148 SMs only
-// if two fit, and verify steps launch thousands of 256-thread blocks.
-template <int COMB_THREADS>
-__global__ void __launch_bounds__(COMB_THREADS, 2048 / COMB_THREADS) combine_kernel(const StepParams p) {
+// if two fit (32 registers a thread), and so do 8 blocks of 256 threads.
+template <int COMB_THREADS, int MINB>
+__global__ void __launch_bounds__(COMB_THREADS, MINB) combine_kernel(const StepParams p) {
     constexpr int COMB_SLOT_LANES = COMB_THREADS / 16;
-    pdl_wait_primary();
-    pdl_launch_dependents();  // a following projection may start its weight loads
     __shared__ float red_o[COMB_SLOT_LANES][HD];
     __shared__ float red_l[COMB_SLOT_LANES];
     __shared__ float red_m[COMB_THREADS / 32];
     __shared__ float red_ss[4];
+    __shared__ float gate_s[HD + 1];  // the gate row and v_scale (step inputs)
     const int ng = p.ngrp, hq_all = HQ * ng;
     const int t = blockIdx.x / hq_all, hh = blockIdx.x % hq_all;  // hh = 16 * group + h
     const int h = hh % p.hp;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // The gate and v_scale are inputs, not results of the earlier kernels: fetch
+    // them while those finish (parked in shared memory, off the register budget).
+    if (tid < HD)
+        gate_s[tid] = __bfloat162float(p.qkv[static_cast<size_t>(t) * QKV_COLS * ng + G_OFF * ng + hh * HD + tid]);
+    else if (tid == HD)
+        gate_s[HD] = __ldg(p.v_scale);
+    pdl_wait_primary();
+    pdl_launch_dependents();  // a following projection may start its weight loads
     // list item (request, chunk, sub) and the token's place in the chunk; the
     // partial rows of an item hold p.hp query heads (sub = hh / hp)
     const int jr = t % p.L;
@@ -42,7 +50,7 @@ __global__ void __launch_bounds__(COMB_THREADS, 2048 / COMB_THREADS) combine_ker
     const int n = p.meta[META_PREFIX + b + 1] - tp;
     const int per = p.meta[META_PER];
     // the output row is addressed only at the end (a 64-bit pointer held across
-    // the loops would not fit the 32-register budget)
+    // the loops would not fit a 32-register budget)
     auto outp = [&]() { return p.out + static_cast<size_t>(t) * OUT_COLS * ng + hh * HD; };
     if (n <= 0 || per <= 0) {  // no key in range (positions outside the contract)
         if (tid < HD) outp()[tid] = __float2bfloat16(NAN);
@@ -97,7 +105,7 @@ __global__ void __launch_bounds__(COMB_THREADS, 2048 / COMB_THREADS) combine_ker
             o += red_o[k][tid];
             l += red_l[k];
         }
-        const float a = o / l * __ldg(p.v_scale);
+        const float a = o / l * gate_s[HD];
         float ss = a * a;
 #pragma unroll
         for (int q = 16; q > 0; q >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, q);
@@ -105,8 +113,7 @@ __global__ void __launch_bounds__(COMB_THREADS, 2048 / COMB_THREADS) combine_ker
         asm volatile("bar.sync 1, 64;\n" ::: "memory");
         const float tot = red_ss[0] + red_ss[1];
         const float rinv = 1.0f / sqrtf(tot * (1.0f / 64.0f) + 1e-6f);
-        const float g = __bfloat162float(
-            p.qkv[static_cast<size_t>(t) * QKV_COLS * ng + G_OFF * ng + hh * HD + tid]);
+        const float g = gate_s[tid];
         outp()[tid] = __float2bfloat16(a * rinv / (1.0f + expf(-g)));
     }
 }
@@ -119,13 +126,22 @@ __global__ void __launch_bounds__(COMB_THREADS, 2048 / COMB_THREADS) combine_ker
 // ---------------------------------------------------------------------------
 constexpr int COMBW_THREADS = 256;
 __global__ void __launch_bounds__(COMBW_THREADS) combine_warp_kernel(const StepParams p) {
-    pdl_wait_primary();
-    pdl_launch_dependents();  // a following projection may start its weight loads
     const int ng = p.ngrp, hq_all = HQ * ng;
     const int lane = threadIdx.x & 31;
     const long long gw = static_cast<long long>(blockIdx.x) * (COMBW_THREADS / 32) + (threadIdx.x >> 5);
-    if (gw >= static_cast<long long>(p.B) * p.L * hq_all) return;
-    const int t = static_cast<int>(gw / hq_all), hh = static_cast<int>(gw % hq_all);
+    const bool live = gw < static_cast<long long>(p.B) * p.L * hq_all;
+    const int t = live ? static_cast<int>(gw / hq_all) : 0, hh = live ? static_cast<int>(gw % hq_all) : 0;
+    // the gate and v_scale are step inputs: fetched while the earlier kernels finish
+    __nv_bfloat162 gv = __floats2bfloat162_rn(0.f, 0.f);
+    float vs = 0.f;
+    if (live) {
+        gv = *reinterpret_cast<const __nv_bfloat162*>(p.qkv + static_cast<size_t>(t) * QKV_COLS * ng +
+                                                       G_OFF * ng + hh * HD + 2 * lane);
+        vs = __ldg(p.v_scale);
+    }
+    pdl_wait_primary();
+    pdl_launch_dependents();  // a following projection may start its weight loads
+    if (!live) return;
     const int h = hh % p.hp;
     const int jr = t % p.L;
     const int b = ((t / p.L) * p.nchunk + jr / p.chunk) * p.nsub + hh / p.hp, j = jr % p.chunk;
@@ -158,14 +174,12 @@ __global__ void __launch_bounds__(COMBW_THREADS) combine_warp_kernel(const StepP
         o1 += w * o.y;
         l += w * p.part_ml[base * 2 + 1];
     }
-    const float vs = __ldg(p.v_scale);
     const float a0 = o0 / l * vs, a1 = o1 / l * vs;
     float ss = a0 * a0 + a1 * a1;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float rinv = 1.0f / sqrtf(ss * (1.0f / 64.0f) + 1e-6f);
-    const __nv_bfloat16* gp = p.qkv + static_cast<size_t>(t) * QKV_COLS * ng + G_OFF * ng + hh * HD + 2 * lane;
-    const float g0 = __bfloat162float(gp[0]), g1 = __bfloat162float(gp[1]);
+    const float g0 = __low2float(gv), g1 = __high2float(gv);
     outp[0] = __float2bfloat16(a0 * rinv / (1.0f + expf(-g0)));
     outp[1] = __float2bfloat16(a1 * rinv / (1.0f + expf(-g1)));
 }
@@ -180,20 +194,29 @@ __global__ void __launch_bounds__(COMBW_THREADS) combine_warp_kernel(const StepP
 // ---------------------------------------------------------------------------
 constexpr int COMBW4_THREADS = 256;
 __global__ void __launch_bounds__(COMBW4_THREADS) combine_warp4_kernel(const StepParams p) {
-    pdl_wait_primary();
-    pdl_launch_dependents();  // a following projection may start its weight loads
     const int ng = p.ngrp, hq_all = HQ * ng;
     const int lane = threadIdx.x & 31, g = lane >> 3, dl = lane & 7;
     const long long gw = static_cast<long long>(blockIdx.x) * (COMBW4_THREADS / 32) + (threadIdx.x >> 5);
-    if (gw >= static_cast<long long>(p.B) * p.L * hq_all) return;
-    const int t = static_cast<int>(gw / hq_all), hh = static_cast<int>(gw % hq_all);
+    const bool live = gw < static_cast<long long>(p.B) * p.L * hq_all;
+    const int t = live ? static_cast<int>(gw / hq_all) : 0, hh = live ? static_cast<int>(gw % hq_all) : 0;
+    const int d0 = 8 * dl + 2 * g;  // the two output dims this lane writes
+    // the gate and v_scale are step inputs: fetched while the earlier kernels finish
+    __nv_bfloat162 gv = __floats2bfloat162_rn(0.f, 0.f);
+    float vs = 0.f;
+    if (live) {
+        gv = *reinterpret_cast<const __nv_bfloat162*>(p.qkv + static_cast<size_t>(t) * QKV_COLS * ng +
+                                                       G_OFF * ng + hh * HD + d0);
+        vs = __ldg(p.v_scale);
+    }
+    pdl_wait_primary();
+    pdl_launch_dependents();  // a following projection may start its weight loads
+    if (!live) return;
     const int h = hh % p.hp;
     const int jr = t % p.L;
     const int b = ((t / p.L) * p.nchunk + jr / p.chunk) * p.nsub + hh / p.hp, j = jr % p.chunk;
     const int tp = p.meta[META_PREFIX + b];
     const int n = p.meta[META_PREFIX + b + 1] - tp;
     const int per = p.meta[META_PER];
-    const int d0 = 8 * dl + 2 * g;  // the two output dims this lane writes
     __nv_bfloat162* outp = reinterpret_cast<__nv_bfloat162*>(p.out + static_cast<size_t>(t) * OUT_COLS * ng +
                                                              hh * HD + d0);
     if (n <= 0 || per <= 0) {  // no key in range (positions outside the contract)
@@ -236,7 +259,6 @@ __global__ void __launch_bounds__(COMBW4_THREADS) combine_warp4_kernel(const Ste
         for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
         l += __shfl_xor_sync(0xffffffffu, l, o);
     }
-    const float vs = __ldg(p.v_scale);
     float ss = 0.f, a0 = 0.f, a1 = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -248,8 +270,6 @@ __global__ void __launch_bounds__(COMBW4_THREADS) combine_warp4_kernel(const Ste
 #pragma unroll
     for (int o = 1; o < 8; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);  // over the 8 dim lanes
     const float rinv = 1.0f / sqrtf(ss * (1.0f / 64.0f) + 1e-6f);
-    const __nv_bfloat162 gv = *reinterpret_cast<const __nv_bfloat162*>(
-        p.qkv + static_cast<size_t>(t) * QKV_COLS * ng + G_OFF * ng + hh * HD + d0);
     const float g0 = __low2float(gv), g1 = __high2float(gv);
     *outp = __floats2bfloat162_rn(a0 * rinv / (1.0f + expf(-g0)), a1 * rinv / (1.0f + expf(-g1)));
 }

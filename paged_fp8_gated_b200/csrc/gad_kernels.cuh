@@ -1,14 +1,14 @@
-// gad_kernels.cuh - the three sm_100a kernels of one attention step.
+// gad_kernels.cuh - the step's shared definitions (head groups, StepParams,
+// the tile list) and its single-token attention kernel.
 //
-//   prep_kernel     per token: QK-norm, RoPE, E4M3 quantise-and-scatter of k/v
-//                   into the cache rows cache_loc[t]; normalised q -> workspace.
 //   decode_kernel   persistent split-KV flash decode over the paged FP8 cache:
 //                   cp.async gathers into a swizzled shared-memory ring, tensor-
 //                   core QK^T and PV (m16n8k16 fp16, fp32 accumulate) with the
 //                   query heads of one KV head packed into the MMA's N side,
 //                   online softmax, one (o, max, sum) partial per CTA segment.
-//   (the combine kernels, which merge the partials and apply the gated output
-//   norm, are in gad_combine.cuh)
+//   (prep_kernel, per token QK-norm, RoPE and the E4M3 cache append, is in
+//   gad_prep.cuh; the combine kernels, which merge the partials and apply the
+//   gated output norm, are in gad_combine.cuh)
 //
 // Method: task page "Gated attention decode (muse_attention_decode)", section
 // "What to compute"; shapes from its section "Shapes".
@@ -107,74 +107,6 @@ constexpr int META_PER = 1;      // tiles per CTA
 constexpr int META_ERROR = 2;    // nonzero: a bounded wait in the decode kernel timed out
 constexpr int META_PREFIX = 3;   // [NB + 1] tile prefix over list items
 constexpr int META_INTS = 4;     // + NB
-
-// ---------------------------------------------------------------------------
-// Kernel 1: split + QK-norm + RoPE + E4M3 quantise-and-scatter.
-// One block per (token, head group); warp w < 16 handles query head w of the
-// group, warps 16 and 17 its two KV heads.  Lane l owns the RoPE pair (l, l + 32).  Done in double so the
-// cache bytes match the double-precision definition exactly: the sum of squares
-// runs in index order with explicit round-to-nearest operations (no fused
-// multiply-add), as does the rotation.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) {
-    pdl_launch_dependents();
-    const int ng = p.ngrp;
-    const int t = blockIdx.x / ng, c = blockIdx.x % ng;
-    if (blockIdx.x == 0 && threadIdx.x == 0) p.meta[META_ERROR] = 0;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const __nv_bfloat16* row = p.qkv + static_cast<size_t>(t) * QKV_COLS * ng;
-    const bool is_q = warp < HQ;
-    const int g = warp - HQ;
-    const int off = is_q ? c * OUT_COLS + warp * HD : K_OFF * ng + c * ROWB + g * HD;
-    const double x0 = static_cast<double>(__bfloat162float(row[off + lane]));
-    const double x1 = static_cast<double>(__bfloat162float(row[off + lane + 32]));
-
-    double ss = 0.0;
-    for (int d = 0; d < 32; ++d) {
-        const double v = __shfl_sync(0xffffffffu, x0, d);
-        ss = __dadd_rn(ss, __dmul_rn(v, v));
-    }
-    for (int d = 0; d < 32; ++d) {
-        const double v = __shfl_sync(0xffffffffu, x1, d);
-        ss = __dadd_rn(ss, __dmul_rn(v, v));
-    }
-    const double r = sqrt(__dadd_rn(ss / 64.0, 1e-6));
-    double u0 = x0 / r, u1 = x1 / r;
-    if (is_q) {
-        u0 = __dmul_rn(u0, 5.473);
-        u1 = __dmul_rn(u1, 5.473);
-    }
-    if (p.use_rope) {
-        const double pos = static_cast<double>(p.positions[t]);
-        const double phi = __dmul_rn(pos, p.inv_freq[lane]);
-        double s, c;
-        sincos(phi, &s, &c);
-        const double r0 = __dsub_rn(__dmul_rn(u0, c), __dmul_rn(u1, s));
-        const double r1 = __dadd_rn(__dmul_rn(u1, c), __dmul_rn(u0, s));
-        u0 = r0;
-        u1 = r1;
-    }
-    if (is_q) {
-        __half* q = p.q_ws + (static_cast<size_t>(blockIdx.x) * HQ + warp) * HD;
-        q[lane] = __double2half(u0);
-        q[lane + 32] = __double2half(u1);
-        return;
-    }
-    const int64_t crow = p.cache_loc[t];
-    if (crow < 0 || crow >= p.num_rows) return;
-    const double ks = static_cast<double>(__ldg(p.k_scale));
-    const double vs = static_cast<double>(__ldg(p.v_scale));
-    const int64_t cofs = crow * (ROWB * ng) + c * ROWB + g * HD;
-    uint8_t* kd = p.k_cache + cofs;
-    uint8_t* vd = p.v_cache + cofs;
-    kd[lane] = __nv_cvt_float_to_fp8(__double2float_rn(u0 / ks), __NV_SATFINITE, __NV_E4M3);
-    kd[lane + 32] = __nv_cvt_float_to_fp8(__double2float_rn(u1 / ks), __NV_SATFINITE, __NV_E4M3);
-    const int voff = V_OFF * ng + c * ROWB + g * HD;
-    const double v0 = static_cast<double>(__bfloat162float(row[voff + lane]));
-    const double v1 = static_cast<double>(__bfloat162float(row[voff + lane + 32]));
-    vd[lane] = __nv_cvt_float_to_fp8(__double2float_rn(v0 / vs), __NV_SATFINITE, __NV_E4M3);
-    vd[lane + 32] = __nv_cvt_float_to_fp8(__double2float_rn(v1 / vs), __NV_SATFINITE, __NV_E4M3);
-}
 
 // ---------------------------------------------------------------------------
 // Kernel 2: split-KV decode.

@@ -33,7 +33,7 @@ def _check_a(a_gpu_bits, a_exact, x_abs_bound):
     return worst
 
 
-@pytest.mark.parametrize("T", [1, 5, 16, 32, 100, 256, 300, 1000])
+@pytest.mark.parametrize("T", [1, 5, 16, 32, 100, 128, 256, 300, 1000])
 def test_oproj_matches_oracle(T, cuda_dev):
     x = W.oproj_input(T, seed=100 + T)
     w = W.oproj_weight()
@@ -48,7 +48,7 @@ def test_oproj_matches_oracle(T, cuda_dev):
     assert (_bits(a) == a_bits).mean() > 0.99
 
 
-@pytest.mark.parametrize("K,N", [(64, 128), (128, 256), (1024, 384)])
+@pytest.mark.parametrize("K,N", [(64, 128), (128, 256), (192, 128), (1024, 384)])
 def test_oproj_small_shapes(K, N, cuda_dev):
     from paged_fp8_gated_b200 import binding
     g = torch.Generator().manual_seed(K + N)
