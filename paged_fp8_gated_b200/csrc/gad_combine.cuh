@@ -81,18 +81,23 @@ __global__ void __launch_bounds__(COMB_THREADS, MINB) combine_kernel(const StepP
     const int sl = tid / 16, dq = tid % 16;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.f;
-#pragma unroll 2
+    // partials in flight per thread: 4 with the registers of one block per SM
+    // (the loop is bound by L2 latency when 16 blocks merge ~1,200 partials each)
+#pragma unroll(MINB == 1 ? 4 : 2)
     for (int s = sl; s < ns; s += COMB_SLOT_LANES) {
         const int base = slot_base(s);
-        const float ms = p.part_ml[base * 2];
-        if (ms == -INFINITY) continue;
-        const float w = exp2f(ms - M);
+        // All three loads are issued before the test (every slot below ns was
+        // written by this step), so unrolled iterations overlap their latency.
+        const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + base * 2);
         const float4 o = *reinterpret_cast<const float4*>(p.part_o + base * HD + 4 * dq);
-        acc.x += w * o.x;
-        acc.y += w * o.y;
-        acc.z += w * o.z;
-        acc.w += w * o.w;
-        lsum += w * p.part_ml[base * 2 + 1];
+        if (ml.x != -INFINITY) {
+            const float w = exp2f(ml.x - M);
+            acc.x += w * o.x;
+            acc.y += w * o.y;
+            acc.z += w * o.z;
+            acc.w += w * o.w;
+            lsum += w * ml.y;
+        }
     }
     *reinterpret_cast<float4*>(&red_o[sl][4 * dq]) = acc;
     if (dq == 0) red_l[sl] = lsum;
@@ -238,20 +243,22 @@ __global__ void __launch_bounds__(COMBW4_THREADS) combine_warp4_kernel(const Ste
 #pragma unroll 2
     for (int s = g; s < ns; s += 4) {
         const int base = slot_base(s);
-        const float ms = p.part_ml[base * 2];
-        if (ms == -INFINITY) continue;
-        const float w = exp2f(ms - M);
+        // loads first (every slot below ns was written by this step), test after
+        const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + base * 2);
         const float4* src = reinterpret_cast<const float4*>(p.part_o + base * HD + 8 * dl);
         const float4 x = src[0], y = src[1];
-        acc[0] += w * x.x;
-        acc[1] += w * x.y;
-        acc[2] += w * x.z;
-        acc[3] += w * x.w;
-        acc[4] += w * y.x;
-        acc[5] += w * y.y;
-        acc[6] += w * y.z;
-        acc[7] += w * y.w;
-        l += w * p.part_ml[base * 2 + 1];
+        if (ml.x != -INFINITY) {
+            const float w = exp2f(ml.x - M);
+            acc[0] += w * x.x;
+            acc[1] += w * x.y;
+            acc[2] += w * x.z;
+            acc[3] += w * x.w;
+            acc[4] += w * y.x;
+            acc[5] += w * y.y;
+            acc[6] += w * y.z;
+            acc[7] += w * y.w;
+            l += w * ml.y;
+        }
     }
 #pragma unroll
     for (int o = 8; o <= 16; o <<= 1) {  // sum the four slot groups
