@@ -315,6 +315,37 @@ def test_window_bounds_with_verify_block():
     assert np.array_equal(kc.reshape(-1, 128), r.k_cache)
 
 
+@pytest.mark.parametrize("S,L,W", [(0, 40, 0), (30, 40, 16), (5, 37, 7)])
+def test_prefill_block_is_sequential_single_token_steps(S, L, W):
+    # The prefill page's attention over a block of L > 8 new tokens is causal in
+    # the block: token j (position S + j) sees the cached keys and the block's
+    # keys up to itself, inside the window when there is one.  So the block
+    # equals L single-token steps run one after another, each appending its own
+    # row first ("Prefill layer (muse_prefill_layer)", "What to compute").
+    c = _tiny(S, L=L, window=W, rope=W > 0, seed=40 + S + L)
+    r = _run(c)
+    kc, vc = c["kc"].copy(), c["vc"].copy()
+    for j in range(L):
+        cj = dict(c)
+        cj["qkv"] = c["qkv"][j:j + 1]
+        cj["pos"] = c["pos"][j:j + 1]
+        cj["cl"] = c["cl"][j:j + 1]
+        cj["kc"], cj["vc"] = kc, vc
+        rj = _run(cj)
+        assert np.array_equal(rj.out[0], r.out[j])
+        assert np.array_equal(rj.attn[0], r.attn[j])
+        kc, vc = rj.k_cache.reshape(kc.shape), rj.v_cache.reshape(vc.shape)
+    assert np.array_equal(kc.reshape(-1, 128), r.k_cache)
+    assert np.array_equal(vc.reshape(-1, 128), r.v_cache)
+    # the block's first token at position 0 sees only its own key: its
+    # attention output is exactly its own dequantised value row
+    if S == 0:
+        for h in range(16):
+            g = h // 8
+            v0 = _values(r.v_cache[0, 64 * g:64 * g + 64]) * c["s"]
+            assert np.array_equal(r.attn[0, 64 * h:64 * h + 64], v0)
+
+
 def test_page_size_1_and_64_layouts_agree():
     inp = W.make_inputs(W.Spec("t", B=3, L=8, seq_lens=[70, 5, 200], page_size=64,
                                kv_scale=1 / 64, seed=12))
