@@ -67,20 +67,12 @@ __global__ void __launch_bounds__(COMB_THREADS, MINB) combine_kernel(const StepP
     const int slot0 = (c_lo + b) * TL;
     const int stride = p.lt * p.hp, row0 = j * p.hp + h;
     auto slot_base = [&](int s) { return (slot0 + s) * stride + row0; };
-    // 1. global max over the slots
-    float mx = -INFINITY;
-    for (int s = tid; s < ns; s += COMB_THREADS) mx = fmaxf(mx, p.part_ml[slot_base(s) * 2]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) red_m[warp] = mx;
-    __syncthreads();
-    float M = red_m[0];
-#pragma unroll
-    for (int w = 1; w < COMB_THREADS / 32; ++w) M = fmaxf(M, red_m[w]);
-    // 2. weighted sums: thread (sl, dq) over slots sl, sl + 16, ...
+    // 1. weighted sums in one pass: thread (sl, dq) over slots sl, sl + lanes,
+    // ..., each slot lane keeping its own running max (weights <= 1), so no
+    // separate pass over the maxima precedes the sums
     const int sl = tid / 16, dq = tid % 16;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float lsum = 0.f;
+    float lsum = 0.f, mrun = -INFINITY;
     // partials in flight per thread: 4 with the registers of one block per SM
     // (the loop is bound by L2 latency when 16 blocks merge ~1,200 partials each)
 #pragma unroll(MINB == 1 ? 4 : 2)
@@ -91,7 +83,16 @@ __global__ void __launch_bounds__(COMB_THREADS, MINB) combine_kernel(const StepP
         const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + base * 2);
         const float4 o = *reinterpret_cast<const float4*>(p.part_o + base * HD + 4 * dq);
         if (ml.x != -INFINITY) {
-            const float w = exp2f(ml.x - M);
+            if (ml.x > mrun) {  // rescale what this lane has summed so far
+                const float a = exp2f(mrun - ml.x);  // 0 while nothing was summed
+                acc.x *= a;
+                acc.y *= a;
+                acc.z *= a;
+                acc.w *= a;
+                lsum *= a;
+                mrun = ml.x;
+            }
+            const float w = exp2f(ml.x - mrun);
             acc.x += w * o.x;
             acc.y += w * o.y;
             acc.z += w * o.z;
@@ -99,8 +100,21 @@ __global__ void __launch_bounds__(COMB_THREADS, MINB) combine_kernel(const StepP
             lsum += w * ml.y;
         }
     }
+    // 2. block max of the lanes' maxima (a warp holds two slot lanes), then
+    // each lane's sums rescaled to it
+    float mx = fmaxf(mrun, __shfl_xor_sync(0xffffffffu, mrun, 16));
+    if (lane == 0) red_m[warp] = mx;
+    __syncthreads();
+    float M = red_m[0];
+#pragma unroll
+    for (int w = 1; w < COMB_THREADS / 32; ++w) M = fmaxf(M, red_m[w]);
+    const float sc = mrun == -INFINITY ? 0.f : exp2f(mrun - M);
+    acc.x *= sc;
+    acc.y *= sc;
+    acc.z *= sc;
+    acc.w *= sc;
     *reinterpret_cast<float4*>(&red_o[sl][4 * dq]) = acc;
-    if (dq == 0) red_l[sl] = lsum;
+    if (dq == 0) red_l[sl] = lsum * sc;
     __syncthreads();
     // 3. threads 0..63: one output dim each
     if (tid < HD) {
@@ -164,20 +178,27 @@ __global__ void __launch_bounds__(COMBW_THREADS) combine_warp_kernel(const StepP
     const int slot0 = (c_lo + b) * TL;  // slot of partial s: slot0 + s (32-bit row indices)
     const int stride = p.lt * p.hp, row0 = j * p.hp + h;
     auto slot_base = [&](int s) { return (slot0 + s) * stride + row0; };
-    float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, p.part_ml[slot_base(s) * 2]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float o0 = 0.f, o1 = 0.f, l = 0.f;
+    // one pass with a running max (the same for every lane: all lanes walk the
+    // same partials); loads first, test after
+    float o0 = 0.f, o1 = 0.f, l = 0.f, mrun = -INFINITY;
+#pragma unroll 2
     for (int s = 0; s < ns; ++s) {
         const int base = slot_base(s);
-        const float ms = p.part_ml[base * 2];
-        if (ms == -INFINITY) continue;
-        const float w = exp2f(ms - M);
+        const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + base * 2);
         const float2 o = *reinterpret_cast<const float2*>(p.part_o + base * HD + 2 * lane);
-        o0 += w * o.x;
-        o1 += w * o.y;
-        l += w * p.part_ml[base * 2 + 1];
+        if (ml.x != -INFINITY) {
+            if (ml.x > mrun) {
+                const float a = exp2f(mrun - ml.x);  // 0 while nothing was summed
+                o0 *= a;
+                o1 *= a;
+                l *= a;
+                mrun = ml.x;
+            }
+            const float w = exp2f(ml.x - mrun);
+            o0 += w * o.x;
+            o1 += w * o.y;
+            l += w * ml.y;
+        }
     }
     const float a0 = o0 / l * vs, a1 = o1 / l * vs;
     float ss = a0 * a0 + a1 * a1;
@@ -234,12 +255,10 @@ __global__ void __launch_bounds__(COMBW4_THREADS) combine_warp4_kernel(const Ste
     const int slot0 = (c_lo + b) * TL;  // slot of partial s: slot0 + s (32-bit row indices)
     const int stride = p.lt * p.hp, row0 = j * p.hp + h;
     auto slot_base = [&](int s) { return (slot0 + s) * stride + row0; };
-    float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, p.part_ml[slot_base(s) * 2]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    // one pass: each slot group keeps its own running max, rescaled to the
+    // warp's max before the groups are summed
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    float l = 0.f;
+    float l = 0.f, mrun = -INFINITY;
 #pragma unroll 2
     for (int s = g; s < ns; s += 4) {
         const int base = slot_base(s);
@@ -248,7 +267,14 @@ __global__ void __launch_bounds__(COMBW4_THREADS) combine_warp4_kernel(const Ste
         const float4* src = reinterpret_cast<const float4*>(p.part_o + base * HD + 8 * dl);
         const float4 x = src[0], y = src[1];
         if (ml.x != -INFINITY) {
-            const float w = exp2f(ml.x - M);
+            if (ml.x > mrun) {  // rescale what this group has summed so far
+                const float a = exp2f(mrun - ml.x);  // 0 while nothing was summed
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] *= a;
+                l *= a;
+                mrun = ml.x;
+            }
+            const float w = exp2f(ml.x - mrun);
             acc[0] += w * x.x;
             acc[1] += w * x.y;
             acc[2] += w * x.z;
@@ -260,6 +286,13 @@ __global__ void __launch_bounds__(COMBW4_THREADS) combine_warp4_kernel(const Ste
             l += w * ml.y;
         }
     }
+    // the warp's max over the four groups (lanes of a group agree), then rescale
+    float M = fmaxf(mrun, __shfl_xor_sync(0xffffffffu, mrun, 8));
+    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 16));
+    const float sc = mrun == -INFINITY ? 0.f : exp2f(mrun - M);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] *= sc;
+    l *= sc;
 #pragma unroll
     for (int o = 8; o <= 16; o <<= 1) {  // sum the four slot groups
 #pragma unroll
