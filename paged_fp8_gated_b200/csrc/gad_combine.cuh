@@ -9,19 +9,29 @@
 
 namespace gad {
 
+// Three forms of the same merge, chosen by the launcher:
+//   combine_kernel<1024, MINB>  steps of at most 16 (token, group) pairs
+//   combine_kernel<256, 8>      other single-token steps
+//   combine_warp4_kernel        other verify blocks
+//   combine_warp_kernel         prefill blocks
+// Each merges in one pass: a lane keeps a running max over the partials it
+// reads (rescaling its sums when the max rises), and the lanes' sums are
+// rescaled to their common max only when they are added together.
+//
 // ---------------------------------------------------------------------------
 // Kernel 3: merge the partials of each (token, head) and apply the gated
-// output norm.  One block per (token, head), over all ngrp * 16 query heads.  A request covered by many CTAs
-// has many partials (a single 80K-key request spreads over ~1,200), so they
-// are read in parallel: thread (sl, dq) accumulates dims 4dq..4dq+3 over
-// partials sl, sl + lanes, ..., then the slot lanes are summed in shared memory.
+// output norm.  One block per (token, head), over all ngrp * 16 query heads.
+// A request covered by many CTAs has many partials (a single 80K-key request
+// spreads over ~1,200), so they are read in parallel: thread (sl, dq)
+// accumulates dims 4dq..4dq+3 over partials sl, sl + lanes, ..., then the
+// slot lanes are summed in shared memory.
 // ---------------------------------------------------------------------------
 // Block width: 1024 threads (64 slot lanes) for steps with few tokens, whose
 // requests are spread over many CTAs; 256 (16 slot lanes) otherwise.
 // MINB blocks per SM: a grid of at most one block per SM (a 1-token step: 16
-// blocks) runs each block faster with registers to spare (56 a thread); a
+// blocks) runs each block faster with registers to spare (47 a thread); a
 // 16-token step launches 256 blocks of 1024 threads, one wave on 148 SMs only
-// if two fit (32 registers a thread), and so do 8 blocks of 256 threads.
+// if two fit (at most 32 registers a thread), and so do 8 blocks of 256.
 template <int COMB_THREADS, int MINB>
 __global__ void __launch_bounds__(COMB_THREADS, MINB) combine_kernel(const StepParams p) {
     constexpr int COMB_SLOT_LANES = COMB_THREADS / 16;
