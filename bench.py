@@ -655,7 +655,7 @@ def main():
         "data": "synthetic",
         "config": {
             "workload": args.workload, "B": B, "L": L, "heads": [hq, hkv], "page_size": ps,
-            "window": inp["window"], "use_rope": inp["use_rope"],
+            "window": inp["window"], "use_rope": inp["use_rope"], "dist": spec.dist,
             "keys_attended": keys, "kv_bytes_per_step": kv_bytes,
             "parallelism": f"replicas x{world}",
             "l2": "256 MiB write+read before every timed step; KV (per step) also exceeds L2",

@@ -226,33 +226,36 @@ def named(name: str, seed: int = 0) -> Spec:
         # one request at 80,000 cached keys, sliding (window 2048, RoPE) or full
         "decode1_sliding": Spec("decode1_sliding", B=1, L=1, ctx=80000, window=2048,
                                 use_rope=True, seed=seed + 11),
-        "decode1_full": Spec("decode1_full", B=1, L=1, ctx=80000, seed=seed + 12),
+        "decode1_full": Spec("decode1_full", B=1, L=1, ctx=80000, dist="coherent", seed=seed + 12),
         # 32 requests, contexts uniform in [40000, 80000], permuted page-1 table
         "decode32_full": Spec("decode32_full", B=32, L=1, ctx_range=(40000, 80000),
-                              seed=seed + 2),
+                              dist="coherent", seed=seed + 2),
         "decode32_sliding": Spec("decode32_sliding", B=32, L=1, ctx_range=(40000, 80000),
                                  window=2048, use_rope=True, seed=seed + 21),
         # diagnostics for the gather pattern: same step with sequential rows, or 64-key pages
         "decode32_full_seq": Spec("decode32_full_seq", B=32, L=1, ctx_range=(40000, 80000),
-                                  permute=False, seed=seed + 2),
+                                  permute=False, dist="coherent", seed=seed + 2),
         "decode32_full_p64": Spec("decode32_full_p64", B=32, L=1, ctx_range=(40000, 80000),
-                                  page_size=64, seed=seed + 2),
+                                  page_size=64, dist="coherent", seed=seed + 2),
         # the page's load table (section "Shapes"): decode and verify at B = 1, 16,
         # 32, sliding and full; requests of B > 1 loads draw contexts uniformly
-        # from [40000, 80000] like decode32_full
-        "decode16_full": Spec("decode16_full", B=16, L=1, ctx_range=(40000, 80000), seed=seed + 51),
+        # from [40000, 80000] like decode32_full; full layers "dist coherent",
+        # sliding layers "dist soft" (the plain draw), as the table gives them
+        "decode16_full": Spec("decode16_full", B=16, L=1, ctx_range=(40000, 80000), dist="coherent",
+                              seed=seed + 51),
         "decode16_sliding": Spec("decode16_sliding", B=16, L=1, ctx_range=(40000, 80000),
                                  window=2048, use_rope=True, seed=seed + 52),
-        "verify1_full": Spec("verify1_full", B=1, L=8, ctx=80000, seed=seed + 53),
+        "verify1_full": Spec("verify1_full", B=1, L=8, ctx=80000, dist="coherent", seed=seed + 53),
         "verify1_sliding": Spec("verify1_sliding", B=1, L=8, ctx=80000, window=2048,
                                 use_rope=True, seed=seed + 54),
-        "verify32_full": Spec("verify32_full", B=32, L=8, ctx_range=(40000, 80000), seed=seed + 55),
+        "verify32_full": Spec("verify32_full", B=32, L=8, ctx_range=(40000, 80000), dist="coherent",
+                              seed=seed + 55),
         "verify32_sliding": Spec("verify32_sliding", B=32, L=8, ctx_range=(40000, 80000),
                                  window=2048, use_rope=True, seed=seed + 56),
         # 16 requests, 8-token causal verify blocks at 80,000 cached keys
         "verify16_sliding": Spec("verify16_sliding", B=16, L=8, ctx=80000, window=2048,
                                  use_rope=True, seed=seed + 31),
-        "verify16_full": Spec("verify16_full", B=16, L=8, ctx=80000, seed=seed + 32),
+        "verify16_full": Spec("verify16_full", B=16, L=8, ctx=80000, dist="coherent", seed=seed + 32),
         # 64-token pages with shuffled ids, cache scale 1/64, gate N(0, 4)
         "paged_full": Spec("paged_full", B=4, L=8, ctx=65536, page_size=64, kv_scale=1 / 64,
                            gate_std=2.0, seed=seed + 41),
