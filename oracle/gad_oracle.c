@@ -40,6 +40,12 @@
  *     (round to nearest even, saturating to +-448, NaN kept).
  *   - All of the step's cache writes happen before any attention read.
  *
+ * Blocks of more than 8 new tokens per request (the page "Prefill layer
+ * (muse_prefill_layer)", q_len 753 and 16,384, section "What to compute")
+ * are the same formula, causal within the block: token j at position p sees
+ * the cached keys and the block's keys up to p (inside the window when there
+ * is one); the code below is written for any L.
+ *
  * The file also holds the output projection that follows the step in the
  * decoder layer (gado_oproj, at the end).
  *
