@@ -137,6 +137,31 @@ def test_oproj_argument_checks(lib, T, K, N, out, status):
     assert lib.last_error()
 
 
+@pytest.mark.parametrize("over,hidden,o_weight,a,status", [
+    (dict(), 100, FAKE, FAKE, -2),            # hidden not a multiple of 128
+    (dict(), 8192, None, FAKE, -1),
+    (dict(), 8192, FAKE, None, -1),
+    (dict(out=FAKE + 8), 8192, FAKE, FAKE, -3),
+    (dict(L=0), 8192, FAKE, FAKE, -2),
+    (dict(L=65537), 8192, FAKE, FAKE, -2),
+    (dict(B=0), 8192, FAKE, FAKE, -2),
+])
+def test_decode_oproj_argument_checks(lib, over, hidden, o_weight, a, status):
+    # the step with its projection chained: the projection's own checks run
+    # first, on the host, before any launch
+    so = lib.lib()
+    args = _ok_args(**over)
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    st = so.gad_attn_decode_oproj(
+        vp(args["qkv"]), vp(args["positions"]), vp(args["seq_lens"]), vp(args["page_table"]),
+        vp(args["cache_loc"]), vp(args["k_cache"]), vp(args["v_cache"]), vp(args["k_scale"]),
+        vp(args["v_scale"]), args["B"], args["L"], args["max_pages"], args["num_rows"], args["page_size"],
+        args["window"], args["use_rope"], vp(args["out"]), vp(args["workspace"]), args["workspace_bytes"],
+        vp(o_weight), hidden, vp(a), None)
+    assert st == status
+    assert lib.last_error()
+
+
 def test_binding_rejects_cpu_tensors(lib):
     import torch
     x = torch.zeros(1, 2304, dtype=torch.bfloat16)
