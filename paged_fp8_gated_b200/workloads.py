@@ -157,13 +157,17 @@ def make_inputs(spec: Spec) -> dict:
         # Large-logit keys at the window's edges: for every token, the oldest key
         # inside its window and the newest key just outside it copy the token's
         # raw query direction (mean over the KV head's 8 query heads), scaled up.
-        # Meant for layers without RoPE, where that raw direction is the one the
-        # scores see; a window off by one key changes the output completely.
-        assert spec.window > 0, "edges needs a sliding window"
+        # On a full layer the range's edges are its oldest key (0) and its newest
+        # cached key.  Meant for layers without RoPE, where that raw direction is
+        # the one the scores see; a range off by one key changes the output.
         qraw = qkv.float()[:, :hq * D].view(T, hkv, hq // hkv, D).mean(2)  # [T, hkv, 64]
         for t in range(T):
             b = t // L
-            for key in (int(positions[t]) - spec.window + 1, int(positions[t]) - spec.window):
+            if spec.window > 0:
+                edge_keys = (int(positions[t]) - spec.window + 1, int(positions[t]) - spec.window)
+            else:
+                edge_keys = (0, int(seq[b]) - 1)
+            for key in edge_keys:
                 if 0 <= key < int(seq[b]):   # cached keys only
                     row = int(page_table[b, key // ps]) * ps + key % ps
                     kdir = _unit_rms(qraw[t])

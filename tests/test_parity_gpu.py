@@ -28,6 +28,10 @@ SMALL = [
     S("b2_ctx9000_full_s64", B=2, ctx=9000, page_size=64, kv_scale=1 / 64, seed=107),
     S("b4_ctx6000_sliding_v8_p64", B=4, L=8, ctx=6000, window=2048, use_rope=True,
       page_size=64, seed=108),
+    S("b4_ctx6000_sliding_v8_soft_p1", B=4, L=8, ctx=6000, window=2048, use_rope=True, seed=153),
+    S("b4_ctx6000_full_v8_edges", B=4, L=8, ctx=6000, page_size=64, dist="edges", seed=150),
+    S("b4_ctx80k_full_mixed_soft", B=4, ctx_range=(1, 80000), page_size=64, seed=151),
+    S("b4_ctx80k_full_mixed_coherent_p1", B=4, ctx_range=(1, 80000), dist="coherent", seed=152),
     # edge cases
     S("ctx0_and_1", B=3, seq_lens=[0, 1, 2], seed=110),
     S("ctx0_verify", B=2, L=8, seq_lens=[0, 3], seed=111),

@@ -104,6 +104,25 @@ def test_edges_put_the_query_direction_at_the_window_edges():
                 assert float(k[row, g].pow(2).mean().sqrt()) > 2.5   # scaled-up key
 
 
+def test_edges_on_a_full_layer_mark_the_oldest_and_newest_cached_keys():
+    inp = W.make_inputs(W.Spec("ef", B=3, ctx=700, dist="edges", seed=17))
+    pt = inp["page_table"].numpy()
+    seq = inp["seq_lens"].numpy()
+    k = _e4m3_values(inp["k_cache"]).reshape(-1, 2, 64)
+    q = inp["qkv"].float()[:, :16 * 64].view(-1, 2, 8, 64).mean(2)
+    rms = k.pow(2).mean(-1).sqrt()                       # [rows, 2]
+    for b in range(3):
+        for key in (0, int(seq[b]) - 1):
+            row = int(pt[b, key])
+            assert float(rms[row].min()) > 2.5
+            for g in range(2):
+                assert float(torch.nn.functional.cosine_similarity(k[row, g], q[b, g], dim=0)) > 0.95
+    # every other row keeps the plain unit-RMS draw
+    marked = {int(pt[b, key]) for b in range(3) for key in (0, int(seq[b]) - 1)}
+    others = [r for r in range(k.shape[0]) if r not in marked]
+    assert float(rms[others].max()) < 2.0
+
+
 def test_outlier_channels_carry_sixteen_times_the_scale():
     inp = W.make_inputs(W.Spec("o", B=1, L=8, ctx=2000, dist="outliers", seed=8))
     k = _e4m3_values(inp["k_cache"]).reshape(-1, 2, 64).abs().mean(0)   # [2, 64]
