@@ -272,6 +272,98 @@ def test_new_cache_rows_are_quantised_normed_keys():
     assert np.array_equal(r.k_cache[:20], c["kc"][:20].reshape(20, 128))
 
 
+# ----------------------------------------------------------------------------
+# RoPE inside the step ("What to compute": the rotation comes after the
+# QK-norm and before the cache write, at each token's own position)
+# ----------------------------------------------------------------------------
+
+def _rotate_np(u, p):
+    """NeoX half-split rotation written out from its definition: pairs
+    (i, i + 32) turn by the angle p * 10000^(-i/32)."""
+    u = np.asarray(u, np.float64)
+    ang = float(p) * 10000.0 ** (-np.arange(32) / 32.0)
+    c, s = np.cos(ang), np.sin(ang)
+    return np.concatenate([u[:32] * c - u[32:] * s, u[32:] * c + u[:32] * s])
+
+
+@pytest.mark.parametrize("scale", [1.0, 1 / 64])
+def test_new_cache_rows_are_quantised_rotated_keys(scale):
+    # the step writes E4M3(rotate(rmsnorm(k), positions[t]) / scale): rotated
+    # before the quantisation, by the token's own position
+    c = _tiny(1000, L=8, rope=True, kv_scale=scale, seed=90)
+    r = _run(c)
+    kraw = (_bf16_bits(c["qkv"][:, 1024:1152]).astype(np.uint32) << 16).view(np.float32)
+    for t in range(8):
+        p = int(c["pos"][t])
+        row = c["cl"][t]
+        for g in range(2):
+            k = kraw[t, g * 64:(g + 1) * 64].astype(np.float64)
+            kn = k / np.sqrt(np.mean(k * k) + 1e-6)
+            expect = _codes((_rotate_np(kn, p) / scale).astype(np.float32))
+            assert np.array_equal(r.k_cache[row, g * 64:(g + 1) * 64], expect), (t, g)
+            # an unrotated key would differ (the positions are far from 0)
+            assert not np.array_equal(expect, _codes((kn / scale).astype(np.float32)))
+
+
+@pytest.mark.parametrize("aligned", [False, True])
+def test_rope_in_step_closed_form_logits(aligned):
+    """Every query is the unit vector e_1, so after the QK-norm and the x5.473
+    it is qn * e_1 (qn = 5.473 / sqrt(1/64 + 1e-6)), and rotated at position p
+    it is qn * (cos(p f) e_1 + sin(p f) e_33) with f = 10000^(-1/32).  Cached
+    key 0 is a * e_1 and cached key 1 is a * e_33 (stored as they are: cached
+    keys were rotated when they were written), so their logits are
+    qn * a * cos(p f) / 8 and qn * a * sin(p f) / 8.  The block's new keys are
+    either e_5 (orthogonal to every rotated query: logit 0) or e_1 (rotated at
+    the writing token's position p_t, so the logit of token j is
+    qn * (cos(p_j f) K_1 + sin(p_j f) K_33) / 8 with K the dequantised codes of
+    kn * cos(p_t f) and kn * sin(p_t f)).  Two tokens at positions 2 and 3
+    fix that each token's q turns by its own position."""
+    S, L = 2, 2
+    c = _tiny(S, L=L, rope=True, seed=91)
+    a = 8.0 if aligned else 0.25           # both are E4M3 values
+    c["qkv"][:, 0:1024] = 0.0
+    for h in range(16):
+        c["qkv"][:, 64 * h + 1] = 1.0      # q_h = e_1
+    c["qkv"][:, 1024:1152] = 0.0
+    j_new = 1 if aligned else 5
+    c["qkv"][:, 1024 + j_new] = 1.0        # k (both KV heads) = e_1 or e_5
+    c["qkv"][:, 1088 + j_new] = 1.0
+    c["qkv"][:, 1152:1280] = 0.5           # new values 0.5 (an E4M3 value)
+    c["kc"][:] = 0
+    c["kc"][0, :, 1] = _codes([a])[0]
+    c["kc"][1, :, 33] = _codes([a])[0]
+    c["vc"][:] = 0
+    c["vc"][0] = 0x38                      # +1
+    c["vc"][1] = 0xB8                      # -1
+    r = _run(c)
+    qn = 5.473 / math.sqrt(1.0 / 64 + 1e-6)
+    kn = 1.0 / math.sqrt(1.0 / 64 + 1e-6)
+    f = 10000.0 ** (-1.0 / 32.0)
+    new_k = []                             # (K_1, K_33) of each new key, dequantised
+    for t in range(L):
+        pt_ = S + t
+        if aligned:
+            k1, k33 = _values(_codes(np.array([kn * math.cos(pt_ * f), kn * math.sin(pt_ * f)],
+                                              np.float32)))
+        else:
+            k1 = k33 = 0.0
+        new_k.append((float(k1), float(k33)))
+    for j in range(L):
+        p = S + j
+        cs, sn = math.cos(p * f), math.sin(p * f)
+        logits = [qn * a * cs / 8, qn * a * sn / 8]
+        vals = [1.0, -1.0]
+        for t in range(j + 1):             # causal in the block
+            logits.append(qn * (cs * new_k[t][0] + sn * new_k[t][1]) / 8)
+            vals.append(0.5)
+        m = max(logits)
+        w = np.exp(np.array(logits) - m)
+        expect = float(np.dot(w, vals) / w.sum())
+        for h in range(16):
+            got = r.attn[j, 64 * h:64 * h + 64]
+            assert np.allclose(got, expect, rtol=1e-12, atol=1e-15), (j, h, got[0], expect)
+
+
 def test_window_equals_truncated_full_attention():
     # sliding window W (no rope, so positions only set ranges) over 40 cached keys
     # == full attention over a cache that holds only the last W-1 cached keys.
