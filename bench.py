@@ -134,7 +134,20 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def oracle_cpu_rate(inp: dict, max_key_heads: float = 40e6) -> dict:
+def cpu_model() -> str:
+    """The host CPU's model name (first "model name" line of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_cpu_rate(inp: dict, max_key_heads: float = 40e6, threads: int | None = None) -> dict:
     """Time the CPU oracle on a bounded sample of the step and return the rate
     it implies in the bench line's unit (KV-cache GB/s of the whole step).
     Decode and verify steps: a prefix of the requests (all heads and tokens of
@@ -153,7 +166,7 @@ def oracle_cpu_rate(inp: dict, max_key_heads: float = 40e6) -> dict:
     keys = []
     for b in range(B):
         keys.append(int(pos[b, -1]) - int(lo_t[b, 0]) + 1)
-    threads = os.cpu_count() or 1
+    threads = threads or os.cpu_count() or 1
     cache = dict(k_cache=inp["k_cache"].reshape(-1, 64 * hkv),
                  v_cache=inp["v_cache"].reshape(-1, 64 * hkv))
     if L > 8:
@@ -223,7 +236,7 @@ def run_reference(args, rank: int, world: int):
                    "page_size": inp["page_size"], "window": inp["window"],
                    "note": "ms_per_step extrapolated from the sample's GB/s to the whole step"},
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": r["cores"],
-                         "kind": "oracle", "sample": r["sample"]},
+                         "kind": "oracle", "sample": r["sample"], "cpu_model": cpu_model()},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -610,6 +623,11 @@ def main():
         cpu = oracle_cpu_rate(inp)
         cpu.pop("seconds", None)
         cpu["value"] = round(cpu["value"], 4)
+        # the same oracle on one thread, on a smaller prefix of the step
+        one = oracle_cpu_rate(inp, max_key_heads=2.5e6, threads=1)
+        cpu["value_1thread"] = round(one["value"], 4)
+        cpu["sample_1thread"] = one["sample"]
+        cpu["cpu_model"] = cpu_model()
 
     if world > 1:
         dist.barrier()

@@ -45,6 +45,10 @@ SMALL = [
       seed=118),
     S("gate_std2_s64", B=2, L=8, ctx=1500, page_size=64, kv_scale=1 / 64, gate_std=2.0, seed=119),
     S("spare_pages", B=2, seq_lens=[333, 777], page_size=64, spare_pages=5, seed=120),
+    # 16 and 17 single-token requests: the combine kernel's one-wave form and
+    # its 256-thread form
+    S("b16_decode_mixed", B=16, ctx_range=(0, 20000), seed=147),
+    S("b17_decode_mixed", B=17, ctx_range=(0, 20000), seed=148),
     # many requests
     S("b1100_decode_p1", B=1100, ctx_range=(0, 300), seed=123),
     S("b1100_decode_p64_sliding", B=1100, ctx_range=(0, 400), window=100, use_rope=True,
@@ -73,6 +77,8 @@ SMALL_DP = [
       page_size=64, kv_scale=1 / 64, gate_std=2.0, seed=141, **DP),
     S("dp_ctx0_and_ragged_v3", B=3, L=3, seq_lens=[0, 63, 130], page_size=64, seed=142, **DP),
     S("dp_edges_sliding", B=2, L=8, ctx=3000, window=2048, dist="edges", seed=143, **DP),
+    # 2 requests x 8 groups = 16 items (the combine's one-wave form)
+    S("dp_b2_decode", B=2, seq_lens=[700, 4000], page_size=64, seed=146, **DP),
     # 512 requests x 8 groups = 4096 list items, the most one call takes
     S("dp_b512_most_items", B=512, ctx_range=(0, 40), seed=144, **DP),
 ]
@@ -186,7 +192,7 @@ FULL = ["pr1", "decode1_sliding", "decode1_full", "decode32_full", "decode32_sli
         # the rest of the page's twelve scored loads
         "decode16_full", "decode16_sliding", "verify1_full", "verify1_sliding",
         "verify32_full", "verify32_sliding"]
-SAMPLED = {"decode32_full": 24, "verify16_full": 24, "paged_full": 32, "decode16_full": 24,
+SAMPLED = {"verify16_full": 24, "paged_full": 32, "decode16_full": 24,
            "verify1_full": 24, "verify32_full": 24, "verify32_sliding": 48}
 
 
