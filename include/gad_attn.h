@@ -25,9 +25,10 @@
  *
  * All pointers are DEVICE pointers unless stated.  All buffers belong to the
  * caller; the library keeps no state between calls except per-device launch
- * settings.  Calls are asynchronous on `stream`, never synchronise the host,
- * never read device values on the host and never allocate, so they can be
- * captured in a CUDA graph.
+ * settings and the scratch pointer registered for the descriptor form
+ * (gad_attn_set_workspace).  Calls are asynchronous on `stream`, never
+ * synchronise the host, never read device values on the host and never
+ * allocate, so they can be captured in a CUDA graph.
  */
 #ifndef GAD_ATTN_H
 #define GAD_ATTN_H
@@ -65,8 +66,19 @@ typedef enum {
                                  counts other than hq = 8 hkv, hkv = 2, 4, 6 .. */
     GAD_ERR_WORKSPACE = -5,   /* workspace NULL or smaller than required        */
     GAD_ERR_CUDA = -6,        /* a CUDA call or kernel launch failed            */
-    GAD_ERR_DEVICE = -7       /* current device is not compute capability 10.x  */
+    GAD_ERR_DEVICE = -7,      /* current device is not compute capability 10.x  */
+    GAD_ERR_DTYPE = -8,       /* a tensor descriptor has the wrong element type */
+    GAD_ERR_STRIDE = -9       /* a tensor descriptor is not densely packed,
+                                 row-major                                      */
 } gad_status;
+
+/* Bits of a step's status word (gad_attn_step_status, gad_oproj_status).
+ * Every wait inside the kernels is bounded: a kernel whose pipeline stalls
+ * (a wait that does not end within 2 s) gives up, lets the work it has in
+ * flight finish, frees its tensor memory and sets its bit, instead of hanging
+ * the GPU.  The step's outputs are then not valid. */
+#define GAD_STATUS_ATTN_WAIT 1   /* an attention kernel gave up a wait */
+#define GAD_STATUS_OPROJ_WAIT 2  /* the output projection gave up a wait */
 
 /*
  * Bytes of device workspace that gad_attn_decode needs for B requests of L
@@ -91,9 +103,9 @@ size_t gad_attn_workspace_bytes_heads(int B, int L, int hq, int hkv);
  *   qkv         bf16 [T, 2304], row-major, 16-byte aligned.  Columns:
  *               q heads [0,1024), k heads [1024,1152), v heads [1152,1280),
  *               gate [1280,2304); each head 64 contiguous values.
- *   positions   int64 [T]: position p of each token.  Token t attends the
- *               cache keys i with lo <= i <= p, lo = 0 (window == 0) or
- *               max(0, p - window + 1).  Contract: p = seq_lens[b] + j.
+ *   positions   int64 [T]: position p of each token, 0 <= p < 2^31.  Token t
+ *               attends the cache keys i with lo <= i <= p, lo = 0 (window == 0)
+ *               or max(0, p - window + 1).  Contract: p = seq_lens[b] + j.
  *   seq_lens    int32 [B]: keys cached before this step (the serving stack's
  *               lengths).  Accepted for interface compatibility; the ranges
  *               come from `positions`.  May be NULL.
@@ -287,6 +299,104 @@ int gad_attn_decode_noalloc(const void* qkv, const int64_t* positions, const int
                             uint8_t* k_cache, uint8_t* v_cache, const float* k_scale,
                             const float* v_scale, int B, int L, int max_pages, int64_t num_rows,
                             int page_size, int window, int use_rope, void* out, void* stream);
+
+/*
+ * Status of the last step that ran with `workspace` (a step of gad_attn_decode,
+ * gad_attn_decode_heads, gad_attn_prefill, gad_attn_decode_oproj or
+ * gad_attn_decode_t): a cudaMemcpyAsync on `stream` of the step's status word
+ * (GAD_STATUS_* bits, 0 when every wait ended in time) into the HOST int
+ * *status.  Read *status only after `stream` has synchronised.  The word sits at
+ * offset 0 of the workspace; each step's first kernel clears it, so it reports
+ * the latest step only.  workspace == NULL reads the word of the built-in
+ * scratch of gad_attn_decode_noalloc on the current device.  Returns GAD_OK,
+ * GAD_ERR_NULL (status NULL), GAD_ERR_ALIGN or GAD_ERR_CUDA.
+ */
+int gad_attn_step_status(const void* workspace, int* status, void* stream);
+
+/*
+ * Status of the standalone projection (gad_oproj): a cudaMemcpyAsync on
+ * `stream` of its device status word into the HOST int *status, then a clear of
+ * the word, both ordered on `stream`.  The word is one per device, shared by
+ * every gad_oproj call on it, and keeps its bits until this call reads them.
+ * Projections chained to a step (gad_attn_decode_oproj) report into the
+ * step's word instead.  Returns GAD_OK, GAD_ERR_NULL or GAD_ERR_CUDA.
+ */
+int gad_oproj_status(int* status, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Tensor-descriptor form                                                     */
+/* ------------------------------------------------------------------------- */
+
+/* Element types of gad_tensor. */
+typedef enum {
+    GAD_DTYPE_BF16 = 1,
+    GAD_DTYPE_E4M3 = 2,  /* FP8 E4M3 codes, one byte each */
+    GAD_DTYPE_U8 = 3,    /* bytes; accepted for the caches as E4M3 codes */
+    GAD_DTYPE_I32 = 4,
+    GAD_DTYPE_I64 = 5,
+    GAD_DTYPE_F32 = 6
+} gad_dtype;
+
+/* A device tensor: data pointer, element type (gad_dtype), rank 1..4, extents
+ * and strides in elements.  The descriptor is read during the call only; the
+ * memory stays the caller's. */
+typedef struct {
+    void* data;
+    int32_t dtype;
+    int32_t ndim;
+    int64_t shape[4];
+    int64_t stride[4];
+} gad_tensor;
+
+/*
+ * Registers caller-owned device scratch for gad_attn_decode_t on the CURRENT
+ * device (256-byte aligned; NULL unregisters).  The library keeps the pointer
+ * and size, never the memory.  Register it before the steps that use it and
+ * outside any stream capture; steps on one device that overlap on the GPU
+ * share this scratch and race, so run them on one stream (or use
+ * gad_attn_decode with a workspace per stream).  Returns GAD_OK,
+ * GAD_ERR_ALIGN, GAD_ERR_CUDA or GAD_ERR_DEVICE.  Host-only.
+ */
+int gad_attn_set_workspace(void* workspace, size_t bytes);
+
+/*
+ * Bytes of scratch gad_attn_decode_t needs for B requests of L tokens with
+ * `max_pages` page-table entries per request, page size `page_size` and
+ * sliding window `window` (0: full), on the CURRENT device; 0 with
+ * gad_last_error() set on bad arguments.  (On this design the size depends on
+ * B, L and the device's SM count only; the other arguments are checked.)
+ */
+size_t gad_attn_workspace_bytes_t(int B, int L, int max_pages, int page_size, int window);
+
+/*
+ * The step with every array passed as a tensor descriptor: exactly the
+ * arguments of the page's attention call ("What to compute" and the inputs
+ * listed in "Shapes"), with the sizes read from the descriptors and
+ * cross-checked:
+ *
+ *   out         bf16 [B, L, 64 hq]      gives B, L (1..GAD_MAX_PREFILL_L) and hq
+ *   qkv         bf16 [B L, 64 (2 hq + 2 hkv)]   gives hkv
+ *   positions   i64 [B L]
+ *   seq_lens    i32 [B], or NULL (checked, not read: ranges come from positions)
+ *   page_table  i32 [B, max_pages]
+ *   cache_loc   i64 [B L]
+ *   k_cache,    e4m3 (or u8) [num_pages, page_size, hkv, 64]
+ *   v_cache
+ *   k_scale,    f32 [1]
+ *   v_scale
+ *
+ * Every descriptor must be densely packed and row-major.  A wrong element type
+ * returns GAD_ERR_DTYPE, a wrong rank or extent GAD_ERR_SHAPE, a wrong stride
+ * GAD_ERR_STRIDE, a NULL descriptor or data pointer GAD_ERR_NULL, and no
+ * registered scratch GAD_ERR_WORKSPACE, all before any launch; then the call
+ * runs gad_attn_decode_heads (or gad_attn_prefill for L > GAD_MAX_L) on the
+ * registered scratch, with their checks, semantics and errors.
+ */
+int gad_attn_decode_t(const gad_tensor* qkv, const gad_tensor* positions, const gad_tensor* seq_lens,
+                      const gad_tensor* page_table, const gad_tensor* cache_loc,
+                      const gad_tensor* k_cache, const gad_tensor* v_cache,
+                      const gad_tensor* k_scale, const gad_tensor* v_scale, int page_size,
+                      int window, int use_rope, const gad_tensor* out, void* stream);
 
 /* Message for the last nonzero status returned on this host thread. */
 const char* gad_last_error(void);

@@ -55,6 +55,25 @@ _lib.gad_attn_decode_timed.restype = ctypes.c_int
 _lib.gad_attn_decode_timed.argtypes = list(_lib.gad_attn_decode.argtypes) + [_vp]
 _lib.gad_attn_decode_noalloc.restype = ctypes.c_int
 _lib.gad_attn_decode_noalloc.argtypes = list(_lib.gad_attn_decode.argtypes[:17]) + [_vp]
+_lib.gad_attn_step_status.restype = ctypes.c_int
+_lib.gad_attn_step_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_int), _vp]
+_lib.gad_oproj_status.restype = ctypes.c_int
+_lib.gad_oproj_status.argtypes = [ctypes.POINTER(ctypes.c_int), _vp]
+
+
+class GadTensor(ctypes.Structure):
+    """gad_tensor: data pointer, element type code, rank, extents, strides (elements)."""
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 4), ("stride", ctypes.c_int64 * 4)]
+
+
+_GT = ctypes.POINTER(GadTensor)
+_lib.gad_attn_set_workspace.restype = ctypes.c_int
+_lib.gad_attn_set_workspace.argtypes = [_vp, ctypes.c_size_t]
+_lib.gad_attn_workspace_bytes_t.restype = ctypes.c_size_t
+_lib.gad_attn_workspace_bytes_t.argtypes = [ctypes.c_int] * 5
+_lib.gad_attn_decode_t.restype = ctypes.c_int
+_lib.gad_attn_decode_t.argtypes = [_GT] * 9 + [ctypes.c_int] * 3 + [_GT, _vp]
 _lib.gad_last_error.restype = ctypes.c_char_p
 _lib.gad_last_error.argtypes = []
 _lib.gad_status_string.restype = ctypes.c_char_p
@@ -69,7 +88,15 @@ EXPORTED = ("gad_attn_decode", "gad_attn_decode_heads", "gad_attn_decode_timed",
             "gad_attn_decode_heads_timed", "gad_attn_prefill", "gad_attn_prefill_timed",
             "gad_attn_prefill_workspace_bytes", "gad_oproj", "gad_attn_decode_oproj",
             "gad_attn_decode_noalloc", "gad_attn_workspace_bytes",
-            "gad_attn_workspace_bytes_heads", "gad_last_error", "gad_status_string")
+            "gad_attn_workspace_bytes_heads", "gad_last_error", "gad_status_string",
+            "gad_attn_step_status", "gad_oproj_status", "gad_attn_set_workspace",
+            "gad_attn_workspace_bytes_t", "gad_attn_decode_t")
+# gad_dtype codes (include/gad_attn.h)
+DTYPE_BF16, DTYPE_E4M3, DTYPE_U8, DTYPE_I32, DTYPE_I64, DTYPE_F32 = 1, 2, 3, 4, 5, 6
+_DTYPE_CODES = {torch.bfloat16: DTYPE_BF16, torch.uint8: DTYPE_U8, torch.int32: DTYPE_I32,
+                torch.int64: DTYPE_I64, torch.float32: DTYPE_F32}
+if hasattr(torch, "float8_e4m3fn"):
+    _DTYPE_CODES[torch.float8_e4m3fn] = DTYPE_E4M3
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -221,9 +248,17 @@ def attn_decode_noalloc(qkv: torch.Tensor, positions: torch.Tensor,
     T = qkv.shape[0]
     if qkv.shape[1] != QKV_COLS or T != B * L:
         raise ValueError(f"qkv must be [B*L={B * L}, {QKV_COLS}], got {tuple(qkv.shape)}")
+    if positions.numel() != T or cache_loc.numel() != T:
+        raise ValueError("positions and cache_loc need one entry per token")
+    if k_cache.shape != v_cache.shape or k_cache.numel() % ROW_BYTES:
+        raise ValueError(f"k_cache and v_cache must have the same shape, {ROW_BYTES} bytes per row")
     num_rows = k_cache.numel() // ROW_BYTES
     if out is None:
         out = torch.empty(B, L, OUT_COLS, dtype=torch.bfloat16, device=qkv.device)
+    else:
+        _need(out, "out", torch.bfloat16)
+        if out.numel() != T * OUT_COLS:
+            raise ValueError(f"out must hold B*L*{OUT_COLS} values")
     s = (stream or torch.cuda.current_stream(qkv.device)).cuda_stream
     st = _lib.gad_attn_decode_noalloc(
         _ptr(qkv), _ptr(positions), _ptr(seq_lens), _ptr(page_table), _ptr(cache_loc),
@@ -316,3 +351,89 @@ def raw_call(**kw) -> int:
 
 def last_error() -> str:
     return _lib.gad_last_error().decode(errors="replace")
+
+
+# ---------------------------------------------------------------------------
+# Status words and the tensor-descriptor form
+# ---------------------------------------------------------------------------
+
+def step_status(workspace: torch.Tensor | None = None, stream: torch.cuda.Stream | None = None) -> int:
+    """GAD_STATUS_* bits of the last step run with `workspace` (None: the
+    allocation-free entry point's built-in scratch); waits for `stream`."""
+    st = ctypes.c_int(-1)
+    dev = workspace.device if workspace is not None else torch.device("cuda", torch.cuda.current_device())
+    s = stream or torch.cuda.current_stream(dev)
+    rc = _lib.gad_attn_step_status(_ptr(workspace), ctypes.byref(st), ctypes.c_void_p(s.cuda_stream))
+    if rc != 0:
+        raise GadError(rc, "gad_attn_step_status")
+    s.synchronize()
+    return int(st.value)
+
+
+def oproj_status(stream: torch.cuda.Stream | None = None) -> int:
+    """GAD_STATUS_* bits of the standalone projections since the last read (then cleared)."""
+    st = ctypes.c_int(-1)
+    s = stream or torch.cuda.current_stream()
+    rc = _lib.gad_oproj_status(ctypes.byref(st), ctypes.c_void_p(s.cuda_stream))
+    if rc != 0:
+        raise GadError(rc, "gad_oproj_status")
+    s.synchronize()
+    return int(st.value)
+
+
+def tensor_desc(t: torch.Tensor | None, dtype: int | None = None, data: int | None = None,
+                shape=None, stride=None) -> GadTensor | None:
+    """gad_tensor for a torch tensor (its pointer, element type, extents and
+    strides); the keyword overrides let tests describe malformed tensors."""
+    if t is None and data is None:
+        return None
+    d = GadTensor()
+    d.data = data if data is not None else t.data_ptr()
+    d.dtype = dtype if dtype is not None else _DTYPE_CODES.get(t.dtype, 0)
+    shp = list(shape if shape is not None else t.shape)
+    std = list(stride if stride is not None else t.stride())
+    d.ndim = len(shp)
+    for i in range(min(4, len(shp))):
+        d.shape[i] = int(shp[i])
+        d.stride[i] = int(std[i])
+    return d
+
+
+def set_workspace(workspace: torch.Tensor | None) -> None:
+    """Register (None: unregister) the scratch gad_attn_decode_t uses on the current device."""
+    rc = _lib.gad_attn_set_workspace(_ptr(workspace), 0 if workspace is None else int(workspace.numel()))
+    if rc != 0:
+        raise GadError(rc, "gad_attn_set_workspace")
+
+
+def workspace_bytes_t(B: int, L: int, max_pages: int, page_size: int, window: int) -> int:
+    n = _lib.gad_attn_workspace_bytes_t(int(B), int(L), int(max_pages), int(page_size), int(window))
+    if n == 0:
+        raise GadError(-2, "gad_attn_workspace_bytes_t")
+    return int(n)
+
+
+def raw_call_t(descs: dict, page_size: int = 1, window: int = 0, use_rope: int = 0, stream=None) -> int:
+    """gad_attn_decode_t on prepared descriptors (missing names pass NULL); returns the status."""
+    names = ("qkv", "positions", "seq_lens", "page_table", "cache_loc", "k_cache", "v_cache",
+             "k_scale", "v_scale")
+    ptrs = [ctypes.byref(descs[n]) if descs.get(n) is not None else None for n in names]
+    out = descs.get("out")
+    return _lib.gad_attn_decode_t(*ptrs, int(page_size), int(window), int(use_rope),
+                                  ctypes.byref(out) if out is not None else None, stream)
+
+
+def attn_decode_t(qkv, positions, seq_lens, page_table, cache_loc, k_cache, v_cache, k_scale, v_scale,
+                  page_size: int, window: int, use_rope: bool, out: torch.Tensor,
+                  stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+    """The step through the descriptor entry point (scratch from set_workspace):
+    the tensors are described as they are; the library checks them."""
+    descs = dict(qkv=tensor_desc(qkv), positions=tensor_desc(positions), seq_lens=tensor_desc(seq_lens),
+                 page_table=tensor_desc(page_table), cache_loc=tensor_desc(cache_loc),
+                 k_cache=tensor_desc(k_cache), v_cache=tensor_desc(v_cache), k_scale=tensor_desc(k_scale),
+                 v_scale=tensor_desc(v_scale), out=tensor_desc(out))
+    s = (stream or torch.cuda.current_stream(out.device)).cuda_stream
+    rc = raw_call_t(descs, page_size, window, int(bool(use_rope)), ctypes.c_void_p(s))
+    if rc != 0:
+        raise GadError(rc, "gad_attn_decode_t")
+    return out

@@ -20,6 +20,7 @@
 #include <string>
 
 #include "gad_attn.h"
+#include "gad_error.h"
 #include "gad_combine.cuh"
 #include "gad_kernels.cuh"
 #include "gad_oproj.cuh"
@@ -28,10 +29,10 @@
 #include "gad_verify_tc.cuh"
 
 namespace {
-
 thread_local std::string g_last_error;
+}  // namespace
 
-int fail(int status, const char* fmt, ...) {
+int gad_fail(int status, const char* fmt, ...) {
     char buf[512];
     va_list ap;
     va_start(ap, fmt);
@@ -40,6 +41,10 @@ int fail(int status, const char* fmt, ...) {
     g_last_error = buf;
     return status;
 }
+
+namespace {
+
+#define fail gad_fail
 
 constexpr int kMaxCtasPerSm = 2;
 constexpr int kMaxDevices = 64;
@@ -53,8 +58,10 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // Verify blocks (L > 1) run verify_tc_kernel (tcgen05), one CTA per SM.
 constexpr int kV1SingleKG = 4, kV1SingleNS = 3, kV1SingleTK = 128;
 
+// Workspace layout.  The first 256 bytes hold the step's status word (offset
+// 0, read back by gad_attn_step_status); the rest is the step's scratch.
 struct WsLayout {
-    size_t q_off, po_off, pml_off, meta_off, total;
+    size_t status_off, q_off, po_off, pml_off, meta_off, total;
 };
 
 // How a step's tokens and heads become tile-list items.  Blocks longer than
@@ -90,6 +97,8 @@ WsLayout ws_layout(int B, int L, int ngrp, int sms) {
     const size_t T = static_cast<size_t>(B) * L;
     const size_t parts = units * sh.lt * sh.hp;
     size_t off = 0;
+    w.status_off = off;
+    off = align_up(off + sizeof(int));
     w.q_off = off;
     off = align_up(off + T * ngrp * GAD_HQ * GAD_HEAD_DIM * 2);
     w.po_off = off;
@@ -115,6 +124,56 @@ int current_device_sms(int* sms, int* major) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// A driver entry point by name (nullptr if the driver does not export it).
+void* driver_fn(const char* name) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return f;
+}
+
+// Unique id of the calling thread's current CUDA context, 0 if there is none
+// yet or the driver cannot say.  Per-device set-up done once (function
+// attributes, device-symbol addresses) is remembered together with this id,
+// so a new context on the device (after cudaDeviceReset, say) repeats it.
+unsigned long long current_ctx_id() {
+    static std::atomic<PFN_cuCtxGetCurrent_v4000> get_cur{nullptr};
+    static std::atomic<PFN_cuCtxGetId_v12000> get_id{nullptr};
+    PFN_cuCtxGetCurrent_v4000 gc = get_cur.load(std::memory_order_acquire);
+    PFN_cuCtxGetId_v12000 gi = get_id.load(std::memory_order_acquire);
+    if (gc == nullptr || gi == nullptr) {
+        gc = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(driver_fn("cuCtxGetCurrent"));
+        gi = reinterpret_cast<PFN_cuCtxGetId_v12000>(driver_fn("cuCtxGetId"));
+        if (gc == nullptr || gi == nullptr) return 0;
+        get_cur.store(gc, std::memory_order_release);
+        get_id.store(gi, std::memory_order_release);
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (gc(&ctx) != CUDA_SUCCESS || ctx == nullptr || gi(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// One-time set-up per (device, context): `done[dev]` holds the id of the
+// context in which it last ran.
+struct OncePerContext {
+    std::atomic<unsigned long long> done[kMaxDevices];
+    bool is_done(int dev, unsigned long long ctx) const {
+        return ctx != 0 && done[dev].load(std::memory_order_acquire) == ctx;
+    }
+    void mark(int dev) { done[dev].store(current_ctx_id(), std::memory_order_release); }
+};
+
+// The current device index, checked against the per-device tables.
+int current_device(int* dev) {
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (*dev < 0 || *dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", *dev);
+    return GAD_OK;
+}
+
 cudaLaunchAttribute pdl_attr() {
     cudaLaunchAttribute a;
     std::memset(&a, 0, sizeof(a));
@@ -131,17 +190,19 @@ int launch_decode(const gad::StepParams& prm, int sms, int tiles_upper, cudaStre
     const size_t smem = C::smem_bytes(prm.NB);
     // Raise the kernel's dynamic shared-memory limit once per device, to the
     // largest size any item count needs, so no attribute call happens during capture.
-    static std::atomic<bool> attr_done[kMaxDevices];
+    static OncePerContext attr_done;
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", dev);
-    if (!attr_done[dev].load(std::memory_order_acquire)) {
+    {
+        const int ds = current_device(&dev);
+        if (ds != GAD_OK) return ds;
+    }
+    cudaError_t e;
+    if (!attr_done.is_done(dev, current_ctx_id())) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(C::smem_bytes(GAD_MAX_B)));
         if (e != cudaSuccess)
             return fail(GAD_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        attr_done[dev].store(true, std::memory_order_release);
+        attr_done.mark(dev);
     }
     int occ = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, gad::DEC_THREADS, smem);
@@ -174,12 +235,14 @@ int launch_verify_tc(const gad::StepParams& prm, int sms, int tiles_upper, cudaS
     using C = gad::vtc::Cfg<NS>;
     auto kern = gad::verify_tc_kernel<PS, NS, MULTI>;
     const size_t smem = C::smem_bytes(prm.NB);
-    static std::atomic<bool> attr_done[kMaxDevices];
+    static OncePerContext attr_done;
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", dev);
-    if (!attr_done[dev].load(std::memory_order_acquire)) {
+    {
+        const int ds = current_device(&dev);
+        if (ds != GAD_OK) return ds;
+    }
+    cudaError_t e;
+    if (!attr_done.is_done(dev, current_ctx_id())) {
         int optin = 0;
         e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         if (e != cudaSuccess)
@@ -187,7 +250,7 @@ int launch_verify_tc(const gad::StepParams& prm, int sms, int tiles_upper, cudaS
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
         if (e != cudaSuccess)
             return fail(GAD_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        attr_done[dev].store(true, std::memory_order_release);
+        attr_done.mark(dev);
     }
     long long grid = sms;
     if (grid > tiles_upper) grid = tiles_upper;
@@ -209,6 +272,7 @@ int launch_verify_tc(const gad::StepParams& prm, int sms, int tiles_upper, cudaS
 // Whether the 8-stage verify kernel's shared memory, with tables for NB list
 // items, fits in `optin` bytes.
 constexpr int kVtcDeepStages = 8, kVtcShallowStages = 4;
+
 bool verify_deep_fits(int NB, int optin) {
     return gad::vtc::Cfg<kVtcDeepStages>::smem_bytes(NB) <= static_cast<size_t>(optin);
 }
@@ -251,17 +315,19 @@ int launch_prefill_tc(const gad::StepParams& prm, int sms, int tiles_upper, cuda
     using C = gad::ptc::Cfg<kPtcStages>;
     auto kern = gad::prefill_tc_kernel<PS, kPtcStages>;
     const size_t smem = C::smem_bytes(prm.NB);
-    static std::atomic<bool> attr_done[kMaxDevices];
+    static OncePerContext attr_done;
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", dev);
-    if (!attr_done[dev].load(std::memory_order_acquire)) {
+    {
+        const int ds = current_device(&dev);
+        if (ds != GAD_OK) return ds;
+    }
+    cudaError_t e;
+    if (!attr_done.is_done(dev, current_ctx_id())) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(C::smem_bytes(GAD_MAX_B)));
         if (e != cudaSuccess)
             return fail(GAD_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        attr_done[dev].store(true, std::memory_order_release);
+        attr_done.mark(dev);
     }
     long long grid = sms;
     if (grid > tiles_upper) grid = tiles_upper;
@@ -306,6 +372,8 @@ int launch_block(const gad::StepParams& prm, int page_size, bool deep, int sms, 
 // ---------------------------------------------------------------------------
 // Error word of the projection kernel (a bounded wait timed out); the
 // standalone entry point has no workspace to hold it.
+// Status word of the standalone projection (gad_oproj), which has no
+// workspace to hold it; read and cleared by gad_oproj_status.
 __device__ int g_oproj_err;
 
 int encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
@@ -344,27 +412,50 @@ int check_oproj(const void* out, const void* w, const void* a, int T, int K, int
     return GAD_OK;
 }
 
-int launch_oproj(const void* out, const void* w, void* a, int T, int K, int N, cudaStream_t s, bool pdl) {
+// Device address of the standalone projection's status word on the current
+// device (looked up once per context).
+int oproj_status_word(int** out) {
+    static OncePerContext looked_up;
+    static std::atomic<void*> addr[kMaxDevices];
+    int dev = 0;
+    const int ds = current_device(&dev);
+    if (ds != GAD_OK) return ds;
+    if (!looked_up.is_done(dev, current_ctx_id())) {
+        void* ea = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ea, g_oproj_err);
+        if (e != cudaSuccess || ea == nullptr)
+            return fail(GAD_ERR_CUDA, "cudaGetSymbolAddress(status word): %s", cudaGetErrorString(e));
+        addr[dev].store(ea, std::memory_order_release);
+        looked_up.mark(dev);
+    }
+    *out = static_cast<int*>(addr[dev].load(std::memory_order_acquire));
+    return GAD_OK;
+}
+
+// err: the status word the kernel reports a timed-out wait into (the step's
+// workspace word when chained to a step, else the standalone word).
+int launch_oproj(const void* out, const void* w, void* a, int T, int K, int N, cudaStream_t s, bool pdl,
+                 int* err) {
     const int tt = T >= gad::opj::TT_MAX ? gad::opj::TT_MAX : (T + 15) / 16 * 16;
     const int nstg = gad::opj::stages(tt, K / gad::opj::BK);
     if (nstg < 1) return fail(GAD_ERR_SHAPE, "projection ring: %d stages", nstg);  // never launched empty
     const size_t smem = gad::opj::smem_bytes(tt, nstg);
-    static std::atomic<bool> attr_done[kMaxDevices];
-    static std::atomic<void*> err_addr[kMaxDevices];
+    static OncePerContext attr_done;
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", dev);
-    if (!attr_done[dev].load(std::memory_order_acquire)) {
+    {
+        const int ds = current_device(&dev);
+        if (ds != GAD_OK) return ds;
+    }
+    cudaError_t e;
+    if (!attr_done.is_done(dev, current_ctx_id())) {
         e = cudaFuncSetAttribute(gad::oproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(1024 + gad::opj::SMEM_BUDGET + gad::opj::ctrl_bytes()));
         if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        void* ea = nullptr;
-        e = cudaGetSymbolAddress(&ea, g_oproj_err);
-        if (e != cudaSuccess || ea == nullptr)
-            return fail(GAD_ERR_CUDA, "cudaGetSymbolAddress(error word): %s", cudaGetErrorString(e));
-        err_addr[dev].store(ea, std::memory_order_release);
-        attr_done[dev].store(true, std::memory_order_release);
+        attr_done.mark(dev);
+    }
+    if (err == nullptr) {
+        const int es = oproj_status_word(&err);
+        if (es != GAD_OK) return es;
     }
     CUtensorMap wmap, xmap;
     int st = encode_bf16_2d(&wmap, w, static_cast<uint64_t>(K), static_cast<uint64_t>(N), gad::opj::BK,
@@ -381,7 +472,7 @@ int launch_oproj(const void* out, const void* w, void* a, int T, int K, int N, c
     prm.N = N;
     prm.tt = tt;
     prm.nstg = nstg;
-    prm.err = static_cast<int*>(err_addr[dev].load(std::memory_order_acquire));
+    prm.err = err;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>(N / gad::opj::BM), static_cast<unsigned>((T + tt - 1) / tt));
@@ -412,6 +503,8 @@ const char* gad_status_string(int status) {
         case GAD_ERR_WORKSPACE: return "GAD_ERR_WORKSPACE";
         case GAD_ERR_CUDA: return "GAD_ERR_CUDA";
         case GAD_ERR_DEVICE: return "GAD_ERR_DEVICE";
+        case GAD_ERR_DTYPE: return "GAD_ERR_DTYPE";
+        case GAD_ERR_STRIDE: return "GAD_ERR_STRIDE";
         default: return "unknown gad_status";
     }
 }
@@ -506,6 +599,8 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
     prm.part_o = reinterpret_cast<float*>(ws + w.po_off);
     prm.part_ml = reinterpret_cast<float*>(ws + w.pml_off);
     prm.meta = reinterpret_cast<int*>(ws + w.meta_off);
+    prm.status = reinterpret_cast<int*>(ws + w.status_off);
+
     prm.lt = sh.lt;
     prm.tl = L == 1 ? kV1SingleKG : 1;
 
@@ -642,7 +737,7 @@ int gad_attn_decode_heads_timed(const void* qkv, const int64_t* positions,
 int gad_oproj(const void* out, const void* o_weight, void* a, int T, int K, int N, void* stream) {
     const int st = check_oproj(out, o_weight, a, T, K, N);
     if (st != GAD_OK) return st;
-    return launch_oproj(out, o_weight, a, T, K, N, static_cast<cudaStream_t>(stream), false);
+    return launch_oproj(out, o_weight, a, T, K, N, static_cast<cudaStream_t>(stream), false, nullptr);
 }
 
 int gad_attn_decode_oproj(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
@@ -661,7 +756,7 @@ int gad_attn_decode_oproj(const void* qkv, const int64_t* positions, const int32
                   out, workspace, workspace_bytes, stream, nullptr);
     if (st != GAD_OK) return st;
     return launch_oproj(out, o_weight, a, B * L, GAD_OUT_COLS, hidden, static_cast<cudaStream_t>(stream),
-                        true);
+                        true, static_cast<int*>(workspace));  // the step's status word (offset 0)
 }
 
 int gad_attn_prefill(const void* qkv, const int64_t* positions, const int32_t* seq_lens,
@@ -705,24 +800,24 @@ int gad_attn_prefill_timed(const void* qkv, const int64_t* positions, const int3
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) uint8_t g_noalloc_scratch[GAD_NOALLOC_SCRATCH_BYTES];
 
-static std::atomic<void*> g_noalloc_addr[kMaxDevices];
-
 // Device address of g_noalloc_scratch on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
+// array's name is only a host-side stand-in, so the address is looked up with
+// the device current, once per context, and remembered.
 static int noalloc_scratch_address(void** out) {
+    static OncePerContext looked_up;
+    static std::atomic<void*> addr[kMaxDevices];
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices) return fail(GAD_ERR_DEVICE, "device index %d", dev);
-    void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
-    if (p == nullptr) {
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    const int ds = current_device(&dev);
+    if (ds != GAD_OK) return ds;
+    if (!looked_up.is_done(dev, current_ctx_id())) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || p == nullptr)
             return fail(GAD_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-        g_noalloc_addr[dev].store(p, std::memory_order_release);
+        addr[dev].store(p, std::memory_order_release);
+        looked_up.mark(dev);
     }
-    *out = p;
+    *out = addr[dev].load(std::memory_order_acquire);
     return GAD_OK;
 }
 
@@ -748,4 +843,38 @@ extern "C" int gad_attn_decode_noalloc(const void* qkv, const int64_t* positions
                     L, GAD_MAX_L, GAD_HQ, GAD_HKV, max_pages, num_rows, page_size, window,
                     use_rope, out,
                     scratch, static_cast<size_t>(GAD_NOALLOC_SCRATCH_BYTES), stream, nullptr);
+}
+
+// ---------------------------------------------------------------------------
+// Status words: a kernel whose bounded wait gave up (a stalled pipeline) sets
+// a bit in its step's status word instead of hanging; these calls bring the
+// word back to the host.
+// ---------------------------------------------------------------------------
+extern "C" int gad_attn_step_status(const void* workspace, int* status, void* stream) {
+    if (!status) return fail(GAD_ERR_NULL, "status must point to a host int");
+    const void* word = workspace;
+    if (word == nullptr) {
+        void* scratch = nullptr;
+        const int st = noalloc_scratch_address(&scratch);
+        if (st != GAD_OK) return st;
+        word = scratch;
+    } else if (!aligned(workspace, kAlign)) {
+        return fail(GAD_ERR_ALIGN, "workspace must be 256-byte aligned");
+    }
+    cudaError_t e = cudaMemcpyAsync(status, word, sizeof(int), cudaMemcpyDeviceToHost,
+                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "cudaMemcpyAsync(status): %s", cudaGetErrorString(e));
+    return GAD_OK;
+}
+
+extern "C" int gad_oproj_status(int* status, void* stream) {
+    if (!status) return fail(GAD_ERR_NULL, "status must point to a host int");
+    int* word = nullptr;
+    const int st = oproj_status_word(&word);
+    if (st != GAD_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(status, word, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(word, 0, sizeof(int), s);
+    if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "projection status: %s", cudaGetErrorString(e));
+    return GAD_OK;
 }

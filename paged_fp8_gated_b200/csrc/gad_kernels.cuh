@@ -71,7 +71,8 @@ struct StepParams {
     __half* q_ws;    // [T][ngrp][16][64]  normalised (rotated) queries
     float* part_o;   // [slots][lt][16][64]  un-normalised partial outputs (slot = CTA + item)
     float* part_ml;  // [slots][lt][16][2]   (running max in log2 units, sum)
-    int* meta;       // see META_*: tile count, tiles per CTA, error word, tile prefix over items
+    int* meta;       // see META_*: tile count, tiles per CTA, tile prefix over items
+    int* status;     // the step's status word (STATUS_* bits), at offset 0 of the workspace
     double inv_freq[HD / 2];  // RoPE: 10000^(-2i/64) for pair i, computed on the host
     int lt;          // token capacity of one partial slot (1 or 8)
     int tl;          // partials per (CTA, request) and KV-head group
@@ -104,9 +105,14 @@ __device__ __forceinline__ ItemRef item_ref(const StepParams& p, int i) {
 // Layout of StepParams::meta (ints).
 constexpr int META_TOTAL = 0;    // tiles in the step
 constexpr int META_PER = 1;      // tiles per CTA
-constexpr int META_ERROR = 2;    // nonzero: a bounded wait in the decode kernel timed out
 constexpr int META_PREFIX = 3;   // [NB + 1] tile prefix over list items
 constexpr int META_INTS = 4;     // + NB
+
+// Bits of the step's status word.  The step's first kernel clears the word;
+// a kernel whose bounded wait gave up sets its bit at the end, after waiting
+// for the kernel before it (so the clear is always ordered first).
+constexpr int STATUS_ATTN_WAIT = 1;   // an attention kernel's wait timed out
+constexpr int STATUS_OPROJ_WAIT = 2;  // the output projection's wait timed out
 
 // ---------------------------------------------------------------------------
 // Kernel 2: split-KV decode.

@@ -36,7 +36,6 @@ constexpr int NSTG_MAX = 16;              // ring stages at most
 constexpr int SMEM_BUDGET = 200 * 1024;   // bytes of ring per CTA
 constexpr int THREADS = 128;
 constexpr int W_STAGE = BM * BK * 2;      // 16 KB of weight rows per stage
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
 __host__ __device__ constexpr int x_stage(int tt) { return tt * BK * 2; }  // token rows per stage
 __host__ __device__ constexpr int ctrl_bytes() { return 8 * (2 * NSTG_MAX + 1) + 8; }  // barriers, TMEM, flag
@@ -52,18 +51,6 @@ __host__ __device__ constexpr uint32_t tmem_cols(int tt) {  // a power of two >=
     return tt <= 32 ? 32u : tt <= 64 ? 64u : tt <= 128 ? 128u : 256u;
 }
 
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
-            *abort_flag = 1;
-            return false;
-        }
-    }
-}
 
 }  // namespace opj
 
@@ -72,7 +59,7 @@ struct OprojParams {
     int T, K, N;
     int tt;            // tokens per CTA: a multiple of 16, at most 256
     int nstg;          // ring stages (stages(tt, K / BK))
-    int* err;          // set to 1 if a bounded wait timed out
+    int* err;          // status word: STATUS_OPROJ_WAIT is or-ed in if a bounded wait gave up
 };
 
 __global__ void __launch_bounds__(opj::THREADS, 1)
@@ -129,13 +116,21 @@ __global__ void __launch_bounds__(opj::THREADS, 1)
             }
             pdl_wait_primary();
             for (int kc = 0; kc < first; ++kc) tma_load_2d(xbuf + kc * xs, &x_map, kc * BK, t0, FULL(kc));
+            int issued = first;  // stages [0, issued) have their loads in flight or landed
             for (int kc = NSTG; kc < nk; ++kc) {
                 const int s = kc % NSTG;
                 if (!wait_bounded(EMPTY(s), (kc / NSTG - 1) & 1, abort_flag)) break;
                 mbar_arrive_expect_tx(FULL(s), bytes);
                 tma_load_2d(wbuf + s * W_STAGE, &w_map, kc * BK, n0, FULL(s));
                 tma_load_2d(xbuf + s * xs, &x_map, kc * BK, t0, FULL(s));
+                issued = kc + 1;
             }
+            // Every load issued must land before the CTA leaves (its shared
+            // memory is the destination): wait for the last one of each stage,
+            // also after an abort.  Without an abort they have all been
+            // consumed by now and these waits return at once.
+            for (int kc = issued > NSTG ? issued - NSTG : 0; kc < issued; ++kc)
+                wait_bounded(FULL(kc % NSTG), (kc / NSTG) & 1, abort_flag, false, TEARDOWN_LIMIT_NS);
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -158,7 +153,9 @@ __global__ void __launch_bounds__(opj::THREADS, 1)
     }
 
     // ---- epilogue: lane = hidden row, columns = tokens ----
-    const bool done = wait_bounded(DONE, 0, abort_flag);
+    // (every MMA issued, also before an abort, is done before tensor memory is
+    // read or freed)
+    const bool done = wait_bounded(DONE, 0, abort_flag, false, TEARDOWN_LIMIT_NS);
     tc_fence_after();
     if (__all_sync(0xffffffffu, done && !*abort_flag)) {  // warp-uniform: tcgen05.ld is collective
         const int n = n0 + warp * 32 + lane;
@@ -183,7 +180,10 @@ __global__ void __launch_bounds__(opj::THREADS, 1)
         tc_fence_after();
         tc_dealloc(tmem, ncols);
     }
-    if (tid == 0 && *abort_flag) atomicExch(p.err, 1);
+    if (tid == 0 && *abort_flag) {
+        pdl_wait_primary();  // the step's first kernel has cleared the status word
+        atomicOr(p.err, STATUS_OPROJ_WAIT);
+    }
     pdl_launch_dependents();
 }
 

@@ -60,7 +60,6 @@ constexpr uint32_t TM_COLS = 512;            // tensor-memory columns allocated
 constexpr uint32_t TM_Q = 0;                 // Q_w at TM_Q + 32 w (fp16 pairs, 32 columns)
 constexpr uint32_t TM_S = 64;                // S_w buffer b at TM_S + 128 w + 64 b (P aliases its first 32)
 constexpr uint32_t TM_O = 320;               // O_w at TM_O + 64 w
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr float RESCALE_LOG2 = 8.f;          // lazy rescale threshold (P stays <= 2^8)
 
 // mbarrier indices
@@ -90,21 +89,6 @@ struct Cfg {
     static_assert(NBARS * 8 + 8 <= static_cast<int>(CTRL_BYTES), "control block");
 };
 
-// Bounded waits (as in the verify kernel): give up after WAIT_LIMIT_NS or
-// once another thread has raised the abort flag.
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                             bool stop_on_abort = true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (stop_on_abort && *abort_flag) return false;
-        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
-            *abort_flag = 1;
-            return false;
-        }
-    }
-}
 
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
     const bool ok = wait_bounded(bar, parity, abort_flag);
@@ -422,7 +406,7 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
         if (ok && i > 0) issue_pv(i - 1, prev_first, prev_seg);
         // every MMA this warp issued is done before the tensor memory is freed
         tc_commit(BAR(BAR_MMA_DONE));
-        const bool done = wait_bounded(BAR(BAR_MMA_DONE), 0, abort_flag, false);
+        const bool done = wait_bounded(BAR(BAR_MMA_DONE), 0, abort_flag, false, TEARDOWN_LIMIT_NS);
         __syncwarp();
         (void)done;
     } else {
@@ -600,7 +584,10 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
         tc_fence_after();
         tc_dealloc(tmem, TM_COLS);
     }
-    if (tid == 0 && *abort_flag) atomicExch(p.meta + META_ERROR, 1);
+    if (tid == 0 && *abort_flag) {
+        pdl_wait_primary();  // the step's first kernel has cleared the status word
+        atomicOr(p.status, STATUS_ATTN_WAIT);
+    }
     pdl_launch_dependents();
 }
 

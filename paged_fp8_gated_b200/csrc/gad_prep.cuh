@@ -25,7 +25,7 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_kernel(const StepParams p) 
     pdl_launch_dependents();
     const int ng = p.ngrp;
     const int t = blockIdx.x / ng, c = blockIdx.x % ng;
-    if (blockIdx.x == 0 && threadIdx.x == 0) p.meta[META_ERROR] = 0;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.status = 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const __nv_bfloat16* row = p.qkv + static_cast<size_t>(t) * QKV_COLS * ng;
     const bool is_q = warp < HQ;

@@ -56,6 +56,57 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Non-blocking probe of the same phase.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Limits of the bounded waits.  A pipeline wait gives up after WAIT_LIMIT_NS;
+// the last waits of a kernel (for its own tensor-core operations and copies in
+// flight, before it frees tensor memory and exits) use TEARDOWN_LIMIT_NS.
+constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;
+constexpr unsigned long long TEARDOWN_LIMIT_NS = 2000000000ull;
+
+// The library built for the tests of the give-up path (and only that build)
+// defines GAD_TEST_GIVE_UP_AT_FIRST_MISS: there a pipeline wait whose phase has
+// not completed at its first, non-blocking probe gives up at once, so every
+// kernel with such a wait takes its give-up path on every run.
+#ifdef GAD_TEST_GIVE_UP_AT_FIRST_MISS
+constexpr bool kGiveUpAtFirstMiss = true;
+#else
+constexpr bool kGiveUpAtFirstMiss = false;
+#endif
+
+// Wait for phase `parity` of `bar`, giving up after `limit` ns (raising the
+// abort flag), or as soon as another thread has raised it if stop_on_abort.
+// Returns false on giving up.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             bool stop_on_abort = true,
+                                             unsigned long long limit = WAIT_LIMIT_NS) {
+    if (kGiveUpAtFirstMiss && limit == WAIT_LIMIT_NS) {
+        if (mbar_test_wait(bar, parity)) return true;
+        *abort_flag = 1;
+        return false;
+    }
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (stop_on_abort && *abort_flag) return false;
+        if (global_timer_ns() - t0 > limit) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }

@@ -55,7 +55,6 @@ constexpr uint32_t TM_COLS = 512;             // tensor-memory columns allocated
 constexpr uint32_t TM_Q = 0;                  // A operand (fp16 pairs): 64 columns
 constexpr uint32_t TM_S = 64;                 // S buffer b at TM_S + 64 b (P aliases its first 32)
 constexpr uint32_t TM_O = 256;                // O: 128 columns (head 0 dims | head 1 dims)
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 constexpr float RESCALE_LOG2 = 8.f;           // lazy rescale threshold (P stays <= 2^8)
 
 // mbarrier indices
@@ -83,22 +82,6 @@ struct Cfg {
     static_assert(NBARS * 8 + 8 <= static_cast<int>(CTRL_BYTES), "control block");
 };
 
-// Wait for phase `parity` of `bar`, giving up after WAIT_LIMIT_NS or as soon
-// as another thread has flagged an abort.  Returns false on giving up (and
-// raises the abort flag).
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                             bool stop_on_abort = true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (stop_on_abort && *abort_flag) return false;
-        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
-            *abort_flag = 1;
-            return false;
-        }
-    }
-}
 
 // Warp-uniform version: the warp continues only if every lane saw the phase.
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
@@ -444,7 +427,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
         if (ok && i > 0) issue_pv(i - 1, prev_first, prev_seg);
         // every MMA this warp issued is done before the tensor memory is freed
         tc_commit(BAR(BAR_MMA_DONE));
-        const bool done = wait_bounded(BAR(BAR_MMA_DONE), 0, abort_flag, false);
+        const bool done = wait_bounded(BAR(BAR_MMA_DONE), 0, abort_flag, false, TEARDOWN_LIMIT_NS);
         __syncwarp();
         (void)done;
     } else {
@@ -587,7 +570,10 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
         tc_fence_after();
         tc_dealloc(tmem, TM_COLS);
     }
-    if (tid == 0 && *abort_flag) atomicExch(p.meta + META_ERROR, 1);
+    if (tid == 0 && *abort_flag) {
+        pdl_wait_primary();  // the step's first kernel has cleared the status word
+        atomicOr(p.status, STATUS_ATTN_WAIT);
+    }
     pdl_launch_dependents();
 }
 
