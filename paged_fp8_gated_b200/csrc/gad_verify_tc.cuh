@@ -381,13 +381,14 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
             tc_fence_after();
             const uint32_t vbuf = f16_base + (k & 1) * F16_BUF + F16_TILE;
             const uint32_t pa = tmem + TM_S + 64u * (k & 1);
+            const uint32_t av[4] = {pa, pa + 8u, pa + 16u, pa + 24u};
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int ks = 0; ks < TK / 16; ++ks)
-                    tc_mma_ts(tmem + TM_O + 64u * h, pa + 8u * ks,
-                              smem_desc_sw128(vbuf + h * HALF_TILE + ks * 2048), ID_O,
-                              (ks > 0 || !first) ? 1u : 0u);
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t vb = vbuf + h * HALF_TILE;
+                const uint64_t bd[4] = {smem_desc_sw128(vb), smem_desc_sw128(vb + 2048),
+                                        smem_desc_sw128(vb + 4096), smem_desc_sw128(vb + 6144)};
+                tc_mma_ts4(tmem + TM_O + 64u * h, av, bd, ID_O, first ? 0u : 1u);
+            }
             tc_commit(BAR(BAR_KV_FREE + (k & 1)));
             return true;
         };
@@ -411,10 +412,14 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
             const uint32_t kbuf = f16_base + (i & 1) * F16_BUF;
             const uint32_t sd = tmem + TM_S + 64u * (i & 1);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                tc_mma_ts(sd, tmem + TM_Q + 8u * ks,
-                          smem_desc_sw128(kbuf + (ks >> 2) * HALF_TILE + (ks & 3) * 32), ID_S,
-                          ks > 0 ? 1u : 0u);
+            for (int hk = 0; hk < 2; ++hk) {  // the contraction's two KV-head halves, 4 K16 steps each
+                const uint32_t qa = tmem + TM_Q + 32u * hk;
+                const uint32_t aq[4] = {qa, qa + 8u, qa + 16u, qa + 24u};
+                const uint32_t kb = kbuf + hk * HALF_TILE;
+                const uint64_t bd[4] = {smem_desc_sw128(kb), smem_desc_sw128(kb + 32),
+                                        smem_desc_sw128(kb + 64), smem_desc_sw128(kb + 96)};
+                tc_mma_ts4(sd, aq, bd, ID_S, hk > 0 ? 1u : 0u);
+            }
             tc_commit(BAR(BAR_S_FULL + (i & 1)));
             if (i > 0 && !issue_pv(i - 1, prev_first, prev_seg)) {
                 ok = false;
