@@ -44,6 +44,13 @@
 namespace gad {
 namespace ptc {
 
+// Which exponentials of the softmax run on the FMA pipe (exp2_poly): the
+// second weight of every POLY_EVERY-th pair of keys, 1 in 8 of them.  Measured
+// on B200 (kernel us, prefill1_full / 16,384 tokens on 32K): none 647.8 /
+// 5,201.8; 1 in 8 638.0 / 5,019.4; 1 in 4 641.9 / 5,088.6; 1 in 2 699.8 /
+// 5,705.6 (the FMA pipe also carries the softmax's other arithmetic).
+constexpr int POLY_EVERY = 4;
+
 constexpr int TK = 64;                       // keys per tile
 constexpr int THREADS = 352;                 // 11 warps
 constexpr int SM_THREADS = 128;              // one softmax warpgroup
@@ -532,10 +539,13 @@ __global__ void __launch_bounds__(ptc::THREADS, 1) prefill_tc_kernel(const StepP
             float l4[4] = {0.f, 0.f, 0.f, 0.f};
             // this warpgroup's turn on the exponentials of tile i (phase i of TURN_w)
             if (!wait_warp(BAR(BAR_TURN + w), i & 1, abort_flag)) break;
+            // every POLY_EVERY-th pair's second weight on the FMA pipe, the
+            // rest on the MUFU unit, so the two run side by side
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
                 const float p0 = fast_exp2(fmaf(s[2 * c], C2, -mc));
-                const float p1 = fast_exp2(fmaf(s[2 * c + 1], C2, -mc));
+                const float x1 = fmaf(s[2 * c + 1], C2, -mc);
+                const float p1 = c % POLY_EVERY == 0 ? exp2_poly(x1) : fast_exp2(x1);
                 l4[c & 3] += p0 + p1;
                 pk[c] = pack_f16x2(p0, p1);
             }

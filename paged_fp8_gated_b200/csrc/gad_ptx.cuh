@@ -78,6 +78,25 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// 2^x on the FMA pipe, for the softmax weights (x <= 2^7; inputs below -125
+// give 2^-125 instead of a smaller value or 0, which is 0 once rounded to
+// fp16).  x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the
+// low mantissa bits) and f in [-1/2, 1/2]; 2^f is the degree-4 polynomial
+// that interpolates it at the five Chebyshev nodes of [-1/2, 1/2] (relative
+// error below 4e-6 with fp32 Horner steps, far below an fp16 rounding), and n
+// is added to the exponent field.  Lets part of a softmax's exponentials run
+// beside those of the MUFU unit.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.f);
+    const float t = x + 0x1.8p+23f;
+    const float f = x - (t - 0x1.8p+23f);
+    float p = fmaf(0x1.3cbf6p-7f, f, 0x1.ca1ce2p-5f);
+    p = fmaf(p, f, 0x1.ebfa4cp-3f);
+    p = fmaf(p, f, 0x1.62e0c2p-1f);
+    p = fmaf(p, f, 1.0f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
