@@ -116,7 +116,7 @@ size_t gad_attn_workspace_bytes_heads(int B, int L, int hq, int hkv);
  *               request reads a row that another token of this step writes
  *               (except its own block's new keys).
  *   k_cache,    uint8 [num_rows, 2, 64] E4M3 codes, 16-byte aligned, with
- *   v_cache     num_rows = num_pages * page_size.  Rows cache_loc[t] are
+ *   v_cache     num_rows = num_pages * page_size < 2^31.  Rows cache_loc[t] are
  *               overwritten; no other byte is written.
  *   k_scale,    float32 [1] each (device): the caches' dequantisation scales.
  *   v_scale

@@ -227,13 +227,55 @@ int launch_decode(const gad::StepParams& prm, int sms, int tiles_upper, cudaStre
     return GAD_OK;
 }
 
+// cuTensorMapEncodeTiled, looked up once through the runtime.
+int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> encode{nullptr};
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode.load(std::memory_order_acquire);
+    if (fn == nullptr) {
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(driver_fn("cuTensorMapEncodeTiled"));
+        if (fn == nullptr) return fail(GAD_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+        encode.store(fn, std::memory_order_release);
+    }
+    *out = fn;
+    return GAD_OK;
+}
+
+// A cache (K or V) as a 2D byte tensor of num_rows rows of row_bytes, read in
+// tiles of one 64-row page x 128 bytes (one head group) with the 128-byte
+// swizzle.
+int encode_cache_pages(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t num_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    const int st = tensor_map_encoder(&fn);
+    if (st != GAD_OK) return st;
+    const cuuint64_t dims[2] = {row_bytes, num_rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {128, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(GAD_ERR_CUDA, "cuTensorMapEncodeTiled (cache pages) failed (%d)", static_cast<int>(r));
+    return GAD_OK;
+}
+
 // Verify blocks (L > 1) on the tcgen05 kernel: one CTA per SM; as many raw
 // stages as the shared memory leaves room for next to the per-request tables.
+// Page size 64: each tile's K and V pages are read by TMA tile loads.
 template <int PS, int NS, bool MULTI>
 int launch_verify_tc(const gad::StepParams& prm, int sms, int tiles_upper, cudaStream_t stream,
                      bool pdl) {
     using C = gad::vtc::Cfg<NS>;
     auto kern = gad::verify_tc_kernel<PS, NS, MULTI>;
+    CUtensorMap kmap, vmap;
+    std::memset(&kmap, 0, sizeof(kmap));
+    std::memset(&vmap, 0, sizeof(vmap));
+    if (PS == 64) {
+        const uint64_t row_bytes = static_cast<uint64_t>(GAD_ROW_BYTES) * prm.ngrp;
+        int st = encode_cache_pages(&kmap, prm.k_cache, row_bytes, static_cast<uint64_t>(prm.num_rows));
+        if (st != GAD_OK) return st;
+        st = encode_cache_pages(&vmap, prm.v_cache, row_bytes, static_cast<uint64_t>(prm.num_rows));
+        if (st != GAD_OK) return st;
+    }
     const size_t smem = C::smem_bytes(prm.NB);
     static OncePerContext attr_done;
     int dev = 0;
@@ -264,7 +306,7 @@ int launch_verify_tc(const gad::StepParams& prm, int sms, int tiles_upper, cudaS
     cudaLaunchAttribute attr = pdl_attr();
     cfg.attrs = &attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kern, prm);
+    e = cudaLaunchKernelEx(&cfg, kern, prm, kmap, vmap);
     if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "verify launch: %s", cudaGetErrorString(e));
     return GAD_OK;
 }
@@ -378,17 +420,9 @@ __device__ int g_oproj_err;
 
 int encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
                    uint32_t box_outer) {
-    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> encode{nullptr};
-    PFN_cuTensorMapEncodeTiled_v12000 fn = encode.load(std::memory_order_acquire);
-    if (fn == nullptr) {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
-        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || f == nullptr)
-            return fail(GAD_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
-        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-        encode.store(fn, std::memory_order_release);
-    }
+    PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    const int st = tensor_map_encoder(&fn);
+    if (st != GAD_OK) return st;
     const cuuint64_t dims[2] = {inner, outer};
     const cuuint64_t strides[1] = {inner * 2};
     const cuuint32_t box[2] = {box_inner, box_outer};
@@ -545,6 +579,8 @@ static int run_step(const void* qkv, const int64_t* positions, const int32_t* pa
                     static_cast<long long>(num_rows));
     if (static_cast<long long>(max_pages) * page_size > INT32_MAX)
         return fail(GAD_ERR_SHAPE, "max_pages * page_size exceeds 2^31");
+    if (num_rows > INT32_MAX)
+        return fail(GAD_ERR_SHAPE, "num_rows=%lld exceeds 2^31", static_cast<long long>(num_rows));
     if (window < 0) return fail(GAD_ERR_UNSUPPORTED, "window=%d < 0", window);
     if (!aligned(qkv, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
         return fail(GAD_ERR_ALIGN, "qkv, out, k_cache and v_cache must be 16-byte aligned");

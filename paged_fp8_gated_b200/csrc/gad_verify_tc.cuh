@@ -36,6 +36,8 @@
 // its tensor memory).
 #pragma once
 
+#include <cuda.h>
+
 #include "gad_kernels.cuh"
 #include "gad_tc.cuh"
 
@@ -64,7 +66,8 @@ constexpr int BAR_S_FULL = 4;     // [2] S of the tile in tensor memory         
 constexpr int BAR_P_FULL = 6;     // [2] P of the tile in tensor memory          (128 softmax arrivals)
 constexpr int BAR_O_FREE = 8;     // O read out at a request's last tile         (128 softmax arrivals)
 constexpr int BAR_MMA_DONE = 9;   // teardown: all MMAs done                     (MMA commit)
-constexpr int NBARS = 10;
+constexpr int BAR_RAW = 10;       // [NS] page size 64: the tile's K and V pages landed (TMA bytes)
+constexpr int NBARS = 10;         // + NS for page size 64
 
 template <int NS>
 struct Cfg {
@@ -72,14 +75,14 @@ struct Cfg {
     static constexpr size_t RAW_BYTES = static_cast<size_t>(NS) * RAW_STAGE;
     static constexpr int IDX_SLOTS = 2 * NS;
     static constexpr size_t IDX_BYTES = static_cast<size_t>(IDX_SLOTS) * TK * 4;
-    static constexpr size_t CTRL_BYTES = 128;  // barriers, tensor-memory base, abort flag
+    static constexpr size_t CTRL_BYTES = 256;  // barriers, tensor-memory base, abort flag
     // + 1024 so the swizzled tiles can start on a 1024-byte boundary
     static size_t smem_bytes(int B) {
         return 1024 + F16_BYTES + RAW_BYTES + IDX_BYTES + CTRL_BYTES +
                static_cast<size_t>(4 * B + 1) * 4;
     }
     static_assert(NS >= 3, "stages");
-    static_assert(NBARS * 8 + 8 <= static_cast<int>(CTRL_BYTES), "control block");
+    static_assert((NBARS + NS) * 8 + 8 <= static_cast<int>(CTRL_BYTES), "control block");
 };
 
 
@@ -93,7 +96,11 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
 
 // MULTI: more than one head group (see decode_kernel).
 template <int PS, int NS, bool MULTI>
-__global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepParams p) {
+// kmap, vmap (page size 64): the K and V caches as 2D tensors of 128 ngrp-byte
+// rows, read one 64-row page per TMA tile load (unused for page size 1).
+__global__ void __launch_bounds__(vtc::THREADS, 1)
+    verify_tc_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
+                     const __grid_constant__ CUtensorMap vmap) {
     using namespace vtc;
     using C = Cfg<NS>;
     extern __shared__ uint8_t smem_raw[];
@@ -103,8 +110,8 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
     uint8_t* raw = smem + C::F16_BYTES;                      // [NS][K rows, V rows]
     int* idx_smem = reinterpret_cast<int*>(raw + C::RAW_BYTES);
     uint8_t* ctrl = reinterpret_cast<uint8_t*>(idx_smem) + C::IDX_BYTES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + NBARS * 8);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + NBARS * 8 + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + (NBARS + NS) * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + (NBARS + NS) * 8 + 4);
     int* tpre = reinterpret_cast<int*>(ctrl + C::CTRL_BYTES);
     int* rlo = tpre + p.NB + 1;
     int* rhi = rlo + p.NB;
@@ -131,6 +138,8 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
         mbar_init(BAR(BAR_P_FULL + 1), 128);
         mbar_init(BAR(BAR_O_FREE), 128);
         mbar_init(BAR(BAR_MMA_DONE), 1);
+        if (PS == 64)
+            for (int st = 0; st < NS; ++st) mbar_init(BAR(BAR_RAW + st), 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -220,12 +229,29 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 }
             }
         };
+        int n_kv_issued = 0;  // tiles whose gathers were issued (the same count in every loader)
         auto issue_kv = [&](const Cur& c) {
             if (c.tau >= t1) return;
             const int k0 = c.k0;
             if (k0 + TK - 1 >= c.rnew) ensure_prep();
             const int* ix = idx_smem + ((c.tau - t0) % C::IDX_SLOTS) * TK;
             const uint32_t base = smem_addr(raw + ((c.tau - t0) % NS) * RAW_STAGE);
+            ++n_kv_issued;
+            if constexpr (PS == 64) {
+                // the tile is one page: its K and V rows by two TMA tile loads
+                // (128-byte swizzle, the layout the gathers below write); a page
+                // index past the table (-1) or rows past the cache fall outside the
+                // tensor and read as zeros
+                if (ltid == 0) {
+                    const int pg = ix[0];
+                    const int y = pg >= 0 ? pg * PS : -PS;
+                    const uint32_t bar = BAR(BAR_RAW + (c.tau - t0) % NS);
+                    mbar_arrive_expect_tx(bar, RAW_STAGE);
+                    tma_load_2d(base, &kmap, static_cast<int>(c.gofs), y, bar);
+                    tma_load_2d(base + TK * ROWB, &vmap, static_cast<int>(c.gofs), y, bar);
+                }
+                return;
+            }
             const int lo = c.lo, hi = c.hi;
             const size_t row_pitch = static_cast<size_t>(ROWB) * ng;
             const size_t gofs = c.gofs;
@@ -288,13 +314,20 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
             tc_st32(ta + (g == 0 ? 32u : 0u), z);
         };
         // raw stage -> fp16 tile: thread = (K or V, row r); 16 codes -> two 16-byte fp16 chunks.
-        auto convert = [&](int stage, int buf) {
+        // With page size 64 whole pages arrive, so keys outside the item's range
+        // [lo, hi] (slots of the page not yet written, or before a window) are
+        // converted as zeros, as the page-size-1 gathers zero-fill them.
+        auto convert = [&](int stage, int buf, int k0, int lo, int hi) {
             const int kv = ltid >> 6, r = ltid & 63;
             const uint32_t src = smem_addr(raw + stage * RAW_STAGE) + kv * TK * ROWB + r * ROWB;
             const uint32_t dst = smem_addr(f16 + buf * F16_BUF) + kv * F16_TILE + r * 128;
             uint4 w[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) w[j] = lds128(src + ((j ^ (r & 7)) << 4));
+            if (PS == 64 && (k0 + r < lo || k0 + r > hi)) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) w[j] = make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const uint32_t row = dst + (j >> 2) * HALF_TILE;
@@ -333,11 +366,13 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
         }
         int seg_b = -1;
         const int n_tiles = t1 - t0;
-        for (int i = 0; i < n_tiles; ++i) {
+        int i = 0;
+        for (; i < n_tiles; ++i) {
             cp_async_wait<NS - 2>();
             const int cb = cc.b;
             const bool seg_start = cb != seg_b;
             bool bad = false;
+            if (PS == 64) bad = !wait_bounded(BAR(BAR_RAW + i % NS), (i / NS) & 1, abort_flag);
             // buffers i & 1 are free once PV(i - 2) is done (which also means every
             // S MMA up to tile i - 1 is done, so the A operand may be replaced)
             if (i >= 2) bad = !wait_bounded(BAR(BAR_KV_FREE + (i & 1)), ((i - 2) >> 1) & 1, abort_flag);
@@ -349,7 +384,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
                 write_q(cb);
                 seg_b = cb;
             }
-            convert(i % NS, i & 1);
+            convert(i % NS, i & 1, cc.k0, cc.lo, cc.hi);
             fence_proxy_async_smem();
             if (seg_start) {
                 tc_wait_st();
@@ -366,6 +401,12 @@ __global__ void __launch_bounds__(vtc::THREADS, 1) verify_tc_kernel(const StepPa
             cur_next(cc);
         }
         cp_async_wait<0>();
+        if (PS == 64 && ltid == 0) {
+            // every page load issued lands before the CTA leaves (its shared
+            // memory is the destination); without an abort they all have
+            for (int tile = i; tile < n_kv_issued; ++tile)
+                wait_bounded(BAR(BAR_RAW + tile % NS), (tile / NS) & 1, abort_flag, false, TEARDOWN_LIMIT_NS);
+        }
     }
     else if (warp == MMA_WARP) {
         // =================== MMA issue (whole warp, one elected lane issues) ===================
