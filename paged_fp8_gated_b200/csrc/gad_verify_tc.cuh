@@ -45,10 +45,12 @@ namespace gad {
 namespace vtc {
 
 constexpr int TK = 64;                        // keys per tile
-constexpr int THREADS = 288;                  // 9 warps
-constexpr int LOAD_T0 = 128;                  // first loader thread (warp 4)
+constexpr int SOFT = 256;                     // softmax threads: warps 0-7, two per row
+constexpr int THREADS = 416;                  // 13 warps
+constexpr int LOAD_T0 = SOFT;                 // first loader thread (warp 8)
+constexpr int LOAD_W0 = LOAD_T0 / 32;
 constexpr int LOADERS = 128;
-constexpr int MMA_WARP = 8;
+constexpr int MMA_WARP = 12;
 constexpr int RAW_STAGE = 2 * TK * ROWB;      // 16 KB: 64 K rows then 64 V rows (E4M3)
 constexpr int HALF_TILE = TK * 128;           // one head of a converted tile: 64 keys x 64 fp16
 constexpr int F16_TILE = 2 * HALF_TILE;       // both heads: 16 KB
@@ -63,8 +65,8 @@ constexpr float RESCALE_LOG2 = 8.f;           // lazy rescale threshold (P stays
 constexpr int BAR_KV_READY = 0;   // [2] converted tile (and A operand) ready   (128 loader arrivals)
 constexpr int BAR_KV_FREE = 2;    // [2] PV of the tile done: buffers free       (MMA commit)
 constexpr int BAR_S_FULL = 4;     // [2] S of the tile in tensor memory          (MMA commit)
-constexpr int BAR_P_FULL = 6;     // [2] P of the tile in tensor memory          (128 softmax arrivals)
-constexpr int BAR_O_FREE = 8;     // O read out at a request's last tile         (128 softmax arrivals)
+constexpr int BAR_P_FULL = 6;     // [2] P of the tile in tensor memory          (256 softmax arrivals)
+constexpr int BAR_O_FREE = 8;     // O read out at a request's last tile         (256 softmax arrivals)
 constexpr int BAR_MMA_DONE = 9;   // teardown: all MMAs done                     (MMA commit)
 constexpr int BAR_RAW = 10;       // [NS] page size 64: the tile's K and V pages landed (TMA bytes)
 constexpr int NBARS = 10;         // + NS for page size 64
@@ -76,9 +78,10 @@ struct Cfg {
     static constexpr int IDX_SLOTS = 2 * NS;
     static constexpr size_t IDX_BYTES = static_cast<size_t>(IDX_SLOTS) * TK * 4;
     static constexpr size_t CTRL_BYTES = 256;  // barriers, tensor-memory base, abort flag
+    static constexpr size_t RED_BYTES = 3 * 2 * 128 * 4;  // softmax pairs: maxima [2 tiles][2 halves], sums
     // + 1024 so the swizzled tiles can start on a 1024-byte boundary
     static size_t smem_bytes(int B) {
-        return 1024 + F16_BYTES + RAW_BYTES + IDX_BYTES + CTRL_BYTES +
+        return 1024 + F16_BYTES + RAW_BYTES + IDX_BYTES + CTRL_BYTES + RED_BYTES +
                static_cast<size_t>(4 * B + 1) * 4;
     }
     static_assert(NS >= 3, "stages");
@@ -112,7 +115,9 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
     uint8_t* ctrl = reinterpret_cast<uint8_t*>(idx_smem) + C::IDX_BYTES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + (NBARS + NS) * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + (NBARS + NS) * 8 + 4);
-    int* tpre = reinterpret_cast<int*>(ctrl + C::CTRL_BYTES);
+    float* red = reinterpret_cast<float*>(ctrl + C::CTRL_BYTES);  // [2 tiles][2 halves][128 rows] maxima
+    float* redl = red + 4 * 128;                                   // [2 halves][128 rows] sums
+    int* tpre = reinterpret_cast<int*>(ctrl + C::CTRL_BYTES + C::RED_BYTES);
     int* rlo = tpre + p.NB + 1;
     int* rhi = rlo + p.NB;
     int* rnew = rhi + p.NB;
@@ -134,9 +139,9 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
         mbar_init(BAR(BAR_KV_FREE + 1), 1);
         mbar_init(BAR(BAR_S_FULL), 1);
         mbar_init(BAR(BAR_S_FULL + 1), 1);
-        mbar_init(BAR(BAR_P_FULL), 128);
-        mbar_init(BAR(BAR_P_FULL + 1), 128);
-        mbar_init(BAR(BAR_O_FREE), 128);
+        mbar_init(BAR(BAR_P_FULL), SOFT);
+        mbar_init(BAR(BAR_P_FULL + 1), SOFT);
+        mbar_init(BAR(BAR_O_FREE), SOFT);
         mbar_init(BAR(BAR_MMA_DONE), 1);
         if (PS == 64)
             for (int st = 0; st < NS; ++st) mbar_init(BAR(BAR_RAW + st), 1);
@@ -169,7 +174,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
     auto tile_k0 = [&](int tau, int b) { return (rlo[b] / TK + (tau - tpre[b])) * TK; };
     const float C2 = __ldg(p.k_scale) * 0.125f * 1.4426950408889634f;  // raw score -> log2 units
 
-    if (warp >= 4 && warp < 8) {
+    if (warp >= LOAD_W0 && warp < MMA_WARP) {
         // =================== loaders: gather, convert, A operand ===================
         const int ltid = tid - LOAD_T0;
         bool prep_done = false;
@@ -309,7 +314,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < 32; ++c) q[c] = 0u;
             }
-            const uint32_t ta = tmem + TM_Q + (static_cast<uint32_t>(32 * (warp - 4)) << 16);
+            const uint32_t ta = tmem + TM_Q + (static_cast<uint32_t>(32 * (warp - LOAD_W0)) << 16);
             tc_st32(ta + (g == 0 ? 0u : 32u), q);
             tc_st32(ta + (g == 0 ? 32u : 0u), z);
         };
@@ -477,13 +482,20 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
         __syncwarp();
         (void)done;
     } else {
-        // =================== softmax: one thread per row ===================
-        const int r = tid;
+        // =================== softmax: two threads per row ===================
+        // Warps w and w + 4 share the tensor-memory lanes of rows 32 (w % 4) ..
+        // + 31 and take 32 keys each; the pair posts its halves' maxima through
+        // shared memory (double-buffered by tile parity) and meets at a named
+        // barrier that also ORs a give-up flag, so both warps of a pair always
+        // stop at the same point.
+        const int half = warp >> 2, qd = warp & 3;
+        const int r = 32 * qd + (tid & 31);
         const int g = r >> 6, j = (r >> 3) & 7, qh = g * GRP + (r & 7);
-        const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
+        const int pair_bar = 2 + qd;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
         int ct = t0, cb = find_req(t0);
         int seg_b = -1, seg_t1 = 0, k0 = 0;  // current request, end of its tiles here, tile key
-        float m_run = -INFINITY, l_run = 0.f;
+        float m_run = -INFINITY, l_run = 0.f;  // running max (raw score units), this half's sum
         int lo_j = INT_MAX, hi_j = -1;
         int seg_len = 0;  // tokens of the current item
         for (int i = 0; ct < t1; ++i) {
@@ -509,32 +521,37 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             }
             const bool seg_end = ct + 1 >= seg_t1;
 
-            if (!wait_warp(BAR(BAR_S_FULL + (i & 1)), (i >> 1) & 1, abort_flag)) break;
+            bool bad = !wait_warp(BAR(BAR_S_FULL + (i & 1)), (i >> 1) & 1, abort_flag);
             tc_fence_after();
             const uint32_t sbuf = tmem + TM_S + 64u * (i & 1) + lane_base;
-            uint32_t sr[64];
-            tc_ld32(sbuf, sr);
-            tc_ld32(sbuf + 32u, sr + 32);
+            uint32_t sr[32];
+            tc_ld32(sbuf + 32u * half, sr);
             tc_wait_ld();
-            float s[64];
-            const int cmin = lo_j == INT_MAX ? TK : lo_j - k0;
-            const int cmax = hi_j - k0;
+            float s[32];
+            const int kb0 = k0 + 32 * half;
+            const int cmin = lo_j == INT_MAX ? 32 : lo_j - kb0;
+            const int cmax = hi_j - kb0;
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            if (cmin <= 0 && cmax >= TK - 1) {
+            if (cmin <= 0 && cmax >= 31) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
+                for (int c = 0; c < 32; ++c) {
                     s[c] = __uint_as_float(sr[c]);
                     m4[c & 3] = fmaxf(m4[c & 3], s[c]);
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
+                for (int c = 0; c < 32; ++c) {
                     s[c] = (c < cmin || c > cmax) ? -INFINITY : __uint_as_float(sr[c]);
                     m4[c & 3] = fmaxf(m4[c & 3], s[c]);
                 }
             }
-            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            // lazy rescale: O (in tensor memory) is corrected only when the max grows a lot
+            float* redm = red + (i & 1) * 2 * 128;
+            redm[half * 128 + r] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            // both halves have read their S (P may overwrite the buffer) and posted their maxima
+            if (bar_red_or(pair_bar, 64, bad)) break;
+            const float mx = fmaxf(redm[r], redm[128 + r]);
+            // lazy rescale: O (in tensor memory) is corrected only when the max
+            // grows a lot; both halves of a row take the same decision
             const float m_new = fmaxf(m_run, mx);
             bool corr = false;
             if (m_new > m_run) {
@@ -546,59 +563,63 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             }
             if (__any_sync(0xffffffffu, corr)) {
                 // PV(i - 1) of this request must be done before O is touched
-                if (!wait_warp(BAR(BAR_KV_FREE + ((i - 1) & 1)), ((i - 1) >> 1) & 1, abort_flag)) break;
-                tc_fence_after();
+                const bool ok = wait_warp(BAR(BAR_KV_FREE + ((i - 1) & 1)), ((i - 1) >> 1) & 1, abort_flag);
                 const float alpha = corr ? fast_exp2((m_run - m_new) * C2) : 1.f;
-                const uint32_t oa = tmem + TM_O + 64u * g + lane_base;
-                uint32_t o[32];
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tc_ld32(oa + 32u * half, o);
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t oa = tmem + TM_O + 64u * g + 32u * half + lane_base;
+                    uint32_t o[32];
+                    tc_ld32(oa, o);
                     tc_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                    tc_st32(oa + 32u * half, o);
+                    tc_st32(oa, o);
+                    tc_wait_st();
                 }
-                tc_wait_st();
+                bad = bad || !ok;
                 if (corr) {
                     l_run *= alpha;
                     m_run = m_new;
                 }
             }
             const float mc = m_run == -INFINITY ? 0.f : m_run * C2;
-            uint32_t pk[32];
+            uint32_t pk[16];
             float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
+            for (int c = 0; c < 16; ++c) {
                 const float p0 = fast_exp2(fmaf(s[2 * c], C2, -mc));
                 const float p1 = fast_exp2(fmaf(s[2 * c + 1], C2, -mc));
                 l4[c & 3] += p0 + p1;
                 pk[c] = pack_f16x2(p0, p1);
             }
             l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            tc_st32(sbuf, pk);
+            tc_st16(sbuf + 16u * half, pk);  // P of keys 32 half .. + 31: columns 16 half .. + 15
             tc_wait_st();
             tc_fence_before();
             mbar_arrive(BAR(BAR_P_FULL + (i & 1)));
 
             if (seg_end) {
-                if (!wait_warp(BAR(BAR_KV_FREE + (i & 1)), (i >> 1) & 1, abort_flag)) break;
+                const bool ok = wait_warp(BAR(BAR_KV_FREE + (i & 1)), (i >> 1) & 1, abort_flag);
+                redl[half * 128 + r] = l_run;
+                // both halves' sums posted
+                if (bar_red_or(pair_bar, 64, bad || !ok)) break;
                 tc_fence_after();
-                const uint32_t oa = tmem + TM_O + 64u * g + lane_base;
-                uint32_t o[64];
+                const uint32_t oa = tmem + TM_O + 64u * g + 32u * half + lane_base;
+                uint32_t o[32];
                 tc_ld32(oa, o);
-                tc_ld32(oa + 32u, o + 32);
                 tc_wait_ld();
                 if (j < seg_len) {
                     const size_t slot = static_cast<size_t>(blockIdx.x) + cb;
                     const size_t base = (slot * p.lt + j) * HQ + qh;
-                    float4* dst = reinterpret_cast<float4*>(p.part_o + base * HD);
+                    float4* dst = reinterpret_cast<float4*>(p.part_o + base * HD + 32 * half);
 #pragma unroll
-                    for (int q = 0; q < 16; ++q)
+                    for (int q = 0; q < 8; ++q)
                         dst[q] = make_float4(__uint_as_float(o[4 * q]), __uint_as_float(o[4 * q + 1]),
                                              __uint_as_float(o[4 * q + 2]), __uint_as_float(o[4 * q + 3]));
-                    p.part_ml[base * 2 + 0] = m_run * C2;
-                    p.part_ml[base * 2 + 1] = l_run;
+                    if (half == 0) {
+                        p.part_ml[base * 2 + 0] = m_run * C2;
+                        p.part_ml[base * 2 + 1] = redl[r] + redl[128 + r];
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive(BAR(BAR_O_FREE));
