@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             if (PS == 64) bad = !wait_bounded(BAR(BAR_RAW + i % NS), (i / NS) & 1, abort_flag);
             // buffers i & 1 are free once PV(i - 2) is done (which also means every
             // S MMA up to tile i - 1 is done, so the A operand may be replaced)
-            if (i >= 2) bad = !wait_bounded(BAR(BAR_KV_FREE + (i & 1)), ((i - 2) >> 1) & 1, abort_flag);
+            if (i >= 2 && !bad) bad = !wait_bounded(BAR(BAR_KV_FREE + (i & 1)), ((i - 2) >> 1) & 1, abort_flag);
             if (i == 1 && seg_start && !bad) bad = !wait_bounded(BAR(BAR_S_FULL), 0, abort_flag);
             // past this barrier: tile i landed for every loader, and every loader
             // has converted tile i - 1, so its raw stage may be refilled
