@@ -182,6 +182,37 @@ cudaLaunchAttribute pdl_attr() {
     return a;
 }
 
+// cuTensorMapEncodeTiled, looked up once through the runtime.
+int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> encode{nullptr};
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode.load(std::memory_order_acquire);
+    if (fn == nullptr) {
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(driver_fn("cuTensorMapEncodeTiled"));
+        if (fn == nullptr) return fail(GAD_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+        encode.store(fn, std::memory_order_release);
+    }
+    *out = fn;
+    return GAD_OK;
+}
+
+// A cache (K or V) as a 2D byte tensor of num_rows rows of row_bytes, read in
+// tiles of one 64-row page x 128 bytes (one head group) with the 128-byte
+// swizzle.
+int encode_cache_pages(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t num_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    const int st = tensor_map_encoder(&fn);
+    if (st != GAD_OK) return st;
+    const cuuint64_t dims[2] = {row_bytes, num_rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {128, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(GAD_ERR_CUDA, "cuTensorMapEncodeTiled (cache pages) failed (%d)", static_cast<int>(r));
+    return GAD_OK;
+}
+
 template <int LT, int PS, int KG, int NS, int MINB, int TK, bool MERGE, bool MULTI>
 int launch_decode(const gad::StepParams& prm, int sms, int tiles_upper, cudaStream_t stream,
                   bool pdl) {
@@ -213,6 +244,16 @@ int launch_decode(const gad::StepParams& prm, int sms, int tiles_upper, cudaStre
     long long grid = static_cast<long long>(sms) * occ;
     if (grid > tiles_upper) grid = tiles_upper;
     if (grid < 1) grid = 1;
+    CUtensorMap kmap, vmap;  // page size 64: the caches' pages, read by TMA tile loads
+    std::memset(&kmap, 0, sizeof(kmap));
+    std::memset(&vmap, 0, sizeof(vmap));
+    if (PS == 64) {
+        const uint64_t row_bytes = static_cast<uint64_t>(GAD_ROW_BYTES) * prm.ngrp;
+        int st = encode_cache_pages(&kmap, prm.k_cache, row_bytes, static_cast<uint64_t>(prm.num_rows));
+        if (st != GAD_OK) return st;
+        st = encode_cache_pages(&vmap, prm.v_cache, row_bytes, static_cast<uint64_t>(prm.num_rows));
+        if (st != GAD_OK) return st;
+    }
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -222,39 +263,8 @@ int launch_decode(const gad::StepParams& prm, int sms, int tiles_upper, cudaStre
     cudaLaunchAttribute attr = pdl_attr();
     cfg.attrs = &attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kern, prm);
+    e = cudaLaunchKernelEx(&cfg, kern, prm, kmap, vmap);
     if (e != cudaSuccess) return fail(GAD_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
-    return GAD_OK;
-}
-
-// cuTensorMapEncodeTiled, looked up once through the runtime.
-int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
-    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> encode{nullptr};
-    PFN_cuTensorMapEncodeTiled_v12000 fn = encode.load(std::memory_order_acquire);
-    if (fn == nullptr) {
-        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(driver_fn("cuTensorMapEncodeTiled"));
-        if (fn == nullptr) return fail(GAD_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
-        encode.store(fn, std::memory_order_release);
-    }
-    *out = fn;
-    return GAD_OK;
-}
-
-// A cache (K or V) as a 2D byte tensor of num_rows rows of row_bytes, read in
-// tiles of one 64-row page x 128 bytes (one head group) with the 128-byte
-// swizzle.
-int encode_cache_pages(CUtensorMap* map, const void* base, uint64_t row_bytes, uint64_t num_rows) {
-    PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    const int st = tensor_map_encoder(&fn);
-    if (st != GAD_OK) return st;
-    const cuuint64_t dims[2] = {row_bytes, num_rows};
-    const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {128, 64};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(GAD_ERR_CUDA, "cuTensorMapEncodeTiled (cache pages) failed (%d)", static_cast<int>(r));
     return GAD_OK;
 }
 

@@ -22,6 +22,7 @@
 #include <cuda_fp8.h>
 
 #include "gad_ptx.cuh"
+#include "gad_tc.cuh"
 
 namespace gad {
 
@@ -220,8 +221,14 @@ struct DecodeCfg {
     static constexpr size_t IDX_BYTES = static_cast<size_t>(IDX_SLOTS) * TK * 4;
     static constexpr size_t MERGE_BYTES =
         static_cast<size_t>(MERGE_WARPS) * MERGE_FLOATS_PER_WARP * 4;
+    // page size 64: one mbarrier per stage (the TMA page loads' bytes) and the
+    // abort flag
+    static constexpr size_t CTRL_BYTES = 64;
+    static_assert(NS * 8 + 8 <= static_cast<int>(CTRL_BYTES), "control block");
+    // + 1024 so the stages can start on a 1024-byte boundary (the 128-byte
+    // swizzle of the TMA page loads is anchored there)
     static size_t smem_bytes(int B) {
-        return KV_BYTES + IDX_BYTES + MERGE_BYTES + static_cast<size_t>(4 * B + 1) * 4;
+        return 1024 + KV_BYTES + IDX_BYTES + MERGE_BYTES + CTRL_BYTES + static_cast<size_t>(4 * B + 1) * 4;
     }
     static_assert(RG >= 1 && RG * HKV * KG == WARPS, "warp split");
     static_assert(NT * RG == LT && MT * KG == TK / 16, "tile split");
@@ -237,15 +244,26 @@ __device__ __forceinline__ int kappa(int l) {
 
 // MULTI: more than one head group (the one-group instantiation keeps the
 // list item equal to the request, with no index arithmetic for groups).
+// Page size 64: a stage's pages arrive by TMA tile loads (kmap, vmap: the K and
+// V caches as 2D tensors of 128 ngrp-byte rows, one 64-row page x 128 bytes a
+// tile, 128-byte swizzle: the layout the page-size-1 gathers write), issued
+// by thread 0 and waited for on the stage's mbarrier.
 template <int LT, int PS, int KG, int NS, int MINB, int TK, bool MERGE, bool MULTI>
-__global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepParams p) {
+__global__ void __launch_bounds__(DEC_THREADS, MINB)
+    decode_kernel(const StepParams p, const __grid_constant__ CUtensorMap kmap,
+                  const __grid_constant__ CUtensorMap vmap) {
     using C = DecodeCfg<LT, KG, NS, TK, MERGE>;
     constexpr int NT = C::NT, MT = C::MT, RG = C::RG;
-    extern __shared__ __align__(1024) uint8_t smem[];
+    constexpr bool TMA = PS == 64;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
     uint8_t* kv_smem = smem;
     int* idx_smem = reinterpret_cast<int*>(smem + C::KV_BYTES);
     float* merge_smem = reinterpret_cast<float*>(smem + C::KV_BYTES + C::IDX_BYTES);
-    int* tpre = reinterpret_cast<int*>(smem + C::KV_BYTES + C::IDX_BYTES + C::MERGE_BYTES);
+    uint8_t* ctrl = smem + C::KV_BYTES + C::IDX_BYTES + C::MERGE_BYTES;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + NS * 8);
+    int* tpre = reinterpret_cast<int*>(ctrl + C::CTRL_BYTES);
     int* rlo = tpre + p.NB + 1;
     int* rhi = rlo + p.NB;
     int* rnew = rhi + p.NB;
@@ -263,6 +281,16 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
     int total, per, t0, t1;
     build_tile_list<TK, MULTI>(p, tpre, rlo, rhi, rnew, DEC_THREADS, total, per, t0, t1);
     if (t0 >= t1) return;
+    const uint32_t bar0 = smem_addr(ctrl);
+    auto STAGE_BAR = [&](int st) { return bar0 + 8u * static_cast<uint32_t>(st); };
+    if (TMA) {
+        if (tid == 0) {
+            for (int st = 0; st < NS; ++st) mbar_init(STAGE_BAR(st), 1);
+            *abort_flag = 0;
+            mbar_fence_init();
+        }
+        __syncthreads();
+    }
     // The normalised q and this step's new cache rows come from the prep kernel,
     // which may still be running (programmatic dependent launch): wait for it
     // only before the first q load or the first gather of a tile holding new
@@ -314,6 +342,7 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
             }
         }
     };
+    int n_issued = 0;  // tiles whose loads were issued (the same count in every thread)
     auto issue_kv = [&](int tau, int b) {
         if (tau >= t1) return;
         const int k0 = tile_k0(tau, b);
@@ -322,6 +351,25 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
         const uint32_t base = smem_addr(kv_smem + ((tau - t0) % NS) * C::STAGE);
         const int lo = rlo[b], hi = rhi[b];
         const size_t gofs = static_cast<size_t>(item_ref<MULTI>(p, b).grp) * ROWB;
+        ++n_issued;
+        if constexpr (TMA) {
+            // the tile's TK / 64 pages, K and V: one TMA tile load each; a page
+            // index past the table (-1) or rows past the cache fall outside the
+            // tensor and read as zeros
+            if (tid == 0) {
+                fence_proxy_async_smem();  // the zeroed rows of this stage's last tile come first
+                const uint32_t bar = STAGE_BAR((tau - t0) % NS);
+                mbar_arrive_expect_tx(bar, C::STAGE);
+#pragma unroll
+                for (int pq = 0; pq < TK / PS; ++pq) {
+                    const int pg = ix[pq];
+                    const int y = pg >= 0 ? pg * PS : -PS;
+                    tma_load_2d(base + pq * PS * ROWB, &kmap, static_cast<int>(gofs), y, bar);
+                    tma_load_2d(base + TK * ROWB + pq * PS * ROWB, &vmap, static_cast<int>(gofs), y, bar);
+                }
+            }
+            return;
+        }
 #pragma unroll
         for (int i = 0; i < TK / 32; ++i) {
             const int r = (tid >> 3) + 32 * i;  // tile row
@@ -604,9 +652,30 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
         cp_async_commit();
     }
     int cur_b = -1;
-    for (int i = 0; ct < t1; ++i) {
+    int i = 0;
+    for (; ct < t1; ++i) {
         cp_async_wait<NS - 2>();
-        __syncthreads();
+        if constexpr (TMA) {
+            // the stage's pages landed; keys of the tile outside the item's range
+            // (page slots not yet written, or before a window) become zeros, as
+            // the page-size-1 gathers zero-fill them: thread (row, half) clears
+            // its half of the K and V rows
+            bool bad = !wait_bounded(STAGE_BAR(i % NS), (i / NS) & 1, abort_flag);
+            const int k0 = tile_k0(ct, cb);
+            const int r = tid >> 1;
+            if (!bad && (k0 + r < rlo[cb] || k0 + r > rhi[cb])) {
+                const uint32_t row = smem_addr(kv_smem + (i % NS) * C::STAGE) + r * ROWB + (tid & 1) * 64;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    sts128(row + 16 * q, make_uint4(0u, 0u, 0u, 0u));
+                    sts128(row + TK * ROWB + 16 * q, make_uint4(0u, 0u, 0u, 0u));
+                }
+                fence_proxy_async_smem();
+            }
+            if (bar_red_or(0, DEC_THREADS, bad)) break;
+        } else {
+            __syncthreads();
+        }
         issue_kv(kt, kb);
         advance(kt, kb);
         issue_idx(xt, xb);
@@ -620,8 +689,18 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB) decode_kernel(const StepPar
         compute_tile(i % NS, tile_k0(ct, cb));
         advance(ct, cb);
     }
-    flush(cur_b);
+    if (cur_b >= 0 && !(TMA && *abort_flag)) flush(cur_b);
     cp_async_wait<0>();
+    if (TMA && tid == 0) {
+        // every page load issued lands before the CTA leaves (its shared memory
+        // is the destination); without an abort they all have
+        for (int tile = i; tile < n_issued; ++tile)
+            wait_bounded(STAGE_BAR(tile % NS), (tile / NS) & 1, abort_flag, false, TEARDOWN_LIMIT_NS);
+        if (*abort_flag) {
+            pdl_wait_primary();  // the step's first kernel has cleared the status word
+            atomicOr(p.status, STATUS_ATTN_WAIT);
+        }
+    }
     pdl_launch_dependents();
 }
 
