@@ -19,14 +19,18 @@
 // the half of its own KV head.
 //
 // Data flow per tile (all in one CTA per SM):
-//   loader warps 4-7  cp.async gathers of raw E4M3 rows into an NS-stage ring
-//                     (as decode_kernel), then E4M3 -> fp16 into a 128-byte-
-//                     swizzled tile (K and V, double-buffered); at a request's
-//                     first tile they also write its A operand into tensor
-//                     memory.
-//   MMA warp 8        S(i) = A . K(i)^T into tensor memory (double-buffered),
+//   loader warps 8-11 raw E4M3 rows into an NS-stage ring (page size 1:
+//                     cp.async gathers, as decode_kernel; page size 64: one
+//                     TMA tile load per page for K and one for V), then
+//                     E4M3 -> fp16 into a 128-byte-swizzled tile (K and V,
+//                     double-buffered); at a request's first tile they also
+//                     write its A operand into tensor memory.
+//   MMA warp 12       S(i) = A . K(i)^T into tensor memory (double-buffered),
 //                     then O += P(i-1) . V(i-1) with P read from tensor memory.
-//   softmax warps 0-3 one thread per row: S from tensor memory, mask, online
+//   softmax warps 0-7 two threads per row (warps w and w + 4 share the
+//                     tensor-memory lanes of rows 32 (w % 4) .. + 31, 32 keys
+//                     each): S from tensor memory, mask, the halves' maxima
+//                     and sums exchanged through shared memory, online
 //                     softmax with lazy rescaling (O is rescaled in tensor
 //                     memory only when the running max grows by more than
 //                     2^8), P as fp16 back into the S columns; at a request's
