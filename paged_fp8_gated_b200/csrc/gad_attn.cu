@@ -321,9 +321,9 @@ int launch_verify_tc(const gad::StepParams& prm, int sms, int tiles_upper, cudaS
     return GAD_OK;
 }
 
-// Whether the 8-stage verify kernel's shared memory, with tables for NB list
+// Whether the deep-ring verify kernel's shared memory, with tables for NB list
 // items, fits in `optin` bytes.
-constexpr int kVtcDeepStages = 8, kVtcShallowStages = 4;
+constexpr int kVtcDeepStages = 6, kVtcShallowStages = 3;
 
 bool verify_deep_fits(int NB, int optin) {
     return gad::vtc::Cfg<kVtcDeepStages>::smem_bytes(NB) <= static_cast<size_t>(optin);

@@ -368,25 +368,20 @@ __global__ void __launch_bounds__(DEC_THREADS, MINB)
                     tma_load_2d(base + TK * ROWB + pq * PS * ROWB, &vmap, static_cast<int>(gofs), y, bar);
                 }
             }
-            return;
-        }
+        } else {
+            static_assert(PS == 1, "page size 64 reads whole pages by TMA");
 #pragma unroll
-        for (int i = 0; i < TK / 32; ++i) {
-            const int r = (tid >> 3) + 32 * i;  // tile row
-            const int j = tid & 7;              // 16-byte chunk
-            const int k = k0 + r;
-            int64_t crow;
-            if (PS == 1) {
-                crow = ix[r];
-            } else {
-                const int pg = ix[r / PS];
-                crow = pg >= 0 ? static_cast<int64_t>(pg) * PS + r % PS : -1;
+            for (int i = 0; i < TK / 32; ++i) {
+                const int r = (tid >> 3) + 32 * i;  // tile row
+                const int j = tid & 7;              // 16-byte chunk
+                const int k = k0 + r;
+                const int64_t crow = ix[r];
+                const bool ok = k >= lo && k <= hi && crow >= 0 && crow < p.num_rows;
+                const size_t off = ok ? static_cast<size_t>(crow) * row_pitch + gofs + j * 16 : 0;
+                const uint32_t d = base + r * ROWB + ((j ^ (r & 7)) << 4);
+                cp_async16(d, p.k_cache + off, ok ? 16 : 0);
+                cp_async16(d + TK * ROWB, p.v_cache + off, ok ? 16 : 0);
             }
-            const bool ok = k >= lo && k <= hi && crow >= 0 && crow < p.num_rows;
-            const size_t off = ok ? static_cast<size_t>(crow) * row_pitch + gofs + j * 16 : 0;
-            const uint32_t d = base + r * ROWB + ((j ^ (r & 7)) << 4);
-            cp_async16(d, p.k_cache + off, ok ? 16 : 0);
-            cp_async16(d + TK * ROWB, p.v_cache + off, ok ? 16 : 0);
         }
     };
 

@@ -59,25 +59,33 @@ constexpr int RAW_STAGE = 2 * TK * ROWB;      // 16 KB: 64 K rows then 64 V rows
 constexpr int HALF_TILE = TK * 128;           // one head of a converted tile: 64 keys x 64 fp16
 constexpr int F16_TILE = 2 * HALF_TILE;       // both heads: 16 KB
 constexpr int F16_BUF = 2 * F16_TILE;         // K tile then V tile: 32 KB
+// Converted K/V tiles in flight.  Three, so that converting tile i waits only
+// for P.V of tile i - 3: with two, the chain "P.V(i - 2) done -> convert tile
+// i -> S(i) issued -> P.V(i - 1) issued (after S(i), in MMA order) -> P.V(i - 1)
+// done -> convert tile i + 1" put a whole conversion and two MMA groups in
+// series for every tile.
+constexpr int NF = 3;
 constexpr uint32_t TM_COLS = 512;             // tensor-memory columns allocated
-constexpr uint32_t TM_Q = 0;                  // A operand (fp16 pairs): 64 columns
+constexpr uint32_t TM_Q = 0;                  // A operand (fp16 pairs) of even items: 64 columns
+constexpr uint32_t TM_Q1 = 192;               // A operand of odd items (an item's A may be written
+                                              // while the previous item's last S MMAs still read theirs)
 constexpr uint32_t TM_S = 64;                 // S buffer b at TM_S + 64 b (P aliases its first 32)
 constexpr uint32_t TM_O = 256;                // O: 128 columns (head 0 dims | head 1 dims)
 constexpr float RESCALE_LOG2 = 8.f;           // lazy rescale threshold (P stays <= 2^8)
 
 // mbarrier indices
-constexpr int BAR_KV_READY = 0;   // [2] converted tile (and A operand) ready   (128 loader arrivals)
-constexpr int BAR_KV_FREE = 2;    // [2] PV of the tile done: buffers free       (MMA commit)
-constexpr int BAR_S_FULL = 4;     // [2] S of the tile in tensor memory          (MMA commit)
-constexpr int BAR_P_FULL = 6;     // [2] P of the tile in tensor memory          (256 softmax arrivals)
-constexpr int BAR_O_FREE = 8;     // O read out at a request's last tile         (256 softmax arrivals)
-constexpr int BAR_MMA_DONE = 9;   // teardown: all MMAs done                     (MMA commit)
-constexpr int BAR_RAW = 10;       // [NS] page size 64: the tile's K and V pages landed (TMA bytes)
-constexpr int NBARS = 10;         // + NS for page size 64
+constexpr int BAR_KV_READY = 0;   // [NF] converted tile (and A operand) ready  (128 loader arrivals)
+constexpr int BAR_KV_FREE = 3;    // [NF] PV of the tile done: buffers free      (MMA commit)
+constexpr int BAR_S_FULL = 6;     // [2] S of the tile in tensor memory          (MMA commit)
+constexpr int BAR_P_FULL = 8;     // [2] P of the tile in tensor memory          (256 softmax arrivals)
+constexpr int BAR_O_FREE = 10;    // O read out at a request's last tile         (256 softmax arrivals)
+constexpr int BAR_MMA_DONE = 11;  // teardown: all MMAs done                     (MMA commit)
+constexpr int BAR_RAW = 12;       // [NS] page size 64: the tile's K and V pages landed (TMA bytes)
+constexpr int NBARS = 12;         // + NS for page size 64
 
 template <int NS>
 struct Cfg {
-    static constexpr size_t F16_BYTES = 2 * F16_BUF;
+    static constexpr size_t F16_BYTES = NF * F16_BUF;
     static constexpr size_t RAW_BYTES = static_cast<size_t>(NS) * RAW_STAGE;
     static constexpr int IDX_SLOTS = 2 * NS;
     static constexpr size_t IDX_BYTES = static_cast<size_t>(IDX_SLOTS) * TK * 4;
@@ -113,7 +121,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-    uint8_t* f16 = smem;                                     // [2][K,V][head][64 keys][128 B]
+    uint8_t* f16 = smem;                                     // [NF][K,V][head][64 keys][128 B]
     uint8_t* raw = smem + C::F16_BYTES;                      // [NS][K rows, V rows]
     int* idx_smem = reinterpret_cast<int*>(raw + C::RAW_BYTES);
     uint8_t* ctrl = reinterpret_cast<uint8_t*>(idx_smem) + C::IDX_BYTES;
@@ -137,10 +145,10 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
     const uint32_t bar0 = smem_addr(ctrl);
     auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
     if (tid == 0) {
-        mbar_init(BAR(BAR_KV_READY), LOADERS);
-        mbar_init(BAR(BAR_KV_READY + 1), LOADERS);
-        mbar_init(BAR(BAR_KV_FREE), 1);
-        mbar_init(BAR(BAR_KV_FREE + 1), 1);
+        for (int f = 0; f < NF; ++f) {
+            mbar_init(BAR(BAR_KV_READY + f), LOADERS);
+            mbar_init(BAR(BAR_KV_FREE + f), 1);
+        }
         mbar_init(BAR(BAR_S_FULL), 1);
         mbar_init(BAR(BAR_S_FULL + 1), 1);
         mbar_init(BAR(BAR_P_FULL), SOFT);
@@ -296,7 +304,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             }
         };
         // A operand of item b's S MMA: row ltid = [q | 0] (KV head 0) or [0 | q].
-        auto write_q = [&](int b) {
+        auto write_q = [&](int b, uint32_t qcol) {
             ensure_prep();
             const int g = ltid >> 6, j = (ltid >> 3) & 7, hh = ltid & 7;
             const ItemRef it = item_ref<MULTI>(p, b);
@@ -318,7 +326,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < 32; ++c) q[c] = 0u;
             }
-            const uint32_t ta = tmem + TM_Q + (static_cast<uint32_t>(32 * (warp - LOAD_W0)) << 16);
+            const uint32_t ta = tmem + qcol + (static_cast<uint32_t>(32 * (warp - LOAD_W0)) << 16);
             tc_st32(ta + (g == 0 ? 0u : 32u), q);
             tc_st32(ta + (g == 0 ? 32u : 0u), z);
         };
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             cur_next(xc);
             cp_async_commit();
         }
-        int seg_b = -1;
+        int seg_b = -1, nseg = 0;
         const int n_tiles = t1 - t0;
         int i = 0;
         for (; i < n_tiles; ++i) {
@@ -382,24 +390,28 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             const bool seg_start = cb != seg_b;
             bool bad = false;
             if (PS == 64) bad = !wait_bounded(BAR(BAR_RAW + i % NS), (i / NS) & 1, abort_flag);
-            // buffers i & 1 are free once PV(i - 2) is done (which also means every
-            // S MMA up to tile i - 1 is done, so the A operand may be replaced)
-            if (i >= 2 && !bad) bad = !wait_bounded(BAR(BAR_KV_FREE + (i & 1)), ((i - 2) >> 1) & 1, abort_flag);
-            if (i == 1 && seg_start && !bad) bad = !wait_bounded(BAR(BAR_S_FULL), 0, abort_flag);
+            // buffers i % NF are free once PV(i - NF) is done, which also means every
+            // S MMA up to tile i - NF + 1 is done: the A operand this item takes
+            // (the one of the item before the previous) is no longer read.  Tile 2
+            // has no such wait; if it starts a third item, S(0) (item 0's) must be done.
+            if (i >= NF && !bad) bad = !wait_bounded(BAR(BAR_KV_FREE + i % NF), ((i - NF) / NF) & 1, abort_flag);
+            static_assert(NF == 3, "the A-operand wait below assumes three buffers");
+            if (i == 2 && seg_start && nseg >= 2 && !bad) bad = !wait_bounded(BAR(BAR_S_FULL), 0, abort_flag);
             // past this barrier: tile i landed for every loader, and every loader
             // has converted tile i - 1, so its raw stage may be refilled
             if (bar_red_or(1, LOADERS, bad)) break;
             if (seg_start) {
-                write_q(cb);
+                write_q(cb, (nseg & 1) ? TM_Q1 : TM_Q);
                 seg_b = cb;
+                ++nseg;
             }
-            convert(i % NS, i & 1, cc.k0, cc.lo, cc.hi);
+            convert(i % NS, i % NF, cc.k0, cc.lo, cc.hi);
             fence_proxy_async_smem();
             if (seg_start) {
                 tc_wait_st();
                 tc_fence_before();
             }
-            mbar_arrive(BAR(BAR_KV_READY + (i & 1)));
+            mbar_arrive(BAR(BAR_KV_READY + i % NF));
             // gathers for tile i + NS - 1 (into the stage of tile i - 1), off the
             // path from "buffer free" to "tile ready"
             issue_kv(kc);
@@ -429,7 +441,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             if (!wait_warp(BAR(BAR_P_FULL + (k & 1)), (k >> 1) & 1, abort_flag)) return false;
             if (first && seg >= 1 && !wait_warp(BAR(BAR_O_FREE), (seg - 1) & 1, abort_flag)) return false;
             tc_fence_after();
-            const uint32_t vbuf = f16_base + (k & 1) * F16_BUF + F16_TILE;
+            const uint32_t vbuf = f16_base + (k % NF) * F16_BUF + F16_TILE;
             const uint32_t pa = tmem + TM_S + 64u * (k & 1);
             const uint32_t av[4] = {pa, pa + 8u, pa + 16u, pa + 24u};
 #pragma unroll
@@ -439,7 +451,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                                         smem_desc_sw128(vb + 4096), smem_desc_sw128(vb + 6144)};
                 tc_mma_ts4(tmem + TM_O + 64u * h, av, bd, ID_O, first ? 0u : 1u);
             }
-            tc_commit(BAR(BAR_KV_FREE + (k & 1)));
+            tc_commit(BAR(BAR_KV_FREE + k % NF));
             return true;
         };
         int ct = t0, cb = find_req(t0);
@@ -454,16 +466,16 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                 seg_b = cb;
                 ++seg;
             }
-            if (!wait_warp(BAR(BAR_KV_READY + (i & 1)), (i >> 1) & 1, abort_flag)) {
+            if (!wait_warp(BAR(BAR_KV_READY + i % NF), (i / NF) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t kbuf = f16_base + (i & 1) * F16_BUF;
+            const uint32_t kbuf = f16_base + (i % NF) * F16_BUF;
             const uint32_t sd = tmem + TM_S + 64u * (i & 1);
 #pragma unroll
             for (int hk = 0; hk < 2; ++hk) {  // the contraction's two KV-head halves, 4 K16 steps each
-                const uint32_t qa = tmem + TM_Q + 32u * hk;
+                const uint32_t qa = tmem + ((seg & 1) ? TM_Q1 : TM_Q) + 32u * hk;
                 const uint32_t aq[4] = {qa, qa + 8u, qa + 16u, qa + 24u};
                 const uint32_t kb = kbuf + hk * HALF_TILE;
                 const uint64_t bd[4] = {smem_desc_sw128(kb), smem_desc_sw128(kb + 32),
@@ -567,7 +579,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             }
             if (__any_sync(0xffffffffu, corr)) {
                 // PV(i - 1) of this request must be done before O is touched
-                const bool ok = wait_warp(BAR(BAR_KV_FREE + ((i - 1) & 1)), ((i - 1) >> 1) & 1, abort_flag);
+                const bool ok = wait_warp(BAR(BAR_KV_FREE + (i - 1) % NF), ((i - 1) / NF) & 1, abort_flag);
                 const float alpha = corr ? fast_exp2((m_run - m_new) * C2) : 1.f;
                 if (ok) {
                     tc_fence_after();
@@ -603,7 +615,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             mbar_arrive(BAR(BAR_P_FULL + (i & 1)));
 
             if (seg_end) {
-                const bool ok = wait_warp(BAR(BAR_KV_FREE + (i & 1)), (i >> 1) & 1, abort_flag);
+                const bool ok = wait_warp(BAR(BAR_KV_FREE + i % NF), (i / NF) & 1, abort_flag);
                 redl[half * 128 + r] = l_run;
                 // both halves' sums posted
                 if (bar_red_or(pair_bar, 64, bad || !ok)) break;
