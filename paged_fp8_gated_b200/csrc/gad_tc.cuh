@@ -168,6 +168,23 @@ __device__ __forceinline__ void tc_mma_ts4(uint32_t d, const uint32_t (&a)[4], c
         "r"(accumulate), "r"(0u), "r"(a[3])
         : "memory");
 }
+// Two K = 32 contractions into two accumulators from one elected lane:
+// D0 (+)= A(a[0]) B(b[0])^T + A(a[1]) B(b[1])^T and D1 (+)= A(a[2]) B(b[2])^T +
+// A(a[3]) B(b[3])^T, each first step accumulating only if `accumulate` is
+// nonzero.  Whole warp, warp-uniform operands.
+__device__ __forceinline__ void tc_mma_ts2x2(uint32_t d0, uint32_t d1, const uint32_t (&a)[4],
+                                             const uint64_t (&b)[4], uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p, e, t;\n .reg .b32 rx;\n elect.sync rx|e, 0xffffffff;\n"
+        " setp.ne.b32 p, %10, 0;\n setp.eq.b32 t, %11, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %7, %6, {%11,%11,%11,%11}, p;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %8, %6, {%11,%11,%11,%11}, t;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%1], [%4], %9, %6, {%11,%11,%11,%11}, p;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%1], [%5], %12, %6, {%11,%11,%11,%11}, t;\n}\n" ::"r"(d0),
+        "r"(d1), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(idesc), "l"(b[0]), "l"(b[1]), "l"(b[2]),
+        "r"(accumulate), "r"(0u), "l"(b[3])
+        : "memory");
+}
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 

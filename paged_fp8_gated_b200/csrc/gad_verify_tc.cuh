@@ -28,13 +28,15 @@
 //   MMA warp 12       S(i) = A . K(i)^T into tensor memory (double-buffered),
 //                     then O += P(i-1) . V(i-1) with P read from tensor memory.
 //   softmax warps 0-7 two threads per row (warps w and w + 4 share the
-//                     tensor-memory lanes of rows 32 (w % 4) .. + 31, 32 keys
-//                     each): S from tensor memory, mask, the halves' maxima
-//                     and sums exchanged through shared memory, online
-//                     softmax with lazy rescaling (O is rescaled in tensor
-//                     memory only when the running max grows by more than
-//                     2^8), P as fp16 back into the S columns; at a request's
-//                     last tile, O's row half -> partial.
+//                     tensor-memory lanes of rows 32 (w % 4) .. + 31): half h
+//                     takes keys 32h .. 32h + 31 of every tile and runs its
+//                     own online softmax over them (own running max and sum,
+//                     own O accumulator O_h, lazy rescaling: O_h is rescaled
+//                     in tensor memory only when its max grows by more than
+//                     2^8), P as fp16 back into its own S columns; at a
+//                     request's last tile the halves merge (m, l) through
+//                     shared memory and each writes half the dims of
+//                     a0 O_0 + a1 O_1 to the partial.
 // Synchronisation by mbarriers; every wait is bounded (an expired wait sets
 // the step's error word and the CTA winds down, waits for its MMAs and frees
 // its tensor memory).
@@ -70,7 +72,8 @@ constexpr uint32_t TM_Q = 0;                  // A operand (fp16 pairs) of even 
 constexpr uint32_t TM_Q1 = 192;               // A operand of odd items (an item's A may be written
                                               // while the previous item's last S MMAs still read theirs)
 constexpr uint32_t TM_S = 64;                 // S buffer b at TM_S + 64 b (P aliases its first 32)
-constexpr uint32_t TM_O = 256;                // O: 128 columns (head 0 dims | head 1 dims)
+constexpr uint32_t TM_O = 256;                // O_0, O_1 (keys 0-31 / 32-63 of every tile), 128
+constexpr uint32_t TM_O_HALF = 128;           // columns each (head 0 dims | head 1 dims)
 constexpr float RESCALE_LOG2 = 8.f;           // lazy rescale threshold (P stays <= 2^8)
 
 // mbarrier indices
@@ -80,8 +83,9 @@ constexpr int BAR_S_FULL = 6;     // [2] S of the tile in tensor memory         
 constexpr int BAR_P_FULL = 8;     // [2] P of the tile in tensor memory          (256 softmax arrivals)
 constexpr int BAR_O_FREE = 10;    // O read out at a request's last tile         (256 softmax arrivals)
 constexpr int BAR_MMA_DONE = 11;  // teardown: all MMAs done                     (MMA commit)
-constexpr int BAR_RAW = 12;       // [NS] page size 64: the tile's K and V pages landed (TMA bytes)
-constexpr int NBARS = 12;         // + NS for page size 64
+constexpr int BAR_PAIR = 12;      // [4] softmax pair qd posted its halves' (max, sum) at a request's end (64)
+constexpr int BAR_RAW = 16;       // [NS] page size 64: the tile's K and V pages landed (TMA bytes)
+constexpr int NBARS = 16;         // + NS for page size 64
 
 template <int NS>
 struct Cfg {
@@ -90,7 +94,8 @@ struct Cfg {
     static constexpr int IDX_SLOTS = 2 * NS;
     static constexpr size_t IDX_BYTES = static_cast<size_t>(IDX_SLOTS) * TK * 4;
     static constexpr size_t CTRL_BYTES = 256;  // barriers, tensor-memory base, abort flag
-    static constexpr size_t RED_BYTES = 3 * 2 * 128 * 4;  // softmax pairs: maxima [2 tiles][2 halves], sums
+    // softmax pairs at a request's end: [2 (request parity)][max, sum][2 halves][128 rows]
+    static constexpr size_t RED_BYTES = 2 * 2 * 2 * 128 * 4;
     // + 1024 so the swizzled tiles can start on a 1024-byte boundary
     static size_t smem_bytes(int B) {
         return 1024 + F16_BYTES + RAW_BYTES + IDX_BYTES + CTRL_BYTES + RED_BYTES +
@@ -127,8 +132,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
     uint8_t* ctrl = reinterpret_cast<uint8_t*>(idx_smem) + C::IDX_BYTES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + (NBARS + NS) * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + (NBARS + NS) * 8 + 4);
-    float* red = reinterpret_cast<float*>(ctrl + C::CTRL_BYTES);  // [2 tiles][2 halves][128 rows] maxima
-    float* redl = red + 4 * 128;                                   // [2 halves][128 rows] sums
+    float* red = reinterpret_cast<float*>(ctrl + C::CTRL_BYTES);  // halves' (max, sum) at a request's end
     int* tpre = reinterpret_cast<int*>(ctrl + C::CTRL_BYTES + C::RED_BYTES);
     int* rlo = tpre + p.NB + 1;
     int* rhi = rlo + p.NB;
@@ -155,6 +159,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
         mbar_init(BAR(BAR_P_FULL + 1), SOFT);
         mbar_init(BAR(BAR_O_FREE), SOFT);
         mbar_init(BAR(BAR_MMA_DONE), 1);
+        for (int q = 0; q < 4; ++q) mbar_init(BAR(BAR_PAIR + q), 64);
         if (PS == 64)
             for (int st = 0; st < NS; ++st) mbar_init(BAR(BAR_RAW + st), 1);
         *abort_flag = 0;
@@ -436,20 +441,22 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
         constexpr uint32_t ID_S = idesc_f16_f32(128, TK, 0);  // S: A . K^T, K-major B
         constexpr uint32_t ID_O = idesc_f16_f32(128, 64, 1);  // O: P . V, MN-major B
         const uint32_t f16_base = smem_addr(f16);
-        // O += P(k) . V(k), as two N = 64 MMAs (one per KV head's dims).
+        // O_h += P(k)[keys of half h] . V(k)[same keys], per KV head's dims (N = 64):
+        // P of keys 0-31 sits in S columns 0-15, of keys 32-63 in columns 32-47.
         auto issue_pv = [&](int k, bool first, int seg) {
             if (!wait_warp(BAR(BAR_P_FULL + (k & 1)), (k >> 1) & 1, abort_flag)) return false;
             if (first && seg >= 1 && !wait_warp(BAR(BAR_O_FREE), (seg - 1) & 1, abort_flag)) return false;
             tc_fence_after();
             const uint32_t vbuf = f16_base + (k % NF) * F16_BUF + F16_TILE;
             const uint32_t pa = tmem + TM_S + 64u * (k & 1);
-            const uint32_t av[4] = {pa, pa + 8u, pa + 16u, pa + 24u};
+            const uint32_t av[4] = {pa, pa + 8u, pa + 32u, pa + 40u};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const uint32_t vb = vbuf + h * HALF_TILE;
                 const uint64_t bd[4] = {smem_desc_sw128(vb), smem_desc_sw128(vb + 2048),
                                         smem_desc_sw128(vb + 4096), smem_desc_sw128(vb + 6144)};
-                tc_mma_ts4(tmem + TM_O + 64u * h, av, bd, ID_O, first ? 0u : 1u);
+                tc_mma_ts2x2(tmem + TM_O + 64u * h, tmem + TM_O + TM_O_HALF + 64u * h, av, bd, ID_O,
+                             first ? 0u : 1u);
             }
             tc_commit(BAR(BAR_KV_FREE + k % NF));
             return true;
@@ -500,20 +507,22 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
     } else {
         // =================== softmax: two threads per row ===================
         // Warps w and w + 4 share the tensor-memory lanes of rows 32 (w % 4) ..
-        // + 31 and take 32 keys each; the pair posts its halves' maxima through
-        // shared memory (double-buffered by tile parity) and meets at a named
-        // barrier that also ORs a give-up flag, so both warps of a pair always
-        // stop at the same point.
+        // + 31; half h = w / 4 takes keys 32h .. 32h + 31 of every tile with its
+        // own running max, sum and O accumulator, so the two never wait for
+        // each other until a request's last tile, where they merge through
+        // shared memory (double-buffered by request parity) after meeting at
+        // the pair's mbarrier (a bounded wait, as every other).
         const int half = warp >> 2, qd = warp & 3;
         const int r = 32 * qd + (tid & 31);
         const int g = r >> 6, j = (r >> 3) & 7, qh = g * GRP + (r & 7);
-        const int pair_bar = 2 + qd;
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+        const uint32_t o_own = tmem + TM_O + TM_O_HALF * half + 64u * g + lane_base;  // O_half, this row's head
         int ct = t0, cb = find_req(t0);
         int seg_b = -1, seg_t1 = 0, k0 = 0;  // current request, end of its tiles here, tile key
-        float m_run = -INFINITY, l_run = 0.f;  // running max (raw score units), this half's sum
+        float m_run = -INFINITY, l_run = 0.f;  // this half's running max (raw score units) and sum
         int lo_j = INT_MAX, hi_j = -1;
         int seg_len = 0;  // tokens of the current item
+        int n_end = 0;    // requests finished here
         for (int i = 0; ct < t1; ++i) {
             const bool seg_start = cb != seg_b;
             if (seg_start) {
@@ -537,11 +546,12 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             }
             const bool seg_end = ct + 1 >= seg_t1;
 
-            bool bad = !wait_warp(BAR(BAR_S_FULL + (i & 1)), (i >> 1) & 1, abort_flag);
+            if (!wait_warp(BAR(BAR_S_FULL + (i & 1)), (i >> 1) & 1, abort_flag)) break;
             tc_fence_after();
-            const uint32_t sbuf = tmem + TM_S + 64u * (i & 1) + lane_base;
+            // this half's S (columns 32 half ..) and, later, its P (columns 32 half .. + 15)
+            const uint32_t sbuf = tmem + TM_S + 64u * (i & 1) + 32u * half + lane_base;
             uint32_t sr[32];
-            tc_ld32(sbuf + 32u * half, sr);
+            tc_ld32(sbuf, sr);
             tc_wait_ld();
             float s[32];
             const int kb0 = k0 + 32 * half;
@@ -550,24 +560,21 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
             if (cmin <= 0 && cmax >= 31) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    s[c] = __uint_as_float(sr[c]);
-                    m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-                }
+                for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(sr[c]);
             } else {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    s[c] = (c < cmin || c > cmax) ? -INFINITY : __uint_as_float(sr[c]);
-                    m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-                }
+                for (int c = 0; c < 32; ++c) s[c] = (c < cmin || c > cmax) ? -INFINITY : __uint_as_float(sr[c]);
             }
-            float* redm = red + (i & 1) * 2 * 128;
-            redm[half * 128 + r] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            // both halves have read their S (P may overwrite the buffer) and posted their maxima
-            if (bar_red_or(pair_bar, 64, bad)) break;
-            const float mx = fmaxf(redm[r], redm[128 + r]);
-            // lazy rescale: O (in tensor memory) is corrected only when the max
-            // grows a lot; both halves of a row take the same decision
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+                m4[c >> 3] = fmax3(m4[c >> 3], s[c], s[c + 1]);
+                m4[c >> 3] = fmax3(m4[c >> 3], s[c + 2], s[c + 3]);
+                m4[c >> 3] = fmax3(m4[c >> 3], s[c + 4], s[c + 5]);
+                m4[c >> 3] = fmax3(m4[c >> 3], s[c + 6], s[c + 7]);
+            }
+            const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+            // lazy rescale: O_half (in tensor memory) is corrected only when this
+            // half's max grows a lot
             const float m_new = fmaxf(m_run, mx);
             bool corr = false;
             if (m_new > m_run) {
@@ -577,27 +584,31 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                     corr = true;
                 }
             }
+            bool bad = false;
             if (__any_sync(0xffffffffu, corr)) {
                 // PV(i - 1) of this request must be done before O is touched
                 const bool ok = wait_warp(BAR(BAR_KV_FREE + (i - 1) % NF), ((i - 1) / NF) & 1, abort_flag);
                 const float alpha = corr ? fast_exp2((m_run - m_new) * C2) : 1.f;
                 if (ok) {
                     tc_fence_after();
-                    const uint32_t oa = tmem + TM_O + 64u * g + 32u * half + lane_base;
-                    uint32_t o[32];
-                    tc_ld32(oa, o);
-                    tc_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                    tc_st32(oa, o);
+                    for (int q = 0; q < 2; ++q) {
+                        uint32_t o[32];
+                        tc_ld32(o_own + 32u * q, o);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                        tc_st32(o_own + 32u * q, o);
+                    }
                     tc_wait_st();
                 }
-                bad = bad || !ok;
+                bad = !ok;
                 if (corr) {
                     l_run *= alpha;
                     m_run = m_new;
                 }
             }
+            if (bad) break;
             const float mc = m_run == -INFINITY ? 0.f : m_run * C2;
             uint32_t pk[16];
             float l4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -609,32 +620,46 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                 pk[c] = pack_f16x2(p0, p1);
             }
             l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            tc_st16(sbuf + 16u * half, pk);  // P of keys 32 half .. + 31: columns 16 half .. + 15
+            tc_st16(sbuf, pk);  // P of this half's keys: its columns 32 half .. + 15
             tc_wait_st();
             tc_fence_before();
             mbar_arrive(BAR(BAR_P_FULL + (i & 1)));
 
             if (seg_end) {
                 const bool ok = wait_warp(BAR(BAR_KV_FREE + i % NF), (i / NF) & 1, abort_flag);
-                redl[half * 128 + r] = l_run;
-                // both halves' sums posted
-                if (bar_red_or(pair_bar, 64, bad || !ok)) break;
+                float* rm = red + (n_end & 1) * 512;  // [max, sum][half][row]
+                rm[half * 128 + r] = m_run == -INFINITY ? -INFINITY : m_run * C2;
+                rm[256 + half * 128 + r] = l_run;
+                mbar_arrive(BAR(BAR_PAIR + qd));  // both halves' (max, sum) posted
+                if (!ok || !wait_warp(BAR(BAR_PAIR + qd), n_end & 1, abort_flag)) break;
+                ++n_end;
+                const float m0 = rm[r], m1 = rm[128 + r];
+                const float m = fmaxf(m0, m1);
+                const float a0 = m == -INFINITY ? 0.f : fast_exp2(m0 - m);
+                const float a1 = m == -INFINITY ? 0.f : fast_exp2(m1 - m);
+                const float l = a0 * rm[256 + r] + a1 * rm[384 + r];
                 tc_fence_after();
+                // dims 32 half .. + 31 of this row's head from both accumulators
                 const uint32_t oa = tmem + TM_O + 64u * g + 32u * half + lane_base;
-                uint32_t o[32];
-                tc_ld32(oa, o);
+                uint32_t o0[32], o1[32];
+                tc_ld32(oa, o0);
+                tc_ld32(oa + TM_O_HALF, o1);
                 tc_wait_ld();
                 if (j < seg_len) {
                     const size_t slot = static_cast<size_t>(blockIdx.x) + cb;
                     const size_t base = (slot * p.lt + j) * HQ + qh;
                     float4* dst = reinterpret_cast<float4*>(p.part_o + base * HD + 32 * half);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        dst[q] = make_float4(__uint_as_float(o[4 * q]), __uint_as_float(o[4 * q + 1]),
-                                             __uint_as_float(o[4 * q + 2]), __uint_as_float(o[4 * q + 3]));
+                    for (int q = 0; q < 8; ++q) {
+                        float v[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            v[e] = a0 * __uint_as_float(o0[4 * q + e]) + a1 * __uint_as_float(o1[4 * q + e]);
+                        dst[q] = make_float4(v[0], v[1], v[2], v[3]);
+                    }
                     if (half == 0) {
-                        p.part_ml[base * 2 + 0] = m_run * C2;
-                        p.part_ml[base * 2 + 1] = redl[r] + redl[128 + r];
+                        p.part_ml[base * 2 + 0] = m;
+                        p.part_ml[base * 2 + 1] = l;
                     }
                 }
                 tc_fence_before();
