@@ -28,15 +28,16 @@
 //   MMA warp 12       S(i) = A . K(i)^T into tensor memory (double-buffered),
 //                     then O += P(i-1) . V(i-1) with P read from tensor memory.
 //   softmax warps 0-7 two threads per row (warps w and w + 4 share the
-//                     tensor-memory lanes of rows 32 (w % 4) .. + 31): half h
-//                     takes keys 32h .. 32h + 31 of every tile and runs its
-//                     own online softmax over them (own running max and sum,
-//                     own O accumulator O_h, lazy rescaling: O_h is rescaled
-//                     in tensor memory only when its max grows by more than
-//                     2^8), P as fp16 back into its own S columns; at a
-//                     request's last tile the halves merge (m, l) through
-//                     shared memory and each writes half the dims of
-//                     a0 O_0 + a1 O_1 to the partial.
+//                     tensor-memory lanes of rows 32 (w % 4) .. + 31): warp
+//                     w takes the tiles of parity w / 4, all 64 keys, and runs
+//                     its own online softmax over them (own running max and
+//                     sum, own O accumulator O_par, lazy rescaling: O_par is
+//                     rescaled in tensor memory only when its max grows by
+//                     more than 2^8), P as fp16 back into the S columns; the
+//                     two work on consecutive tiles at the same time.  At a
+//                     request's last tile they merge (m, l) through shared
+//                     memory and each writes half the dims of a0 O_0 + a1 O_1
+//                     to the partial.
 // Synchronisation by mbarriers; every wait is bounded (an expired wait sets
 // the step's error word and the CTA winds down, waits for its MMAs and frees
 // its tensor memory).
@@ -72,15 +73,15 @@ constexpr uint32_t TM_Q = 0;                  // A operand (fp16 pairs) of even 
 constexpr uint32_t TM_Q1 = 192;               // A operand of odd items (an item's A may be written
                                               // while the previous item's last S MMAs still read theirs)
 constexpr uint32_t TM_S = 64;                 // S buffer b at TM_S + 64 b (P aliases its first 32)
-constexpr uint32_t TM_O = 256;                // O_0, O_1 (keys 0-31 / 32-63 of every tile), 128
-constexpr uint32_t TM_O_HALF = 128;           // columns each (head 0 dims | head 1 dims)
+constexpr uint32_t TM_O = 256;                // O_0, O_1 (even / odd tiles), 128 columns each
+constexpr uint32_t TM_O_HALF = 128;           // (head 0 dims | head 1 dims)
 constexpr float RESCALE_LOG2 = 8.f;           // lazy rescale threshold (P stays <= 2^8)
 
 // mbarrier indices
 constexpr int BAR_KV_READY = 0;   // [NF] converted tile (and A operand) ready  (128 loader arrivals)
 constexpr int BAR_KV_FREE = 3;    // [NF] PV of the tile done: buffers free      (MMA commit)
 constexpr int BAR_S_FULL = 6;     // [2] S of the tile in tensor memory          (MMA commit)
-constexpr int BAR_P_FULL = 8;     // [2] P of the tile in tensor memory          (256 softmax arrivals)
+constexpr int BAR_P_FULL = 8;     // [2] P of the tile in tensor memory          (128 softmax arrivals)
 constexpr int BAR_O_FREE = 10;    // O read out at a request's last tile         (256 softmax arrivals)
 constexpr int BAR_MMA_DONE = 11;  // teardown: all MMAs done                     (MMA commit)
 constexpr int BAR_PAIR = 12;      // [4] softmax pair qd posted its halves' (max, sum) at a request's end (64)
@@ -155,8 +156,8 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
         }
         mbar_init(BAR(BAR_S_FULL), 1);
         mbar_init(BAR(BAR_S_FULL + 1), 1);
-        mbar_init(BAR(BAR_P_FULL), SOFT);
-        mbar_init(BAR(BAR_P_FULL + 1), SOFT);
+        mbar_init(BAR(BAR_P_FULL), SOFT / 2);
+        mbar_init(BAR(BAR_P_FULL + 1), SOFT / 2);
         mbar_init(BAR(BAR_O_FREE), SOFT);
         mbar_init(BAR(BAR_MMA_DONE), 1);
         for (int q = 0; q < 4; ++q) mbar_init(BAR(BAR_PAIR + q), 64);
@@ -441,37 +442,36 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
         constexpr uint32_t ID_S = idesc_f16_f32(128, TK, 0);  // S: A . K^T, K-major B
         constexpr uint32_t ID_O = idesc_f16_f32(128, 64, 1);  // O: P . V, MN-major B
         const uint32_t f16_base = smem_addr(f16);
-        // O_h += P(k)[keys of half h] . V(k)[same keys], per KV head's dims (N = 64):
-        // P of keys 0-31 sits in S columns 0-15, of keys 32-63 in columns 32-47.
-        auto issue_pv = [&](int k, bool first, int seg) {
+        // O_(k & 1) += P(k) . V(k), per KV head's dims (N = 64); `pos` is k's
+        // index within its request (the first tile of each parity overwrites).
+        auto issue_pv = [&](int k, int pos, int seg) {
             if (!wait_warp(BAR(BAR_P_FULL + (k & 1)), (k >> 1) & 1, abort_flag)) return false;
-            if (first && seg >= 1 && !wait_warp(BAR(BAR_O_FREE), (seg - 1) & 1, abort_flag)) return false;
+            if (pos == 0 && seg >= 1 && !wait_warp(BAR(BAR_O_FREE), (seg - 1) & 1, abort_flag)) return false;
             tc_fence_after();
             const uint32_t vbuf = f16_base + (k % NF) * F16_BUF + F16_TILE;
             const uint32_t pa = tmem + TM_S + 64u * (k & 1);
-            const uint32_t av[4] = {pa, pa + 8u, pa + 32u, pa + 40u};
+            const uint32_t av[4] = {pa, pa + 8u, pa + 16u, pa + 24u};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const uint32_t vb = vbuf + h * HALF_TILE;
                 const uint64_t bd[4] = {smem_desc_sw128(vb), smem_desc_sw128(vb + 2048),
                                         smem_desc_sw128(vb + 4096), smem_desc_sw128(vb + 6144)};
-                tc_mma_ts2x2(tmem + TM_O + 64u * h, tmem + TM_O + TM_O_HALF + 64u * h, av, bd, ID_O,
-                             first ? 0u : 1u);
+                tc_mma_ts4(tmem + TM_O + TM_O_HALF * (k & 1) + 64u * h, av, bd, ID_O, pos >= 2 ? 1u : 0u);
             }
             tc_commit(BAR(BAR_KV_FREE + k % NF));
             return true;
         };
         int ct = t0, cb = find_req(t0);
-        int seg_b = -1, seg = -1;
-        bool prev_first = false;
+        int seg_b = -1, seg = -1, seg_i0 = 0;  // current request, its count and first tile here
+        int prev_pos = 0;
         int prev_seg = -1;
         bool ok = true;
         int i = 0;
         for (; ct < t1; ++i) {
-            const bool first = cb != seg_b;
-            if (first) {
+            if (cb != seg_b) {
                 seg_b = cb;
                 ++seg;
+                seg_i0 = i;
             }
             if (!wait_warp(BAR(BAR_KV_READY + i % NF), (i / NF) & 1, abort_flag)) {
                 ok = false;
@@ -490,15 +490,15 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                 tc_mma_ts4(sd, aq, bd, ID_S, hk > 0 ? 1u : 0u);
             }
             tc_commit(BAR(BAR_S_FULL + (i & 1)));
-            if (i > 0 && !issue_pv(i - 1, prev_first, prev_seg)) {
+            if (i > 0 && !issue_pv(i - 1, prev_pos, prev_seg)) {
                 ok = false;
                 break;
             }
-            prev_first = first;
+            prev_pos = i - seg_i0;
             prev_seg = seg;
             advance(ct, cb);
         }
-        if (ok && i > 0) issue_pv(i - 1, prev_first, prev_seg);
+        if (ok && i > 0) issue_pv(i - 1, prev_pos, prev_seg);
         // every MMA this warp issued is done before the tensor memory is freed
         tc_commit(BAR(BAR_MMA_DONE));
         const bool done = wait_bounded(BAR(BAR_MMA_DONE), 0, abort_flag, false, TEARDOWN_LIMIT_NS);
@@ -507,19 +507,20 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
     } else {
         // =================== softmax: two threads per row ===================
         // Warps w and w + 4 share the tensor-memory lanes of rows 32 (w % 4) ..
-        // + 31; half h = w / 4 takes keys 32h .. 32h + 31 of every tile with its
-        // own running max, sum and O accumulator, so the two never wait for
-        // each other until a request's last tile, where they merge through
-        // shared memory (double-buffered by request parity) after meeting at
-        // the pair's mbarrier (a bounded wait, as every other).
-        const int half = warp >> 2, qd = warp & 3;
+        // + 31; warp w takes the tiles of parity par = w / 4 (all 64 keys) with
+        // its own running max, sum and O accumulator, so the two work on
+        // consecutive tiles at once and never wait for each other until a
+        // request's last tile, where they merge through shared memory
+        // (double-buffered by request parity) after meeting at the pair's
+        // mbarrier (a bounded wait, as every other).
+        const int par = warp >> 2, qd = warp & 3;
         const int r = 32 * qd + (tid & 31);
         const int g = r >> 6, j = (r >> 3) & 7, qh = g * GRP + (r & 7);
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
-        const uint32_t o_own = tmem + TM_O + TM_O_HALF * half + 64u * g + lane_base;  // O_half, this row's head
+        const uint32_t o_own = tmem + TM_O + TM_O_HALF * par + 64u * g + lane_base;  // O_par, this row's head
         int ct = t0, cb = find_req(t0);
         int seg_b = -1, seg_t1 = 0, k0 = 0;  // current request, end of its tiles here, tile key
-        float m_run = -INFINITY, l_run = 0.f;  // this half's running max (raw score units) and sum
+        float m_run = -INFINITY, l_run = 0.f;  // running max (raw score units) and sum over this parity's tiles
         int lo_j = INT_MAX, hi_j = -1;
         int seg_len = 0;  // tokens of the current item
         int n_end = 0;    // requests finished here
@@ -546,101 +547,119 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             }
             const bool seg_end = ct + 1 >= seg_t1;
 
-            if (!wait_warp(BAR(BAR_S_FULL + (i & 1)), (i >> 1) & 1, abort_flag)) break;
-            tc_fence_after();
-            // this half's S (columns 32 half ..) and, later, its P (columns 32 half .. + 15)
-            const uint32_t sbuf = tmem + TM_S + 64u * (i & 1) + 32u * half + lane_base;
-            uint32_t sr[32];
-            tc_ld32(sbuf, sr);
-            tc_wait_ld();
-            float s[32];
-            const int kb0 = k0 + 32 * half;
-            const int cmin = lo_j == INT_MAX ? 32 : lo_j - kb0;
-            const int cmax = hi_j - kb0;
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            if (cmin <= 0 && cmax >= 31) {
+            if ((i & 1) == par) {
+                if (!wait_warp(BAR(BAR_S_FULL + par), (i >> 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t sbuf = tmem + TM_S + 64u * par + lane_base;
+                const int cmin = lo_j == INT_MAX ? TK : lo_j - k0;
+                const int cmax = hi_j - k0;
+                const bool full = cmin <= 0 && cmax >= TK - 1;
+                uint32_t sr[32];
+                // pass 1: the row's max over the tile's 64 keys (two 32-column loads)
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(sr[c]);
-            } else {
+                for (int ch = 0; ch < 2; ++ch) {
+                    tc_ld32(sbuf + 32u * ch, sr);
+                    tc_wait_ld();
+                    if (!full) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) s[c] = (c < cmin || c > cmax) ? -INFINITY : __uint_as_float(sr[c]);
-            }
-#pragma unroll
-            for (int c = 0; c < 32; c += 8) {
-                m4[c >> 3] = fmax3(m4[c >> 3], s[c], s[c + 1]);
-                m4[c >> 3] = fmax3(m4[c >> 3], s[c + 2], s[c + 3]);
-                m4[c >> 3] = fmax3(m4[c >> 3], s[c + 4], s[c + 5]);
-                m4[c >> 3] = fmax3(m4[c >> 3], s[c + 6], s[c + 7]);
-            }
-            const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
-            // lazy rescale: O_half (in tensor memory) is corrected only when this
-            // half's max grows a lot
-            const float m_new = fmaxf(m_run, mx);
-            bool corr = false;
-            if (m_new > m_run) {
-                if (m_run == -INFINITY || seg_start || (m_new - m_run) * C2 <= RESCALE_LOG2) {
-                    if (m_run == -INFINITY || seg_start) m_run = m_new;
-                } else {
-                    corr = true;
-                }
-            }
-            bool bad = false;
-            if (__any_sync(0xffffffffu, corr)) {
-                // PV(i - 1) of this request must be done before O is touched
-                const bool ok = wait_warp(BAR(BAR_KV_FREE + (i - 1) % NF), ((i - 1) / NF) & 1, abort_flag);
-                const float alpha = corr ? fast_exp2((m_run - m_new) * C2) : 1.f;
-                if (ok) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        uint32_t o[32];
-                        tc_ld32(o_own + 32u * q, o);
-                        tc_wait_ld();
-#pragma unroll
-                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                        tc_st32(o_own + 32u * q, o);
+                        for (int c = 0; c < 32; ++c)
+                            if (32 * ch + c < cmin || 32 * ch + c > cmax) sr[c] = __float_as_uint(-INFINITY);
                     }
-                    tc_wait_st();
-                }
-                bad = !ok;
-                if (corr) {
-                    l_run *= alpha;
-                    m_run = m_new;
-                }
-            }
-            if (bad) break;
-            const float mc = m_run == -INFINITY ? 0.f : m_run * C2;
-            uint32_t pk[16];
-            float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const float p0 = fast_exp2(fmaf(s[2 * c], C2, -mc));
-                const float p1 = fast_exp2(fmaf(s[2 * c + 1], C2, -mc));
-                l4[c & 3] += p0 + p1;
-                pk[c] = pack_f16x2(p0, p1);
+                    for (int c = 0; c < 32; c += 8) {
+                        m4[c >> 3] = fmax3(m4[c >> 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                        m4[c >> 3] = fmax3(m4[c >> 3], __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+                        m4[c >> 3] = fmax3(m4[c >> 3], __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+                        m4[c >> 3] = fmax3(m4[c >> 3], __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+                    }
+                }
+                const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+                // lazy rescale: O_par (in tensor memory) is corrected only when
+                // this warp's max grows a lot
+                const float m_new = fmaxf(m_run, mx);
+                bool corr = false;
+                if (m_new > m_run) {
+                    if (m_run == -INFINITY || (m_new - m_run) * C2 <= RESCALE_LOG2) {
+                        if (m_run == -INFINITY) m_run = m_new;
+                    } else {
+                        corr = true;
+                    }
+                }
+                bool bad = false;
+                if (__any_sync(0xffffffffu, corr)) {
+                    // P.V of this warp's previous tile (i - 2, same request) must be
+                    // done before O_par is touched
+                    const bool ok = wait_warp(BAR(BAR_KV_FREE + (i - 2) % NF), ((i - 2) / NF) & 1, abort_flag);
+                    const float alpha = corr ? fast_exp2((m_run - m_new) * C2) : 1.f;
+                    if (ok) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            uint32_t o[32];
+                            tc_ld32(o_own + 32u * q, o);
+                            tc_wait_ld();
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                            tc_st32(o_own + 32u * q, o);
+                        }
+                        tc_wait_st();
+                    }
+                    bad = !ok;
+                    if (corr) {
+                        l_run *= alpha;
+                        m_run = m_new;
+                    }
+                }
+                if (bad) break;
+                // pass 2: P = 2^(s - m) for each 32-key half, written as fp16 over the
+                // S columns already read (keys 32 ch .. -> columns 16 ch ..)
+                const float mc = m_run == -INFINITY ? 0.f : m_run * C2;
+                float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    tc_ld32(sbuf + 32u * ch, sr);
+                    tc_wait_ld();
+                    if (!full) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (32 * ch + c < cmin || 32 * ch + c > cmax) sr[c] = __float_as_uint(-INFINITY);
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * c]), C2, -mc));
+                        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), C2, -mc));
+                        l4[c & 3] += p0 + p1;
+                        pk[c] = pack_f16x2(p0, p1);
+                    }
+                    tc_st16(sbuf + 16u * ch, pk);
+                }
+                l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+                tc_wait_st();
+                tc_fence_before();
+                mbar_arrive(BAR(BAR_P_FULL + par));
             }
-            l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            tc_st16(sbuf, pk);  // P of this half's keys: its columns 32 half .. + 15
-            tc_wait_st();
-            tc_fence_before();
-            mbar_arrive(BAR(BAR_P_FULL + (i & 1)));
 
             if (seg_end) {
+                // the request's last P.V (in MMA order, every earlier one too) done
                 const bool ok = wait_warp(BAR(BAR_KV_FREE + i % NF), (i / NF) & 1, abort_flag);
-                float* rm = red + (n_end & 1) * 512;  // [max, sum][half][row]
-                rm[half * 128 + r] = m_run == -INFINITY ? -INFINITY : m_run * C2;
-                rm[256 + half * 128 + r] = l_run;
-                mbar_arrive(BAR(BAR_PAIR + qd));  // both halves' (max, sum) posted
+                float* rm = red + (n_end & 1) * 512;  // [max, sum][parity][row]
+                rm[par * 128 + r] = m_run == -INFINITY ? -INFINITY : m_run * C2;
+                rm[256 + par * 128 + r] = l_run;
+                mbar_arrive(BAR(BAR_PAIR + qd));  // both warps' (max, sum) posted
                 if (!ok || !wait_warp(BAR(BAR_PAIR + qd), n_end & 1, abort_flag)) break;
                 ++n_end;
                 const float m0 = rm[r], m1 = rm[128 + r];
                 const float m = fmaxf(m0, m1);
-                const float a0 = m == -INFINITY ? 0.f : fast_exp2(m0 - m);
-                const float a1 = m == -INFINITY ? 0.f : fast_exp2(m1 - m);
+                // a parity with no tile of this request (or only masked keys) has
+                // weight 0; its accumulator may hold another request's values
+                const float a0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - m);
+                const float a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - m);
                 const float l = a0 * rm[256 + r] + a1 * rm[384 + r];
                 tc_fence_after();
-                // dims 32 half .. + 31 of this row's head from both accumulators
-                const uint32_t oa = tmem + TM_O + 64u * g + 32u * half + lane_base;
+                // dims 32 par .. + 31 of this row's head from both accumulators
+                const uint32_t oa = tmem + TM_O + 64u * g + 32u * par + lane_base;
                 uint32_t o0[32], o1[32];
                 tc_ld32(oa, o0);
                 tc_ld32(oa + TM_O_HALF, o1);
@@ -648,16 +667,19 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                 if (j < seg_len) {
                     const size_t slot = static_cast<size_t>(blockIdx.x) + cb;
                     const size_t base = (slot * p.lt + j) * HQ + qh;
-                    float4* dst = reinterpret_cast<float4*>(p.part_o + base * HD + 32 * half);
+                    float4* dst = reinterpret_cast<float4*>(p.part_o + base * HD + 32 * par);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         float v[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            v[e] = a0 * __uint_as_float(o0[4 * q + e]) + a1 * __uint_as_float(o1[4 * q + e]);
+                        for (int e = 0; e < 4; ++e) {
+                            const float x0 = a0 != 0.f ? a0 * __uint_as_float(o0[4 * q + e]) : 0.f;
+                            const float x1 = a1 != 0.f ? a1 * __uint_as_float(o1[4 * q + e]) : 0.f;
+                            v[e] = x0 + x1;
+                        }
                         dst[q] = make_float4(v[0], v[1], v[2], v[3]);
                     }
-                    if (half == 0) {
+                    if (par == 0) {
                         p.part_ml[base * 2 + 0] = m;
                         p.part_ml[base * 2 + 1] = l;
                     }
