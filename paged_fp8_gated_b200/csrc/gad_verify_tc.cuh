@@ -85,8 +85,8 @@ constexpr int BAR_P_FULL = 8;     // [2] P of the tile in tensor memory         
 constexpr int BAR_O_FREE = 10;    // O read out at a request's last tile         (256 softmax arrivals)
 constexpr int BAR_MMA_DONE = 11;  // teardown: all MMAs done                     (MMA commit)
 constexpr int BAR_PAIR = 12;      // [4] softmax pair qd posted its halves' (max, sum) at a request's end (64)
-constexpr int BAR_RAW = 16;       // [NS] page size 64: the tile's K and V pages landed (TMA bytes)
-constexpr int NBARS = 16;         // + NS for page size 64
+constexpr int BAR_RAW = 16;       // [NS] the tile's K and V rows landed (TMA bytes, or 128 gathers' arrivals)
+constexpr int NBARS = 16;         // + NS
 
 template <int NS>
 struct Cfg {
@@ -161,8 +161,9 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
         mbar_init(BAR(BAR_O_FREE), SOFT);
         mbar_init(BAR(BAR_MMA_DONE), 1);
         for (int q = 0; q < 4; ++q) mbar_init(BAR(BAR_PAIR + q), 64);
-        if (PS == 64)
-            for (int st = 0; st < NS; ++st) mbar_init(BAR(BAR_RAW + st), 1);
+        // raw stages: the TMA page loads' bytes (one arrival), or the
+        // gathers of one softmax parity group (128 tracked arrivals)
+        for (int st = 0; st < NS; ++st) mbar_init(BAR(BAR_RAW + st), PS == 64 ? 1 : SOFT / 2);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -192,121 +193,111 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
     auto tile_k0 = [&](int tau, int b) { return (rlo[b] / TK + (tau - tpre[b])) * TK; };
     const float C2 = __ldg(p.k_scale) * 0.125f * 1.4426950408889634f;  // raw score -> log2 units
 
+    bool prep_done = false;
+    auto ensure_prep = [&]() {
+        if (!prep_done) {
+            pdl_wait_primary();
+            prep_done = true;
+        }
+    };
+    // A cursor over the tile list that keeps its item's data in registers:
+    // shared memory is read only when it enters a new item (a chain of
+    // dependent shared-memory reads per tile slowed the loaders).
+    struct Cur {
+        int tau, b, end, k0, lo, hi, rnew;
+        const int32_t* pt;  // page-table row of the item's request
+        size_t gofs;        // byte offset of the item's head group in a cache row
+    };
+    auto cur_enter = [&](Cur& c) {  // c.tau and c.b set
+        c.end = tpre[c.b + 1];
+        c.lo = rlo[c.b];
+        c.hi = rhi[c.b];
+        c.rnew = rnew[c.b];
+        c.k0 = (c.lo / TK + (c.tau - tpre[c.b])) * TK;
+        const ItemRef it = item_ref<MULTI>(p, c.b);
+        c.pt = p.page_table + static_cast<size_t>(it.req) * p.max_pages;
+        c.gofs = static_cast<size_t>(it.grp) * ROWB;
+    };
+    auto cur_init = [&](Cur& c, int tau) {
+        c.tau = tau;
+        c.b = find_req(tau);
+        cur_enter(c);
+    };
+    auto cur_next = [&](Cur& c) {
+        ++c.tau;
+        c.k0 += TK;
+        if (c.tau >= c.end && c.tau < t1 && c.b < B - 1) {
+            do {
+                ++c.b;
+            } while (c.b < B - 1 && c.tau >= tpre[c.b + 1]);
+            cur_enter(c);
+        }
+    };
+    // rows this step writes (the prep kernel, which may still run) are read
+    // only after it has finished
+    auto k_needs_prep = [&](const Cur& c) { return c.k0 + TK - 1 >= c.rnew; };
+    // Page size 1: the softmax warps gather the K and V rows (warps that issue
+    // cp.async limit the gather rate, and the loaders have the conversion to
+    // do).  One parity group (128 threads) fills one tile's raw stage: thread t
+    // copies 16-byte chunk t % 8 of rows t / 8 + 16 q (q < 4) for K and V, so
+    // that eight lanes cover a whole 128-byte row, then lets the stage's
+    // mbarrier track its copies.
+    const size_t row_pitch = static_cast<size_t>(ROWB) * ng;
+    auto row_entries = [&](const Cur& c, int gt, int (&e)[4]) {  // page-table entries of the rows, or -1
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int k = c.k0 + (gt >> 3) + 16 * q;
+            e[q] = (c.tau < t1 && k >= c.lo && k <= c.hi && k < p.max_pages) ? __ldg(c.pt + k) : -1;
+        }
+    };
+    auto gather_rows = [&](const Cur& c, int gt, const int (&e)[4]) {
+        if (k_needs_prep(c)) ensure_prep();
+        const int jc = gt & 7;
+        const uint32_t base = smem_addr(raw + ((c.tau - t0) % NS) * RAW_STAGE);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = (gt >> 3) + 16 * q;
+            const bool ok = e[q] >= 0 && e[q] < p.num_rows;
+            const size_t off = ok ? static_cast<size_t>(e[q]) * row_pitch + c.gofs + 16 * jc : 0;
+            const uint32_t d = base + r * ROWB + ((jc ^ (r & 7)) << 4);
+            cp_async16(d, p.k_cache + off, ok ? 16 : 0);
+            cp_async16(d + TK * ROWB, p.v_cache + off, ok ? 16 : 0);
+        }
+        cp_async_mbar_arrive_noinc(BAR(BAR_RAW + (c.tau - t0) % NS));
+    };
+
     if (warp >= LOAD_W0 && warp < MMA_WARP) {
         // =================== loaders: gather, convert, A operand ===================
         const int ltid = tid - LOAD_T0;
-        bool prep_done = false;
-        auto ensure_prep = [&]() {
-            if (!prep_done) {
-                pdl_wait_primary();
-                prep_done = true;
-            }
-        };
-        // A cursor over the tile list that keeps its item's data in registers:
-        // shared memory is read only when it enters a new item (a chain of
-        // dependent shared-memory reads per tile slowed the loaders).
-        struct Cur {
-            int tau, b, end, k0, lo, hi, rnew;
-            const int32_t* pt;  // page-table row of the item's request
-            size_t gofs;        // byte offset of the item's head group in a cache row
-        };
-        auto cur_enter = [&](Cur& c) {  // c.tau and c.b set
-            c.end = tpre[c.b + 1];
-            c.lo = rlo[c.b];
-            c.hi = rhi[c.b];
-            c.rnew = rnew[c.b];
-            c.k0 = (c.lo / TK + (c.tau - tpre[c.b])) * TK;
-            const ItemRef it = item_ref<MULTI>(p, c.b);
-            c.pt = p.page_table + static_cast<size_t>(it.req) * p.max_pages;
-            c.gofs = static_cast<size_t>(it.grp) * ROWB;
-        };
-        auto cur_init = [&](Cur& c, int tau) {
-            c.tau = tau;
-            c.b = find_req(tau);
-            cur_enter(c);
-        };
-        auto cur_next = [&](Cur& c) {
-            ++c.tau;
-            c.k0 += TK;
-            if (c.tau >= c.end && c.tau < t1 && c.b < B - 1) {
-                do {
-                    ++c.b;
-                } while (c.b < B - 1 && c.tau >= tpre[c.b + 1]);
-                cur_enter(c);
-            }
-        };
+        // Page size 64: the loaders fetch each tile's page index (NS - 1 tiles
+        // ahead of its load) and issue its two TMA page loads.
         auto issue_idx = [&](const Cur& c) {
             if (c.tau >= t1) return;
             int* dst = idx_smem + ((c.tau - t0) % C::IDX_SLOTS) * TK;
-            if (PS == 1) {
-                if (ltid < TK) {
-                    const int k = c.k0 + ltid;
-                    if (k >= c.lo && k <= c.hi && k < p.max_pages) cp_async4(smem_addr(dst + ltid), c.pt + k);
-                    else dst[ltid] = -1;
-                }
-            } else {
-                if (ltid < TK / PS) {
-                    const int pg = c.k0 / PS + ltid;
-                    if (pg < p.max_pages) cp_async4(smem_addr(dst + ltid), c.pt + pg);
-                    else dst[ltid] = -1;
-                }
+            if (ltid < TK / PS) {
+                const int pg = c.k0 / PS + ltid;
+                if (pg < p.max_pages) cp_async4(smem_addr(dst + ltid), c.pt + pg);
+                else dst[ltid] = -1;
             }
         };
-        int n_kv_issued = 0;  // tiles whose gathers were issued (the same count in every loader)
+        int n_kv_issued = 0;  // tiles whose page loads were issued (the same count in every loader)
         auto issue_kv = [&](const Cur& c) {
             if (c.tau >= t1) return;
-            const int k0 = c.k0;
-            if (k0 + TK - 1 >= c.rnew) ensure_prep();
+            if (k_needs_prep(c)) ensure_prep();
             const int* ix = idx_smem + ((c.tau - t0) % C::IDX_SLOTS) * TK;
             const uint32_t base = smem_addr(raw + ((c.tau - t0) % NS) * RAW_STAGE);
             ++n_kv_issued;
-            if constexpr (PS == 64) {
-                // the tile is one page: its K and V rows by two TMA tile loads
-                // (128-byte swizzle, the layout the gathers below write); a page
-                // index past the table (-1) or rows past the cache fall outside the
-                // tensor and read as zeros
-                if (ltid == 0) {
-                    const int pg = ix[0];
-                    const int y = pg >= 0 ? pg * PS : -PS;
-                    const uint32_t bar = BAR(BAR_RAW + (c.tau - t0) % NS);
-                    mbar_arrive_expect_tx(bar, RAW_STAGE);
-                    tma_load_2d(base, &kmap, static_cast<int>(c.gofs), y, bar);
-                    tma_load_2d(base + TK * ROWB, &vmap, static_cast<int>(c.gofs), y, bar);
-                }
-                return;
-            }
-            const int lo = c.lo, hi = c.hi;
-            const size_t row_pitch = static_cast<size_t>(ROWB) * ng;
-            const size_t gofs = c.gofs;
-            constexpr int ROWS = TK * 8 / LOADERS;  // rows per thread
-            const int j = ltid & 7;                 // 16-byte chunk
-            // all page-table reads first, then the copies (the copies are ordered
-            // asm statements the reads could not move across)
-            int pix[ROWS];
-#pragma unroll
-            for (int i = 0; i < ROWS; ++i) {
-                const int r = (ltid >> 3) + (LOADERS / 8) * i;
-                pix[i] = PS == 1 ? ix[r] : ix[r / PS];
-            }
-            size_t off[ROWS];
-            int nbytes[ROWS];
-#pragma unroll
-            for (int i = 0; i < ROWS; ++i) {
-                const int r = (ltid >> 3) + (LOADERS / 8) * i;
-                const int k = k0 + r;
-                int64_t crow;
-                if (PS == 1) crow = pix[i];
-                else crow = pix[i] >= 0 ? static_cast<int64_t>(pix[i]) * PS + r % PS : -1;
-                const bool ok = k >= lo && k <= hi && crow >= 0 && crow < p.num_rows;
-                off[i] = ok ? static_cast<size_t>(crow) * row_pitch + gofs + j * 16 : 0;
-                nbytes[i] = ok ? 16 : 0;
-            }
-#pragma unroll
-            for (int i = 0; i < ROWS; ++i) {
-                const int r = (ltid >> 3) + (LOADERS / 8) * i;
-                const uint32_t d = base + r * ROWB + ((j ^ (r & 7)) << 4);
-                cp_async16(d, p.k_cache + off[i], nbytes[i]);
-                cp_async16(d + TK * ROWB, p.v_cache + off[i], nbytes[i]);
+            // the tile is one page: its K and V rows by two TMA tile loads
+            // (128-byte swizzle, the layout the page-size-1 gathers write); a page
+            // index past the table (-1) or rows past the cache fall outside the
+            // tensor and read as zeros
+            if (ltid == 0) {
+                const int pg = ix[0];
+                const int y = pg >= 0 ? pg * PS : -PS;
+                const uint32_t bar = BAR(BAR_RAW + (c.tau - t0) % NS);
+                mbar_arrive_expect_tx(bar, RAW_STAGE);
+                tma_load_2d(base, &kmap, static_cast<int>(c.gofs), y, bar);
+                tma_load_2d(base + TK * ROWB, &vmap, static_cast<int>(c.gofs), y, bar);
             }
         };
         // A operand of item b's S MMA: row ltid = [q | 0] (KV head 0) or [0 | q].
@@ -369,33 +360,35 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             }
         };
 
-        Cur xc, kc, cc;  // page-table cursor (NS - 1 tiles ahead), gather cursor, current tile
+        Cur xc, kc, cc;  // page-index cursor (NS - 1 tiles ahead), page-load cursor, current tile
         cur_init(xc, t0);
         kc = xc;
         cc = xc;
-        for (int d = 0; d < NS - 1; ++d) {
-            issue_idx(xc);
-            cur_next(xc);
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
-        bar_red_or(1, LOADERS, false);
-        for (int d = 0; d < NS - 1; ++d) {
-            issue_kv(kc);
-            cur_next(kc);
-            issue_idx(xc);
-            cur_next(xc);
+        if (PS == 64) {
+            for (int d = 0; d < NS - 1; ++d) {
+                issue_idx(xc);
+                cur_next(xc);
+            }
             cp_async_commit();
+            cp_async_wait<0>();
+            bar_red_or(1, LOADERS, false);
+            for (int d = 0; d < NS - 1; ++d) {
+                issue_kv(kc);
+                cur_next(kc);
+                issue_idx(xc);
+                cur_next(xc);
+                cp_async_commit();
+            }
         }
         int seg_b = -1, nseg = 0;
         const int n_tiles = t1 - t0;
         int i = 0;
         for (; i < n_tiles; ++i) {
-            cp_async_wait<NS - 2>();
+            if (PS == 64) cp_async_wait<NS - 2>();  // the page indices NS - 1 tiles ahead
             const int cb = cc.b;
             const bool seg_start = cb != seg_b;
-            bool bad = false;
-            if (PS == 64) bad = !wait_bounded(BAR(BAR_RAW + i % NS), (i / NS) & 1, abort_flag);
+            // tile i's raw stage filled (page loads, or the softmax warps' gathers)
+            bool bad = !wait_bounded(BAR(BAR_RAW + i % NS), (i / NS) & 1, abort_flag);
             // buffers i % NF are free once PV(i - NF) is done, which also means every
             // S MMA up to tile i - NF + 1 is done: the A operand this item takes
             // (the one of the item before the previous) is no longer read.  Tile 2
@@ -403,8 +396,8 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             if (i >= NF && !bad) bad = !wait_bounded(BAR(BAR_KV_FREE + i % NF), ((i - NF) / NF) & 1, abort_flag);
             static_assert(NF == 3, "the A-operand wait below assumes three buffers");
             if (i == 2 && seg_start && nseg >= 2 && !bad) bad = !wait_bounded(BAR(BAR_S_FULL), 0, abort_flag);
-            // past this barrier: tile i landed for every loader, and every loader
-            // has converted tile i - 1, so its raw stage may be refilled
+            // past this barrier: every loader has converted tile i - 1, so its raw
+            // stage may be refilled
             if (bar_red_or(1, LOADERS, bad)) break;
             if (seg_start) {
                 write_q(cb, (nseg & 1) ? TM_Q1 : TM_Q);
@@ -418,13 +411,15 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                 tc_fence_before();
             }
             mbar_arrive(BAR(BAR_KV_READY + i % NF));
-            // gathers for tile i + NS - 1 (into the stage of tile i - 1), off the
+            // page loads for tile i + NS - 1 (into the stage of tile i - 1), off the
             // path from "buffer free" to "tile ready"
-            issue_kv(kc);
-            cur_next(kc);
-            issue_idx(xc);
-            cur_next(xc);
-            cp_async_commit();
+            if (PS == 64) {
+                issue_kv(kc);
+                cur_next(kc);
+                issue_idx(xc);
+                cur_next(xc);
+                cp_async_commit();
+            }
             cur_next(cc);
         }
         cp_async_wait<0>();
@@ -524,6 +519,25 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
         int lo_j = INT_MAX, hi_j = -1;
         int seg_len = 0;  // tokens of the current item
         int n_end = 0;    // requests finished here
+        // page size 1: this group gathers tiles par, par + 2, .. below NS - 1
+        // now, and tile i + NS - 1 once it has taken tile i (whose S MMA being
+        // done means tile i - 1 is converted, so that stage is free)
+        const int gt = tid & 127;
+        Cur gc;
+        int pend[4] = {-1, -1, -1, -1};  // page-table entries of this thread's rows in tile gc, loaded a tile early
+        if (PS == 1) {
+            for (int T = par; T < NS - 1 && t0 + T < t1; T += 2) {
+                cur_init(gc, t0 + T);
+                row_entries(gc, gt, pend);
+                gather_rows(gc, gt, pend);
+            }
+            if (t0 + par + NS - 1 < t1) {
+                cur_init(gc, t0 + par + NS - 1);
+                row_entries(gc, gt, pend);
+            } else {
+                gc.tau = t1;
+            }
+        }
         for (int i = 0; ct < t1; ++i) {
             const bool seg_start = cb != seg_b;
             if (seg_start) {
@@ -639,6 +653,12 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                 tc_wait_st();
                 tc_fence_before();
                 mbar_arrive(BAR(BAR_P_FULL + par));
+                if (PS == 1 && gc.tau < t1) {
+                    gather_rows(gc, gt, pend);
+                    cur_next(gc);
+                    cur_next(gc);
+                    row_entries(gc, gt, pend);
+                }
             }
 
             if (seg_end) {
@@ -691,6 +711,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             if (seg_end)
                 while (cb < B - 1 && ct >= tpre[cb + 1]) ++cb;
         }
+        cp_async_wait<0>();  // every gather this thread issued has landed before the CTA leaves
     }
 
     // ---- teardown ----
