@@ -19,12 +19,13 @@
 // the half of its own KV head.
 //
 // Data flow per tile (all in one CTA per SM):
-//   loader warps 8-11 raw E4M3 rows into an NS-stage ring (page size 1:
-//                     cp.async gathers, as decode_kernel; page size 64: one
-//                     TMA tile load per page for K and one for V), then
-//                     E4M3 -> fp16 into a 128-byte-swizzled tile (K and V,
-//                     double-buffered); at a request's first tile they also
-//                     write its A operand into tensor memory.
+//   loader warps 8-11 wait for a tile's raw E4M3 rows in an NS-stage ring
+//                     (page size 1: gathered by the softmax warps, below; page
+//                     size 64: one TMA tile load per page for K and one for
+//                     V, issued here), then E4M3 -> fp16 into 128-byte-
+//                     swizzled tiles (K and V, NF buffers); at a request's
+//                     first tile they also write its A operand into tensor
+//                     memory.
 //   MMA warp 12       S(i) = A . K(i)^T into tensor memory (double-buffered),
 //                     then O += P(i-1) . V(i-1) with P read from tensor memory.
 //   softmax warps 0-7 two threads per row (warps w and w + 4 share the
@@ -37,7 +38,10 @@
 //                     two work on consecutive tiles at the same time.  At a
 //                     request's last tile they merge (m, l) through shared
 //                     memory and each writes half the dims of a0 O_0 + a1 O_1
-//                     to the partial.
+//                     to the partial.  With page size 1 each parity group also
+//                     issues the cp.async gathers of tile i + NS - 1 once it
+//                     has taken tile i (more warps issuing gathers raise the
+//                     rate at which random rows arrive).
 // Synchronisation by mbarriers; every wait is bounded (an expired wait sets
 // the step's error word and the CTA winds down, waits for its MMAs and frees
 // its tensor memory).
@@ -538,6 +542,14 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                 gc.tau = t1;
             }
         }
+        // the position of this row's token in an item, requested one item ahead
+        // (a global load at each item's first tile would sit on the path)
+        auto load_pos = [&](int b) {
+            const ItemRef it = item_ref<MULTI>(p, b);
+            return j < it.len ? p.positions[static_cast<size_t>(it.t0) + j] : int64_t{-1};
+        };
+        int pf_b = cb;
+        int64_t pf_pos = load_pos(cb);
         for (int i = 0; ct < t1; ++i) {
             const bool seg_start = cb != seg_b;
             if (seg_start) {
@@ -548,8 +560,13 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                 l_run = 0.f;
                 const ItemRef it = item_ref<MULTI>(p, cb);
                 seg_len = it.len;
+                const int64_t pos64 = pf_b == cb ? pf_pos : load_pos(cb);
+                if (seg_t1 < t1) {
+                    pf_b = cb + 1;
+                    pf_pos = load_pos(cb + 1);
+                }
                 if (j < it.len) {
-                    const int pos = static_cast<int>(p.positions[static_cast<size_t>(it.t0) + j]);
+                    const int pos = static_cast<int>(pos64);
                     hi_j = pos;
                     lo_j = p.window > 0 ? max(0, pos - p.window + 1) : 0;
                 } else {
