@@ -190,10 +190,6 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
         }
         return lo;
     };
-    auto advance = [&](int& tau, int& b) {
-        ++tau;
-        while (b < B - 1 && tau >= tpre[b + 1]) ++b;
-    };
     auto tile_k0 = [&](int tau, int b) { return (rlo[b] / TK + (tau - tpre[b])) * TK; };
     const float C2 = __ldg(p.k_scale) * 0.125f * 1.4426950408889634f;  // raw score -> log2 units
 
@@ -384,13 +380,21 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                 cp_async_commit();
             }
         }
-        int seg_b = -1, nseg = 0;
+        int seg_b = -1, nseg = 0, seg_i0 = 0;  // current item, items begun, its first tile
         const int n_tiles = t1 - t0;
         int i = 0;
         for (; i < n_tiles; ++i) {
             if (PS == 64) cp_async_wait<NS - 2>();  // the page indices NS - 1 tiles ahead
             const int cb = cc.b;
             const bool seg_start = cb != seg_b;
+            // A new item's A operand is written before the waits below (its q
+            // load then overlaps them) when its buffer is known to be free: the
+            // first two items' buffers are fresh; else the buffer's last reader,
+            // the S MMA of the previous item's predecessor's last tile (<= i - 3
+            // when the previous item had two tiles or more), is done once PV(i - 4)
+            // is, which the wait of tile i - 1 saw.
+            const bool early_q = seg_start && (nseg < 2 || (seg_i0 <= i - 2 && i >= NF + 1));
+            if (early_q) write_q(cb, (nseg & 1) ? TM_Q1 : TM_Q);
             // tile i's raw stage filled (page loads, or the softmax warps' gathers)
             bool bad = !wait_bounded(BAR(BAR_RAW + i % NS), (i / NS) & 1, abort_flag);
             // buffers i % NF are free once PV(i - NF) is done, which also means every
@@ -404,8 +408,9 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             // stage may be refilled
             if (bar_red_or(1, LOADERS, bad)) break;
             if (seg_start) {
-                write_q(cb, (nseg & 1) ? TM_Q1 : TM_Q);
+                if (!early_q) write_q(cb, (nseg & 1) ? TM_Q1 : TM_Q);
                 seg_b = cb;
+                seg_i0 = i;
                 ++nseg;
             }
             convert(i % NS, i % NF, cc.k0, cc.lo, cc.hi);
@@ -461,6 +466,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             return true;
         };
         int ct = t0, cb = find_req(t0);
+        int cb_end = tpre[cb + 1];             // first tile past item cb (kept in a register)
         int seg_b = -1, seg = -1, seg_i0 = 0;  // current request, its count and first tile here
         int prev_pos = 0;
         int prev_seg = -1;
@@ -495,7 +501,10 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
             }
             prev_pos = i - seg_i0;
             prev_seg = seg;
-            advance(ct, cb);
+            if (++ct >= cb_end && ct < t1) {
+                while (cb < B - 1 && ct >= tpre[cb + 1]) ++cb;
+                cb_end = tpre[cb + 1];
+            }
         }
         if (ok && i > 0) issue_pv(i - 1, prev_pos, prev_seg);
         // every MMA this warp issued is done before the tensor memory is freed
