@@ -48,9 +48,9 @@ FALLBACK_TC_TFLOPS = 1590.0  # dense bf16/fp16 burst
 # kernel on a workload, from the ncu captures summarised in profiles/, keyed by
 # the hash of that kernel's sources when the counters were taken (null once the
 # sources change).
-TRAFFIC = {("decode32_full", "a80b76dba19c6946"): 474212096,
-           ("verify16_full", "a154510131ded95a"): 336915200,
-           ("prefill1_full", "f178d2499de4754f"): 22619648}
+TRAFFIC = {("decode32_full", "834f05e301e35d17"): 474125824,
+           ("verify16_full", "923d4135dc10c8e0"): 337029888,
+           ("prefill1_full", "858fcaf6f8a660ac"): 22620416}
 
 # Sources of the step's main kernel: decode_kernel for single-token steps,
 # verify_tc_kernel for verify blocks, prefill_tc_kernel for longer blocks (the
