@@ -88,7 +88,7 @@ constexpr int BAR_S_FULL = 6;     // [2] S of the tile in tensor memory         
 constexpr int BAR_P_FULL = 8;     // [2] P of the tile in tensor memory          (128 softmax arrivals)
 constexpr int BAR_O_FREE = 10;    // O read out at a request's last tile         (256 softmax arrivals)
 constexpr int BAR_MMA_DONE = 11;  // teardown: all MMAs done                     (MMA commit)
-constexpr int BAR_PAIR = 12;      // [4] softmax pair qd posted its halves' (max, sum) at a request's end (64)
+constexpr int BAR_PAIR = 12;      // [4] softmax pair qd posted both parities' (max, sum) at a request's end (64)
 constexpr int BAR_RAW = 16;       // [NS] the tile's K and V rows landed (TMA bytes, or 128 gathers' arrivals)
 constexpr int NBARS = 16;         // + NS
 
@@ -99,7 +99,7 @@ struct Cfg {
     static constexpr int IDX_SLOTS = 2 * NS;
     static constexpr size_t IDX_BYTES = static_cast<size_t>(IDX_SLOTS) * TK * 4;
     static constexpr size_t CTRL_BYTES = 256;  // barriers, tensor-memory base, abort flag
-    // softmax pairs at a request's end: [2 (request parity)][max, sum][2 halves][128 rows]
+    // softmax pairs at a request's end: [2 (request parity)][max, sum][2 (tile parity)][128 rows]
     static constexpr size_t RED_BYTES = 2 * 2 * 2 * 128 * 4;
     // + 1024 so the swizzled tiles can start on a 1024-byte boundary
     static size_t smem_bytes(int B) {
@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
     uint8_t* ctrl = reinterpret_cast<uint8_t*>(idx_smem) + C::IDX_BYTES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + (NBARS + NS) * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + (NBARS + NS) * 8 + 4);
-    float* red = reinterpret_cast<float*>(ctrl + C::CTRL_BYTES);  // halves' (max, sum) at a request's end
+    float* red = reinterpret_cast<float*>(ctrl + C::CTRL_BYTES);  // the pairs' (max, sum) at a request's end
     int* tpre = reinterpret_cast<int*>(ctrl + C::CTRL_BYTES + C::RED_BYTES);
     int* rlo = tpre + p.NB + 1;
     int* rhi = rlo + p.NB;
@@ -652,7 +652,7 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
                     }
                 }
                 if (bad) break;
-                // pass 2: P = 2^(s - m) for each 32-key half, written as fp16 over the
+                // pass 2: P = 2^(s - m) for each 32-key chunk, written as fp16 over the
                 // S columns already read (keys 32 ch .. -> columns 16 ch ..)
                 const float mc = m_run == -INFINITY ? 0.f : m_run * C2;
                 float l4[4] = {0.f, 0.f, 0.f, 0.f};
