@@ -234,6 +234,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
     d |= static_cast<uint64_t>(2u) << 61;            // 128-byte swizzle
     return d;
 }
+// The same for an MN-major operand two 64-element atoms wide along N: the
+// second atom (N 64..127) starts `lbo` bytes after the first (the leading
+// byte offset of the MN-major swizzled layout; 8-row groups along K stay
+// 1024 bytes apart).
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn2(uint32_t addr, uint32_t lbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;  // leading byte offset: next N atom
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;            // stride byte offset: next 8-row group
+    d |= static_cast<uint64_t>(1u) << 46;                    // descriptor version (sm_100)
+    d |= static_cast<uint64_t>(2u) << 61;                    // 128-byte swizzle
+    return d;
+}
 
 // mbarrier arrive that also expects `bytes` of asynchronous (TMA) transactions.
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {

@@ -444,24 +444,22 @@ __global__ void __launch_bounds__(vtc::THREADS, 1)
         // The warp runs the control flow together so that every operand of the
         // MMA and commit instructions is warp-uniform.
         constexpr uint32_t ID_S = idesc_f16_f32(128, TK, 0);  // S: A . K^T, K-major B
-        constexpr uint32_t ID_O = idesc_f16_f32(128, 64, 1);  // O: P . V, MN-major B
+        constexpr uint32_t ID_O = idesc_f16_f32(128, 128, 1);  // O: P . V, MN-major B, both heads' dims
         const uint32_t f16_base = smem_addr(f16);
-        // O_(k & 1) += P(k) . V(k), per KV head's dims (N = 64); `pos` is k's
-        // index within its request (the first tile of each parity overwrites).
+        // O_(k & 1) += P(k) . V(k) over both KV heads' dims at once (N = 128:
+        // the two heads' V tiles are the MN-major operand's two 64-wide atoms,
+        // HALF_TILE bytes apart; each row keeps its own head's half); `pos` is
+        // k's index within its request (the first tile of each parity overwrites).
         auto issue_pv = [&](int k, int pos, int seg) {
             if (!wait_warp(BAR(BAR_P_FULL + (k & 1)), (k >> 1) & 1, abort_flag)) return false;
             if (pos == 0 && seg >= 1 && !wait_warp(BAR(BAR_O_FREE), (seg - 1) & 1, abort_flag)) return false;
             tc_fence_after();
-            const uint32_t vbuf = f16_base + (k % NF) * F16_BUF + F16_TILE;
+            const uint32_t vb = f16_base + (k % NF) * F16_BUF + F16_TILE;
             const uint32_t pa = tmem + TM_S + 64u * (k & 1);
             const uint32_t av[4] = {pa, pa + 8u, pa + 16u, pa + 24u};
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t vb = vbuf + h * HALF_TILE;
-                const uint64_t bd[4] = {smem_desc_sw128(vb), smem_desc_sw128(vb + 2048),
-                                        smem_desc_sw128(vb + 4096), smem_desc_sw128(vb + 6144)};
-                tc_mma_ts4(tmem + TM_O + TM_O_HALF * (k & 1) + 64u * h, av, bd, ID_O, pos >= 2 ? 1u : 0u);
-            }
+            const uint64_t bd[4] = {smem_desc_sw128_mn2(vb, HALF_TILE), smem_desc_sw128_mn2(vb + 2048, HALF_TILE),
+                                    smem_desc_sw128_mn2(vb + 4096, HALF_TILE), smem_desc_sw128_mn2(vb + 6144, HALF_TILE)};
+            tc_mma_ts4(tmem + TM_O + TM_O_HALF * (k & 1), av, bd, ID_O, pos >= 2 ? 1u : 0u);
             tc_commit(BAR(BAR_KV_FREE + k % NF));
             return true;
         };
