@@ -49,7 +49,7 @@ FALLBACK_TC_TFLOPS = 1590.0  # dense bf16/fp16 burst
 # the hash of that kernel's sources when the counters were taken (null once the
 # sources change).
 TRAFFIC = {("decode32_full", "834f05e301e35d17"): 474125824,
-           ("verify16_full", "8463297c3c11a218"): 337029888,
+           ("verify16_full", "2af58576cdd3f211"): 336986624,
            ("prefill1_full", "858fcaf6f8a660ac"): 22620416}
 
 # Sources of the step's main kernel: decode_kernel for single-token steps,
