@@ -50,7 +50,7 @@ FALLBACK_TC_TFLOPS = 1590.0  # dense bf16/fp16 burst
 # sources change).
 TRAFFIC = {("decode32_full", "834f05e301e35d17"): 474125824,
            ("verify16_full", "2af58576cdd3f211"): 336986624,
-           ("prefill1_full", "858fcaf6f8a660ac"): 22620416}
+           ("prefill1_full", "2973f5b1d8caa22c"): 22620160}
 
 # Sources of the step's main kernel: decode_kernel for single-token steps,
 # verify_tc_kernel for verify blocks, prefill_tc_kernel for longer blocks (the
