@@ -41,6 +41,9 @@ SMALL = [
     S("ragged_pages_v8", B=4, L=8, seq_lens=[56, 57, 63, 120], page_size=64, seed=115),
     S("L3_block", B=3, L=3, seq_lens=[100, 1000, 64], seed=116),
     S("many_requests", B=40, ctx_range=(0, 3000), seed=117),
+    # more list items than the verify kernel's deeper ring leaves table room
+    # for: its shallow configuration (three raw stages)
+    S("many_items_v8_shallow_ring", B=1800, L=8, ctx_range=(0, 100), seed=162),
     S("many_requests_v8_sliding", B=40, L=8, ctx_range=(0, 5000), window=256, use_rope=True,
       seed=118),
     S("gate_std2_s64", B=2, L=8, ctx=1500, page_size=64, kv_scale=1 / 64, gate_std=2.0, seed=119),
@@ -81,6 +84,8 @@ SMALL_DP = [
     S("dp_b2_decode", B=2, seq_lens=[700, 4000], page_size=64, seed=146, **DP),
     # 512 requests x 8 groups = 4096 list items, the most one call takes
     S("dp_b512_most_items", B=512, ctx_range=(0, 40), seed=144, **DP),
+    # 256 requests x 8 groups = 2048 verify items: the shallow ring at page size 64
+    S("dp_b256_v8_shallow_ring", B=256, L=8, ctx_range=(0, 40), page_size=64, seed=161, **DP),
 ]
 
 
